@@ -1,0 +1,329 @@
+"""Benchmark of the VC-Attention forward (V-Smooth prep + ExpCast-FP8 attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mid_32k_d128] [--no-cpu-baseline]
+
+One step is one pass of the whole hot path over the workload: V-Smooth prep
+(k-means, regroup, K/V quantisation) and the attention forward, on inputs
+resident in HBM.  The metric is attention TFLOPS, 4*B*H*N^2*d over the step
+time.  Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun, one process per GPU): every (b, h) problem is
+independent, so each rank runs its own copy of the workload with no data-path
+collective (weak scaling); the step time is the max over ranks.
+
+--impl reference times the CPU oracle (the only other implementation of the
+method there is) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_fp8_attention_smooth_b200 import synth  # noqa: E402
+
+BETA = 64
+METRIC = "attn fwd TFLOPS (4*B*H*N^2*d/t) at N=32K, d=128; % of B200 FP8 tensor peak"
+FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor ratio on B200
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_sample(w, rows: int, threads: int):
+    """Time the oracle (prep of one head + replay of `rows` query rows over all
+    keys) and extrapolate to the per-head attention throughput in TFLOPS."""
+    import oracle
+
+    q, k, v = (synth.head_bits(w, t, 0, 0) for t in "qkv")
+    sel = np.linspace(0, w.N - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    prep = oracle.prep_head(k, v, C=w.C, iters=w.iters, bk=w.block)
+    t1 = time.perf_counter()
+    oracle.forward_head(q, k, v, sel, C=w.C, iters=w.iters, bk=w.block, beta=BETA, prep=prep, threads=threads)
+    t2 = time.perf_counter()
+    head_s = (t1 - t0) + (t2 - t1) * (w.N / rows)
+    head_flops = 4.0 * float(w.N) ** 2 * w.d
+    return dict(value=head_flops / head_s / 1e12, prep_s=t1 - t0, rows_s=t2 - t1, head_s=head_s)
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------- arms
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    cores = cpu_cores()
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(w, max(8, rows // 8), cores)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = oracle_sample(w, rows, cores)
+        vals.append(r["value"])
+        secs.append(r["head_s"])
+    value = statistics.median(vals)
+    sample = (f"head 0 of {w.name}: full k-means/regroup/quantise prep + replay of {rows} strided query rows "
+              f"over all {w.N} keys, extrapolated to the head's {w.N} rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(secs) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 emulation of e4m3",
+        "data": "synthetic", "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "C": w.C, "kmeans_iters": w.iters,
+            "block": w.block, "beta": BETA, "v_smooth": True,
+            "l2": f"inputs {3 * w.B * w.H * w.N * w.d * 2 / 1e9:.2f} GB per step > 126 MB L2 (no flush needed)"}
+
+
+def launches_per_step(p) -> int:
+    prep = (1 + 3 * p.iters + 2 * (p.iters - 1) + 2) if p.smooth else 4
+    return prep + 2
+
+
+def run_ours(args, w):
+    import bit_fp8_attention_smooth_b200 as vc
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    vc.lib()
+    params = vc.Params.for_workload(w, beta=BETA)
+    shape = (w.B, w.H, w.N, w.d)
+
+    # inputs resident in HBM (pinned host copies kept for the end-to-end leg)
+    host = {t: synth.tensor_bf16(w, t, out=torch.empty(shape, dtype=torch.bfloat16).pin_memory()) for t in "qkv"}
+    qd, kd, vd = (host[t].to(dev) for t in "qkv")
+    out = torch.empty_like(qd)
+    prep = vc.alloc_prep(shape, params, dev)
+    ws = vc.alloc_workspace(shape, params, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        vc.smooth_prepare(kd, vd, params, prep=prep, workspace=ws)
+        if evs is not None:
+            evs[1].record(stream)
+        vc.attn_fwd(qd, prep, params, out=out, workspace=ws)
+        if evs is not None:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    vc.check(ws)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    vc.check(ws)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    prep_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    attn_ms = max_over_ranks(attn_ms, dev)
+    prep_ms = max_over_ranks(prep_ms, dev)
+    ms_per_step = total_ms / args.steps
+    flops = w.attn_flops
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+
+    # end to end through the public API from pinned host buffers
+    e2e = vc.HostAttention(shape, params, dev)
+    o_host = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    for _ in range(max(1, args.warmup // 2)):
+        e2e(host["q"], host["k"], host["v"], o_host)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e(host["q"], host["k"], host["v"], o_host)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    vc.check(e2e.ws)
+
+    if rank == 0:
+        peaks = load_peaks()
+        fp8_peak = peaks["bf16_sustained"] * FP8_PER_BF16
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic", "config": config_of(w),
+            "attn_ms": attn_ms, "prep_ms": prep_ms, "attn_tflops": attn_tflops,
+            "frac_of_nominal_fp8_4500": value / 4500.0, "attn_frac_of_nominal_fp8_4500": attn_tflops / 4500.0,
+            "roofline": {
+                "bound": "tensor", "kernel": "vc_attn_fwd (Q quantise + vc_attn_kernel)",
+                "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
+                "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16)",
+                "traffic": None,
+            },
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": e2e.h2d_bytes, "d2h_bytes_per_step": e2e.d2h_bytes},
+            "gpu_launches": launches_per_step(params) * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            cores = cpu_cores()
+            r = oracle_sample(w, args.ref_rows, cores)
+            line["cpu_baseline"] = {
+                "value": r["value"], "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                "sample": (f"head 0: full prep ({r['prep_s']:.1f} s) + {args.ref_rows} strided query rows over all "
+                           f"keys ({r['rows_s']:.1f} s), extrapolated to the head's {w.N} rows"),
+            }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mid_32k_d128", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

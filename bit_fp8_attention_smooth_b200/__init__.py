@@ -1,0 +1,253 @@
+"""VC-Attention (V-Smooth + ExpCast-FP8) forward for NVIDIA B200, Python binding.
+
+A thin ctypes layer over the C ABI in include/vc_attention.h (libvcattn.so,
+built in-tree by ``python -m bit_fp8_attention_smooth_b200.build``).  It only
+marshals arguments: torch supplies device memory and streams, every step of
+the computation runs in the library's CUDA kernels.  There is no CPU fallback:
+if the library is missing or the device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Dict, Optional
+
+import torch
+
+from . import synth  # noqa: F401  (seeded workloads, no method arithmetic)
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvcattn.so")
+
+VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_CUDA, VC_ERR_DEVICE_TIMEOUT, VC_ERR_WORKSPACE = range(6)
+
+
+class VcError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("d", ctypes.c_int32)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("C", ctypes.c_int32), ("iters", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("beta", ctypes.c_int32), ("smooth", ctypes.c_int32), ("resid_fmt", ctypes.c_int32),
+                ("wait_limit_ns", ctypes.c_int64)]
+
+
+class _Prep(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("perm", "labels", "k_fp8", "k_scale", "vt_fp8", "v_mean", "v_scale")]
+
+
+PREP_FIELDS = ("perm", "labels", "k_fp8", "k_scale", "vt_fp8", "v_mean", "v_scale")
+
+_lib = None
+
+
+def lib():
+    """Load libvcattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m bit_fp8_attention_smooth_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64
+        PS, PP, PR = ctypes.POINTER(_Shape), ctypes.POINTER(_Params), ctypes.POINTER(_Prep)
+        sig = {
+            "vc_abi_version": (ctypes.c_int, []),
+            "vc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "vc_prep_buffer_bytes": (ctypes.c_int, [PS, PP, ctypes.POINTER(S)]),
+            "vc_workspace_bytes": (ctypes.c_int, [PS, PP, ctypes.POINTER(S)]),
+            "vc_smooth_prepare": (ctypes.c_int, [P, P, PS, PP, PR, P, S, P]),
+            "vc_attn_fwd": (ctypes.c_int, [P, PR, PS, PP, P, P, S, P]),
+            "vc_attention": (ctypes.c_int, [P, P, P, PS, PP, PR, P, P, S, P]),
+            "vc_check": (ctypes.c_int, [P, P]),
+            "vc_e4m3_encode": (ctypes.c_int, [P, P, i64, P]),
+            "vc_expcast_bytes": (ctypes.c_int, [P, P, P, P, i64, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().vc_status_string(status).decode()
+    except Exception:  # library not loadable: still give a readable message
+        return f"status {status}"
+
+
+def _ok(status: int, what: str):
+    if status != VC_OK:
+        raise VcError(status, what)
+
+
+@dataclasses.dataclass
+class Params:
+    """V-Smooth / ExpCast settings (see vc_params in include/vc_attention.h)."""
+
+    C: int = 64
+    iters: int = 10
+    block: int = 128
+    beta: int = 64
+    smooth: bool = True
+    resid_fmt: int = 0
+    wait_limit_ns: int = 0
+
+    def c(self) -> _Params:
+        return _Params(self.C, self.iters, self.block, self.beta, int(self.smooth), self.resid_fmt, self.wait_limit_ns)
+
+    @classmethod
+    def for_workload(cls, w, **kw) -> "Params":
+        return cls(C=w.C, iters=w.iters, block=w.block, **kw)
+
+
+def _shape(t: torch.Tensor) -> _Shape:
+    if t.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    B, H, N, d = t.shape
+    return _Shape(B, H, N, d)
+
+
+def _check_input(t: torch.Tensor, name: str):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def prep_sizes(shape, params: Params):
+    sh = _Shape(*shape) if not isinstance(shape, _Shape) else shape
+    out = (ctypes.c_size_t * 7)()
+    _ok(lib().vc_prep_buffer_bytes(ctypes.byref(sh), ctypes.byref(params.c()), out), "vc_prep_buffer_bytes")
+    return list(out)
+
+
+def workspace_bytes(shape, params: Params) -> int:
+    sh = _Shape(*shape) if not isinstance(shape, _Shape) else shape
+    n = ctypes.c_size_t()
+    _ok(lib().vc_workspace_bytes(ctypes.byref(sh), ctypes.byref(params.c()), ctypes.byref(n)), "vc_workspace_bytes")
+    return n.value
+
+
+def alloc_workspace(shape, params: Params, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace (the status word must start at 0)."""
+    return torch.zeros(workspace_bytes(shape, params), dtype=torch.uint8, device=device)
+
+
+def alloc_prep(shape, params: Params, device="cuda") -> Dict[str, torch.Tensor]:
+    """Caller-owned prep buffers with their logical shapes and dtypes."""
+    B, H, N, d = shape
+    T = -(-N // params.block)
+    Tp = T * params.block
+    return {
+        "perm": torch.empty((B, H, N), dtype=torch.int32, device=device),
+        "labels": torch.empty((B, H, N), dtype=torch.int32, device=device),
+        "k_fp8": torch.empty((B, H, Tp, d), dtype=torch.uint8, device=device),
+        "k_scale": torch.empty((B, H, T), dtype=torch.float32, device=device),
+        "vt_fp8": torch.empty((B, H, d, Tp), dtype=torch.uint8, device=device),
+        "v_mean": torch.empty((B, H, T, d), dtype=torch.float32, device=device),
+        "v_scale": torch.empty((B, H, d), dtype=torch.float32, device=device),
+    }
+
+
+def _prep_struct(prep: Dict[str, torch.Tensor]) -> _Prep:
+    vals = []
+    for n in PREP_FIELDS:
+        t = prep.get(n)
+        vals.append(None if t is None else t.data_ptr())
+    return _Prep(*vals)
+
+
+def smooth_prepare(K: torch.Tensor, V: torch.Tensor, params: Params, prep=None, workspace=None, stream=None):
+    """V-Smooth prep; returns the prep buffers (k-means labels included)."""
+    _check_input(K, "K")
+    _check_input(V, "V")
+    shape = tuple(K.shape)
+    prep = alloc_prep(shape, params, K.device) if prep is None else prep
+    ws = alloc_workspace(shape, params, K.device) if workspace is None else workspace
+    st = lib().vc_smooth_prepare(K.data_ptr(), V.data_ptr(), ctypes.byref(_shape(K)), ctypes.byref(params.c()),
+                                 ctypes.byref(_prep_struct(prep)), ws.data_ptr(), ws.numel(), _stream(stream))
+    _ok(st, "vc_smooth_prepare")
+    return prep
+
+
+def attn_fwd(Q: torch.Tensor, prep, params: Params, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """ExpCast-FP8 attention over prepped K/V; returns O (bf16, Q's layout)."""
+    _check_input(Q, "Q")
+    shape = tuple(Q.shape)
+    out = torch.empty_like(Q) if out is None else out
+    ws = alloc_workspace(shape, params, Q.device) if workspace is None else workspace
+    st = lib().vc_attn_fwd(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
+                           ctypes.byref(params.c()), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    _ok(st, "vc_attn_fwd")
+    return out
+
+
+def attention(Q, K, V, params: Params, out=None, prep=None, workspace=None, stream=None) -> torch.Tensor:
+    """The drop-in call: V-Smooth prep then ExpCast-FP8 attention."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _check_input(t, n)
+    shape = tuple(Q.shape)
+    out = torch.empty_like(Q) if out is None else out
+    prep = alloc_prep(shape, params, Q.device) if prep is None else prep
+    ws = alloc_workspace(shape, params, Q.device) if workspace is None else workspace
+    st = lib().vc_attention(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(_shape(Q)),
+                            ctypes.byref(params.c()), ctypes.byref(_prep_struct(prep)), out.data_ptr(),
+                            ws.data_ptr(), ws.numel(), _stream(stream))
+    _ok(st, "vc_attention")
+    return out
+
+
+def check(workspace: torch.Tensor, stream=None) -> None:
+    """Synchronise and raise VcError if a kernel recorded a device-side timeout."""
+    _ok(lib().vc_check(workspace.data_ptr(), _stream(stream)), "vc_check")
+
+
+def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
+    assert x.dtype == torch.float32 and x.is_cuda and x.is_contiguous()
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _ok(lib().vc_e4m3_encode(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)), "vc_e4m3_encode")
+    return out
+
+
+def expcast_bytes(A: torch.Tensor, s: torch.Tensor, cb: torch.Tensor, stream=None) -> torch.Tensor:
+    for t in (A, s, cb):
+        assert t.dtype == torch.float32 and t.is_cuda and t.is_contiguous() and t.shape == A.shape
+    out = torch.empty(A.shape, dtype=torch.uint8, device=A.device)
+    _ok(lib().vc_expcast_bytes(A.data_ptr(), s.data_ptr(), cb.data_ptr(), out.data_ptr(), A.numel(), _stream(stream)),
+        "vc_expcast_bytes")
+    return out
+
+
+class HostAttention:
+    """End-to-end call from pinned host buffers: H2D copies, the CUDA path, D2H
+    copy of O, all on one stream (device buffers are allocated once)."""
+
+    def __init__(self, shape, params: Params, device="cuda"):
+        self.shape, self.params = tuple(shape), params
+        self.q = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.k = torch.empty_like(self.q)
+        self.v = torch.empty_like(self.q)
+        self.o = torch.empty_like(self.q)
+        self.prep = alloc_prep(self.shape, params, device)
+        self.ws = alloc_workspace(self.shape, params, device)
+        self.h2d_bytes = 3 * self.q.numel() * 2
+        self.d2h_bytes = self.o.numel() * 2
+
+    def __call__(self, q_host, k_host, v_host, o_host, stream=None):
+        self.q.copy_(q_host, non_blocking=True)
+        self.k.copy_(k_host, non_blocking=True)
+        self.v.copy_(v_host, non_blocking=True)
+        attention(self.q, self.k, self.v, self.params, out=self.o, prep=self.prep, workspace=self.ws, stream=stream)
+        o_host.copy_(self.o, non_blocking=True)
+        return o_host

@@ -1,0 +1,59 @@
+// vc_launch.cuh -- argument blocks and launchers shared by the entry points
+// (vc_api.cu) and the kernels (vc_attn.cu, vc_prep.cu).
+#pragma once
+
+#include "vc_device.cuh"
+
+namespace vc {
+
+struct AttnArgs {
+    const float* sq;       // [BH, N] per-token Q scale
+    const float* k_scale;  // [BH, T]
+    const float* v_mean;   // [BH, T, D]
+    const float* v_scale;  // [BH, D]
+    __nv_bfloat16* out;    // [BH, N, D]
+    int N, T;
+    float kappa;  // fp32(8 * log2(e) / sqrt(D))
+    int beta;
+    DevCtl ctl;
+};
+
+struct KmState {  // per (b, h), 16 bytes of workspace
+    int changed;
+    int done;
+    int pad0, pad1;
+};
+
+struct PrepLaunch {
+    const __nv_bfloat16* K;
+    const __nv_bfloat16* V;
+    int BH, N, D, C, iters, BK, smooth;
+    // outputs
+    int32_t* perm;
+    uint8_t* k_fp8;
+    float* k_scale;
+    uint8_t* vt_fp8;
+    float* v_mean;
+    float* v_scale;
+    // workspace
+    int32_t* labels;
+    float* cent_t;
+    double* sums;
+    int32_t* cstart;
+    int32_t* ccount;
+    int32_t* hist;
+    int32_t* offs;
+    KmState* state;
+    uint32_t* vamax;
+};
+
+cudaError_t launch_attn(int D, int BK, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnArgs& a, int BH, cudaStream_t stream);
+cudaError_t launch_prep(const PrepLaunch& p, cudaStream_t s);
+cudaError_t launch_quant_q(const __nv_bfloat16* Q, uint8_t* q_fp8, float* sq, int64_t tokens, int D,
+                           cudaStream_t s);
+cudaError_t launch_e4m3_encode(const float* x, uint8_t* out, int64_t n, cudaStream_t s);
+cudaError_t launch_expcast(const float* A, const float* s, const float* cb, uint8_t* out, int64_t n,
+                           cudaStream_t stream);
+
+}  // namespace vc

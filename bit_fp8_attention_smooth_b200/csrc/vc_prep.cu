@@ -1,0 +1,500 @@
+// vc_prep.cu -- V-Smooth prep and Q quantisation on sm_100a.
+//
+// V-Smooth (chooseai.io news 7051, section "核心方法之一：V-Smooth 把 value 的
+// 离群值收拢"; zerohour.day key facts): a lightweight k-means puts similar value
+// tokens into the same hardware block; the block mean is subtracted and kept
+// in high precision; the residual is quantised to E4M3 with per-channel scales.
+// K moves with V so every (k_j, v_j) pair stays together.
+//
+// Kernels, per call, for all (b, h) at once:
+//   km_init                   strided centroid init c_k = v[floor(k N / C)]
+//   per pass: km_assign       labels = argmin_k |v - c_k|^2 (fp32, ties -> lowest k),
+//                             per-(cluster, 128-token block) histogram, change count
+//             km_scan         exclusive scan -> stable positions; a head whose labels
+//                             did not change is final (its later passes would repeat)
+//             km_scatter      perm[position] = token (stable within a cluster)
+//             km_update       fp64 member sums over each cluster's contiguous range
+//             km_finalize     c_k = sum / count (empty clusters keep c_k)
+//   prep_kv_block             per block: K amax scale + E4M3 K, V block mean (fp64 sum),
+//                             residual channel amax
+//   prep_v_quant              per-channel residual scale, E4M3 residual, transposed
+//   quant_q                   per-token E4M3 Q (used by the attention call)
+#include <math.h>
+
+#include "vc_launch.cuh"
+
+namespace vc {
+
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// ------------------------------------------------------------------ k-means
+// cent_t: centroids channel-major [BH, D, C] fp32.
+__global__ void km_init(const __nv_bfloat16* __restrict__ V, float* __restrict__ cent_t, double* __restrict__ sums,
+                        KmState* __restrict__ state, uint32_t* __restrict__ vamax, int N, int C, int D) {
+    const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+    if (c >= D) return;
+    const int64_t src = ((int64_t)k * N) / C;
+    cent_t[((size_t)bh * D + c) * C + k] = bf2f(V[((size_t)bh * N + src) * D + c]);
+    sums[((size_t)bh * C + k) * D + c] = 0.0;
+    if (k == 0) {
+        vamax[(size_t)bh * D + c] = 0u;
+        if (c == 0) state[bh] = KmState{0, 0, 0, 0};
+    }
+}
+
+constexpr int KM_TOK = 128;  // tokens per assign block
+
+template <int D>
+__global__ void __launch_bounds__(256) km_assign(const __nv_bfloat16* __restrict__ V, const float* __restrict__ cent_t,
+                                                 int32_t* __restrict__ labels, int32_t* __restrict__ hist,
+                                                 KmState* __restrict__ state, int N, int C, int it) {
+    extern __shared__ float sm[];
+    const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x;
+    if (state[bh].done) return;
+    const int Cpad = (C + 63) & ~63;
+    float* cent_s = sm;                      // [D][Cpad]
+    float* v_s = cent_s + D * Cpad;          // [D][KM_TOK]
+    float* cnorm = v_s + D * KM_TOK;         // [Cpad]
+    int* hist_s = reinterpret_cast<int*>(cnorm + Cpad);  // [C]
+    const int tid = threadIdx.x;
+    const int n0 = blk * KM_TOK;
+    const int valid = min(KM_TOK, N - n0);
+
+    for (int i = tid; i < D * Cpad; i += 256) {
+        const int c = i / Cpad, k = i % Cpad;
+        cent_s[i] = k < C ? cent_t[((size_t)bh * D + c) * C + k] : 0.0f;
+    }
+    for (int i = tid; i < C; i += 256) hist_s[i] = 0;
+    for (int i = tid; i < KM_TOK * (D / 8); i += 256) {
+        const int r = i % KM_TOK, c8 = i / KM_TOK;
+        float f[8];
+        if (r < valid) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(V + ((size_t)bh * N + n0 + r) * D + 8 * c8);
+            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = bf2f(h[e]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v_s[(8 * c8 + e) * KM_TOK + r] = f[e];
+    }
+    __syncthreads();
+    for (int k = tid; k < Cpad; k += 256) {
+        float s = 0.0f;
+        for (int c = 0; c < D; ++c) s = fmaf(cent_s[c * Cpad + k], cent_s[c * Cpad + k], s);
+        cnorm[k] = s;
+    }
+    __syncthreads();
+
+    const int g = tid >> 3, h = tid & 7;  // tokens 4g..4g+3; centroids 8h..8h+7 of each 64-chunk
+    float best_d[4];
+    int best_k[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        best_d[i] = INFINITY;
+        best_k[i] = 0;
+    }
+    for (int cc = 0; cc < Cpad; cc += 64) {
+        float acc[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+#pragma unroll 4
+        for (int c = 0; c < D; ++c) {
+            const float4 vv = *reinterpret_cast<const float4*>(v_s + c * KM_TOK + 4 * g);
+            const float4 ca = *reinterpret_cast<const float4*>(cent_s + c * Cpad + cc + 8 * h);
+            const float4 cb = *reinterpret_cast<const float4*>(cent_s + c * Cpad + cc + 8 * h + 4);
+            const float v4[4] = {vv.x, vv.y, vv.z, vv.w};
+            const float c8[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(v4[i], c8[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int k = cc + 8 * h + j;
+            if (k < C) {
+                const float cn = cnorm[k];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float dist = cn - 2.0f * acc[i][j];
+                    if (dist < best_d[i]) {
+                        best_d[i] = dist;
+                        best_k[i] = k;
+                    }
+                }
+            }
+        }
+    }
+    // reduce over the 8 lanes sharing a token group (lowest index on ties)
+#pragma unroll
+    for (int m = 1; m < 8; m <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float od = __shfl_xor_sync(0xffffffffu, best_d[i], m);
+            const int ok = __shfl_xor_sync(0xffffffffu, best_k[i], m);
+            if (od < best_d[i] || (od == best_d[i] && ok < best_k[i])) {
+                best_d[i] = od;
+                best_k[i] = ok;
+            }
+        }
+    }
+    int changed = 0;
+    if (h == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = 4 * g + i;
+            if (r < valid) {
+                int32_t* lp = labels + (size_t)bh * N + n0 + r;
+                if (it == 0 || *lp != best_k[i]) ++changed;
+                *lp = best_k[i];
+                atomicAdd(&hist_s[best_k[i]], 1);
+            }
+        }
+    }
+    changed = __reduce_add_sync(0xffffffffu, changed);
+    if ((tid & 31) == 0 && changed) atomicAdd(&state[bh].changed, changed);
+    __syncthreads();
+    for (int k = tid; k < C; k += 256) hist[((size_t)bh * C + k) * nblk + blk] = hist_s[k];
+}
+
+// Exclusive scan of hist[bh] in (cluster, block) order -> offs; cluster ranges.
+__global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist, int32_t* __restrict__ offs,
+                                                int32_t* __restrict__ cstart, int32_t* __restrict__ ccount,
+                                                KmState* __restrict__ state, int N, int C, int nblk, int it) {
+    __shared__ int s_part[1024];
+    __shared__ int s_skip;
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    if (tid == 0) {
+        int skip = state[bh].done;
+        if (!skip && it > 0 && state[bh].changed == 0) {
+            state[bh].done = 1;  // labels repeat the previous pass: perm is final
+            skip = 1;
+        }
+        if (!skip) state[bh].changed = 0;
+        s_skip = skip;
+    }
+    __syncthreads();
+    if (s_skip) return;
+    const int64_t L = (int64_t)C * nblk;
+    const int64_t per = (L + 1023) / 1024;
+    const int64_t a = imin64(L, per * tid), b = imin64(L, a + per);
+    const int32_t* hh = hist + (size_t)bh * L;
+    int32_t* oo = offs + (size_t)bh * L;
+    int s = 0;
+    for (int64_t i = a; i < b; ++i) s += hh[i];
+    s_part[tid] = s;
+    __syncthreads();
+    for (int d = 1; d < 1024; d <<= 1) {
+        const int v = tid >= d ? s_part[tid - d] : 0;
+        __syncthreads();
+        s_part[tid] += v;
+        __syncthreads();
+    }
+    int run = s_part[tid] - s;  // exclusive prefix of this segment
+    for (int64_t i = a; i < b; ++i) {
+        oo[i] = run;
+        run += hh[i];
+    }
+    __syncthreads();
+    for (int k = tid; k < C; k += 1024) {
+        const int st = oo[(int64_t)k * nblk];
+        const int en = k + 1 < C ? oo[(int64_t)(k + 1) * nblk] : N;
+        cstart[(size_t)bh * C + k] = st;
+        ccount[(size_t)bh * C + k] = en - st;
+    }
+}
+
+__global__ void __launch_bounds__(KM_TOK) km_scatter(const int32_t* __restrict__ labels,
+                                                     const int32_t* __restrict__ offs, int32_t* __restrict__ perm,
+                                                     const KmState* __restrict__ state, int N, int C) {
+    __shared__ int lab_s[KM_TOK];
+    const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x, r = threadIdx.x;
+    if (state[bh].done) return;
+    const int j = blk * KM_TOK + r;
+    const int L = j < N ? labels[(size_t)bh * N + j] : -1;
+    lab_s[r] = L;
+    __syncthreads();
+    if (j >= N) return;
+    int rank = 0;
+    for (int q = 0; q < r; ++q) rank += (lab_s[q] == L);
+    perm[(size_t)bh * N + offs[((size_t)bh * C + L) * nblk + blk] + rank] = j;
+}
+
+constexpr int KM_SLICES = 8;
+
+template <int D>
+__global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ perm,
+                                                 const int32_t* __restrict__ cstart,
+                                                 const int32_t* __restrict__ ccount, double* __restrict__ sums,
+                                                 const KmState* __restrict__ state, int N, int C) {
+    const int k = blockIdx.x, sl = blockIdx.y, bh = blockIdx.z;
+    if (state[bh].done) return;
+    const int cnt = ccount[(size_t)bh * C + k];
+    if (cnt == 0) return;
+    const int st = cstart[(size_t)bh * C + k];
+    const int a = st + (int)(((int64_t)cnt * sl) / KM_SLICES);
+    const int b = st + (int)(((int64_t)cnt * (sl + 1)) / KM_SLICES);
+    constexpr int RG = 128 / D;
+    const int c = threadIdx.x % D, rg = threadIdx.x / D;
+    double acc = 0.0;
+    const int32_t* pp = perm + (size_t)bh * N;
+    const __nv_bfloat16* vb = V + (size_t)bh * N * D;
+    for (int i = a + rg; i < b; i += RG) acc += (double)bf2f(vb[(size_t)pp[i] * D + c]);
+    if (b > a) atomicAdd(&sums[((size_t)bh * C + k) * D + c], acc);
+}
+
+__global__ void km_finalize(float* __restrict__ cent_t, double* __restrict__ sums, const int32_t* __restrict__ ccount,
+                            const KmState* __restrict__ state, int C, int D) {
+    const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+    if (c >= D || state[bh].done) return;
+    const int cnt = ccount[(size_t)bh * C + k];
+    double* sp = &sums[((size_t)bh * C + k) * D + c];
+    if (cnt > 0) cent_t[((size_t)bh * D + c) * C + k] = (float)(*sp / (double)cnt);
+    *sp = 0.0;
+}
+
+// ------------------------------------------------------------------ block quantisation
+// One CTA per (block of BK regrouped tokens, head).  K: amax over the block,
+// inv = 448/amax, code = E4M3(k * inv), k_scale = amax/448.  V: block mean
+// (fp64 sum / valid, rounded to fp32; zero when smooth == 0), residual channel
+// amax folded into vamax with an integer max on the fp32 bits (all >= 0).
+template <int D, int BK>
+__global__ void __launch_bounds__(128) prep_kv_block(const __nv_bfloat16* __restrict__ K,
+                                                     const __nv_bfloat16* __restrict__ V,
+                                                     const int32_t* __restrict__ perm, int smooth,
+                                                     uint8_t* __restrict__ k_fp8, float* __restrict__ k_scale,
+                                                     float* __restrict__ v_mean, uint32_t* __restrict__ vamax, int N,
+                                                     int T) {
+    constexpr int RG = 128 / D;  // row groups
+    __shared__ int tok_s[BK];
+    __shared__ double vsum_s[RG][D];
+    __shared__ float kmax_s[128];
+    __shared__ float vmax_s[RG][D];
+    const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const int c = tid % D, rg = tid / D;
+    const int valid = min(BK, N - b * BK);
+    for (int r = tid; r < BK; r += 128) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    __syncthreads();
+    const __nv_bfloat16* kb = K + (size_t)bh * N * D + c;
+    const __nv_bfloat16* vb = V + (size_t)bh * N * D + c;
+    float kmax = 0.0f;
+    double vsum = 0.0;
+    for (int r = rg; r < valid; r += RG) {
+        const size_t row = (size_t)tok_s[r] * D;
+        kmax = fmaxf(kmax, fabsf(bf2f(kb[row])));
+        vsum += (double)bf2f(vb[row]);
+    }
+    kmax_s[tid] = kmax;
+    vsum_s[rg][c] = vsum;
+    __syncthreads();
+    for (int s = 64; s > 0; s >>= 1) {
+        if (tid < s) kmax_s[tid] = fmaxf(kmax_s[tid], kmax_s[tid + s]);
+        __syncthreads();
+    }
+    const float amax = kmax_s[0];
+    const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
+    if (tid == 0) k_scale[(size_t)bh * T + b] = __fdiv_rn(amax, 448.0f);
+    double tot = 0.0;
+#pragma unroll
+    for (int q = 0; q < RG; ++q) tot += vsum_s[q][c];
+    const float mu = smooth ? (float)(tot / (double)valid) : 0.0f;
+    if (rg == 0) v_mean[((size_t)bh * T + b) * D + c] = mu;
+    uint8_t* kout = k_fp8 + ((size_t)bh * T * BK + (size_t)b * BK) * D;
+    float vmax = 0.0f;
+    for (int r = rg; r < BK; r += RG) {
+        uint8_t code = 0;
+        if (r < valid) {
+            const size_t row = (size_t)tok_s[r] * D;  // second read of the gathered rows hits L2
+            code = (uint8_t)(e4m3x2(__fmul_rn(bf2f(kb[row]), inv), 0.0f) & 0xFF);
+            vmax = fmaxf(vmax, fabsf(__fsub_rn(bf2f(vb[row]), mu)));
+        }
+        kout[(size_t)r * D + c] = code;
+    }
+    vmax_s[rg][c] = vmax;
+    __syncthreads();
+    if (rg == 0) {
+        float m = vmax_s[0][c];
+#pragma unroll
+        for (int q = 1; q < RG; ++q) m = fmaxf(m, vmax_s[q][c]);
+        atomicMax(&vamax[(size_t)bh * D + c], __float_as_uint(m));
+    }
+}
+
+// V-Smooth off: identity order, every token in cluster 0.
+__global__ void identity_order(int32_t* __restrict__ perm, int32_t* __restrict__ labels, int64_t total, int N) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        perm[i] = (int32_t)(i % N);
+        labels[i] = 0;
+    }
+}
+
+// E4M3 residual with per-channel scales, written transposed: vt[bh][c][token].
+template <int D, int BK>
+__global__ void __launch_bounds__(128) prep_v_quant(const __nv_bfloat16* __restrict__ V,
+                                                    const int32_t* __restrict__ perm, int smooth,
+                                                    const float* __restrict__ v_mean,
+                                                    const uint32_t* __restrict__ vamax, uint8_t* __restrict__ vt_fp8,
+                                                    float* __restrict__ v_scale, int N, int T) {
+    constexpr int RG = 128 / D;
+    constexpr int STRIDE = BK + 4;  // bytes per channel row in smem (conflict-free word stores)
+    __shared__ int tok_s[BK];
+    __shared__ uint32_t cs[D * STRIDE / 4];
+    const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const int c = tid % D, rg = tid / D;
+    const int valid = min(BK, N - b * BK);
+    const int Tp = T * BK;
+    for (int r = tid; r < BK; r += 128) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    const float amax = __uint_as_float(vamax[(size_t)bh * D + c]);
+    const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
+    if (b == 0 && rg == 0) v_scale[(size_t)bh * D + c] = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    const float mu = v_mean[((size_t)bh * T + b) * D + c];
+    __syncthreads();
+    for (int r4 = rg; r4 < BK / 4; r4 += RG) {
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int r = 4 * r4 + e;
+            x[e] = 0.0f;
+            if (r < valid) {
+                const float v = bf2f(V[((size_t)bh * N + tok_s[r]) * D + c]);
+                x[e] = __fmul_rn(__fsub_rn(v, mu), inv);
+            }
+        }
+        const uint32_t w = (uint32_t)e4m3x2(x[0], x[1]) | ((uint32_t)e4m3x2(x[2], x[3]) << 16);
+        // padding tokens must be code 0 (x = +0 encodes to 0x00)
+        cs[(c * STRIDE) / 4 + r4] = w;
+    }
+    __syncthreads();
+    constexpr int CHUNKS = BK / 16;
+    for (int i = tid; i < D * CHUNKS; i += 128) {
+        const int cc = i / CHUNKS, ch = i % CHUNKS;
+        const uint32_t* src = cs + (cc * STRIDE) / 4 + ch * 4;
+        *reinterpret_cast<uint4*>(vt_fp8 + ((size_t)bh * D + cc) * Tp + (size_t)b * BK + 16 * ch) =
+            make_uint4(src[0], src[1], src[2], src[3]);
+    }
+}
+
+// Per-token Q: amax over d, inv = 448/amax, code = E4M3(q * inv), sq = amax/448.
+template <int D>
+__global__ void __launch_bounds__(256) quant_q(const __nv_bfloat16* __restrict__ Q, uint8_t* __restrict__ q_fp8,
+                                               float* __restrict__ sq, int64_t tokens) {
+    constexpr int PER = D / 32;  // values per lane
+    const int64_t tok = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (tok >= tokens) return;
+    float x[PER];
+    const __nv_bfloat16* src = Q + tok * D + lane * PER;
+    if constexpr (PER == 4) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(src);
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = bf2f(h[e]);
+    } else {
+        const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) x[e] = bf2f(h[e]);
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) m = fmaxf(m, fabsf(x[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float inv = m > 0.0f ? __fdiv_rn(448.0f, m) : 0.0f;
+    if constexpr (PER == 4) {
+        const uint32_t w = (uint32_t)e4m3x2(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv)) |
+                           ((uint32_t)e4m3x2(__fmul_rn(x[2], inv), __fmul_rn(x[3], inv)) << 16);
+        *reinterpret_cast<uint32_t*>(q_fp8 + tok * D + lane * 4) = w;
+    } else {
+        *reinterpret_cast<uint16_t*>(q_fp8 + tok * D + lane * 2) =
+            e4m3x2(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv));
+    }
+    if (lane == 0) sq[tok] = __fdiv_rn(m, 448.0f);
+}
+
+__global__ void e4m3_encode_kernel(const float* __restrict__ x, uint8_t* __restrict__ out, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        out[i] = (uint8_t)(e4m3x2(x[i], 0.0f) & 0xFF);
+}
+
+// ------------------------------------------------------------------ host launchers
+
+template <int D>
+static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
+    const int nblk = (p.N + KM_TOK - 1) / KM_TOK;
+    const int Cpad = (p.C + 63) & ~63;
+    const size_t smem = sizeof(float) * ((size_t)D * Cpad + (size_t)D * KM_TOK + Cpad) + sizeof(int) * p.C;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    km_init<<<dim3(p.C, p.BH), D, 0, s>>>(p.V, p.cent_t, p.sums, p.state, p.vamax, p.N, p.C, D);
+    for (int it = 0; it < p.iters; ++it) {
+        km_assign<D><<<dim3(nblk, p.BH), 256, smem, s>>>(p.V, p.cent_t, p.labels, p.hist, p.state, p.N, p.C, it);
+        km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it);
+        km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C);
+        if (it + 1 < p.iters) {
+            km_update<D><<<dim3(p.C, KM_SLICES, p.BH), 128, 0, s>>>(p.V, p.perm, p.cstart, p.ccount, p.sums, p.state,
+                                                                    p.N, p.C);
+            km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.cent_t, p.sums, p.ccount, p.state, p.C, D);
+        }
+    }
+    return cudaGetLastError();
+}
+
+template <int D, int BK>
+static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
+    const int T = (p.N + BK - 1) / BK;
+    if (!p.smooth) {  // plain per-channel FP8 V: identity order, zeroed channel maxima
+        const int64_t total = (int64_t)p.BH * p.N;
+        identity_order<<<(unsigned)imin64((total + 255) / 256, 148 * 32), 256, 0, s>>>(p.perm, p.labels,
+                                                                                             total, p.N);
+        cudaError_t e = cudaMemsetAsync(p.vamax, 0, sizeof(uint32_t) * (size_t)p.BH * D, s);
+        if (e != cudaSuccess) return e;
+    }
+    prep_kv_block<D, BK><<<dim3(T, p.BH), 128, 0, s>>>(p.K, p.V, p.perm, p.smooth, p.k_fp8, p.k_scale, p.v_mean,
+                                                       p.vamax, p.N, T);
+    prep_v_quant<D, BK><<<dim3(T, p.BH), 128, 0, s>>>(p.V, p.perm, p.smooth, p.v_mean, p.vamax, p.vt_fp8, p.v_scale,
+                                                      p.N, T);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const PrepLaunch& p, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    if (p.smooth) {
+        e = p.D == 128 ? kmeans_t<128>(p, s) : kmeans_t<64>(p, s);
+        if (e != cudaSuccess) return e;
+    }
+    if (p.D == 128 && p.BK == 128) return blocks_t<128, 128>(p, s);
+    if (p.D == 128 && p.BK == 64) return blocks_t<128, 64>(p, s);
+    if (p.D == 64 && p.BK == 128) return blocks_t<64, 128>(p, s);
+    return blocks_t<64, 64>(p, s);
+}
+
+cudaError_t launch_quant_q(const __nv_bfloat16* Q, uint8_t* q_fp8, float* sq, int64_t tokens, int D,
+                           cudaStream_t s) {
+    const unsigned grid = (unsigned)((tokens + 7) / 8);
+    if (D == 128)
+        quant_q<128><<<grid, 256, 0, s>>>(Q, q_fp8, sq, tokens);
+    else
+        quant_q<64><<<grid, 256, 0, s>>>(Q, q_fp8, sq, tokens);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_e4m3_encode(const float* x, uint8_t* out, int64_t n, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)imin64((n + 255) / 256, 148 * 16);
+    e4m3_encode_kernel<<<grid, 256, 0, s>>>(x, out, n);
+    return cudaGetLastError();
+}
+
+}  // namespace vc

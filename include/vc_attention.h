@@ -1,0 +1,166 @@
+/*
+ * vc_attention.h -- C ABI of the VC-Attention forward for NVIDIA B200 (sm_100a):
+ * V-Smooth prep followed by an ExpCast-FP8 attention kernel.
+ *
+ * Method sources (prose only; no code or equations are published):
+ *   chooseai.io news 7051 (VC-Attention), sections "核心方法之一：V-Smooth ..."
+ *     and "核心方法之二：ExpCast-FP8 ..."
+ *   theclarity.today, "Quantizing value residuals and casting softmax to FP8
+ *     speeds Nunchux's attention kernel 1.46x on an H200"
+ *   zerohour.day summary "Nunchux AI Introduces VC-Attention ...", key facts
+ *   RuntimeWire, "Nunchux speeds video diffusion with value smoothing and FP8
+ *     softmax casting", section "The arithmetic behind the speedup"
+ *
+ * The op is a drop-in, training-free replacement of a non-causal
+ * self-attention call over one long token sequence; the clustering runs inside
+ * the call (theclarity.today, V-Smooth paragraph).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major, on the current CUDA device, and owned by
+ *     the caller.  The library never allocates device or host memory and keeps
+ *     no state beyond a cached driver entry point.
+ *   - All GPU work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and runs asynchronously.  No entry point synchronises,
+ *     except vc_check.
+ *   - Pointers must be 16-byte aligned device pointers (256-byte aligned is
+ *     recommended).  Inputs must be finite.
+ *   - Return values: VC_OK, or an error code.  Argument errors are detected on
+ *     the host before any launch.  Launch failures return VC_ERR_CUDA.
+ *     A kernel whose internal wait exceeds params->wait_limit_ns records
+ *     VC_ERR_DEVICE_TIMEOUT in the workspace status word, stops cleanly and
+ *     leaves its outputs undefined; vc_check reports it.
+ *
+ * Shapes: B batches, H heads, N tokens, head dim d (64 or 128).  The hardware
+ * block is `block` tokens (64 or 128) and equals the key/value tile of the
+ * attention kernel.  T = ceil(N / block) blocks; Tp = T * block.
+ */
+#ifndef VC_ATTENTION_H
+#define VC_ATTENTION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VC_ABI_VERSION 1
+
+typedef enum {
+    VC_OK = 0,
+    VC_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad size or parameter */
+    VC_ERR_UNSUPPORTED = 2,    /* d or block outside {64,128}, NVFP4 residual, not sm_100 */
+    VC_ERR_CUDA = 3,           /* a CUDA runtime or driver call failed */
+    VC_ERR_DEVICE_TIMEOUT = 4, /* a device-side wait ran out (see wait_limit_ns) */
+    VC_ERR_WORKSPACE = 5       /* workspace smaller than vc_workspace_bytes() */
+} vc_status;
+
+/* Q, K, V and O layout: bf16 [B, H, N, d]. */
+typedef struct {
+    int32_t B, H, N, d;
+} vc_shape;
+
+typedef struct {
+    int32_t C;             /* k-means clusters, 1 <= C <= min(N, 256) */
+    int32_t iters;         /* k-means assignment passes, 1 <= iters <= 64 */
+    int32_t block;         /* hardware block = KV tile: 64 or 128 tokens */
+    int32_t beta;          /* ExpCast shift: byte = round(8z + 56 + beta); integer in [0, 70] */
+    int32_t smooth;        /* 1 = V-Smooth; 0 = plain per-channel FP8 V (identity order, zero means) */
+    int32_t resid_fmt;     /* 0 = E4M3 residual (the only format built) */
+    int64_t wait_limit_ns; /* bound on any single device-side wait; 0 = 2 s */
+} vc_params;
+
+/*
+ * V-Smooth prep outputs (device pointers, caller-owned).  Positions are in
+ * regrouped order: position i holds original token perm[i].
+ *   perm     int32 [B,H,N]        stable order by k-means cluster id
+ *   labels   int32 [B,H,N]        cluster id of each original token (optional: may be NULL)
+ *   k_fp8    uint8 [B,H,Tp,d]     E4M3 K rows in regrouped order; rows >= N are 0
+ *   k_scale  fp32  [B,H,T]        per-block K scale: K ~= k_scale[b] * E4M3(k_fp8)
+ *   vt_fp8   uint8 [B,H,d,Tp]     E4M3 V residual, channel-major (transposed);
+ *                                 columns >= N are 0
+ *   v_mean   fp32  [B,H,T,d]      block means of V (kept in fp32)
+ *   v_scale  fp32  [B,H,d]        per-channel residual scale:
+ *                                 V[perm[i]] ~= v_mean[i / block] + v_scale * E4M3(vt_fp8[:, i])
+ */
+typedef struct {
+    int32_t* perm;
+    int32_t* labels;
+    uint8_t* k_fp8;
+    float* k_scale;
+    uint8_t* vt_fp8;
+    float* v_mean;
+    float* v_scale;
+} vc_prep;
+
+/* ABI version of the loaded library (VC_ABI_VERSION). */
+int vc_abi_version(void);
+
+/* Static, human-readable name of a vc_status value. */
+const char* vc_status_string(int status);
+
+/* Byte sizes of the seven vc_prep buffers, in struct order, for this shape and
+ * block size.  bytes must point to 7 size_t.  Host only; no CUDA call. */
+vc_status vc_prep_buffer_bytes(const vc_shape* shape, const vc_params* params, size_t* bytes);
+
+/* Workspace size needed by vc_smooth_prepare, vc_attn_fwd and vc_attention
+ * (the largest of the three).  The workspace holds k-means state, quantised Q
+ * and the device status word; it must be zero-filled once before its first
+ * use (the status word must start at 0) and may be reused across calls on the
+ * same stream.  Host only. */
+vc_status vc_workspace_bytes(const vc_shape* shape, const vc_params* params, size_t* bytes);
+
+/*
+ * V-Smooth prep (chooseai.io news 7051, V-Smooth section; zerohour.day key
+ * facts: per-channel E4M3 residual after block-mean subtraction).
+ *   K, V    bf16 [B,H,N,d] device input
+ *   out     prep buffers to fill (labels may be NULL)
+ * Per (b, h): k-means over the N value vectors (strided init
+ * c_k = V[floor(k N / C)], `iters` assignment passes, squared Euclidean
+ * distance, ties to the lowest cluster, empty clusters keep their centroid);
+ * stable regroup by cluster id; per block: K amax scale and E4M3 K, V mean,
+ * V residual; per channel: residual amax scale and E4M3 residual.
+ */
+vc_status vc_smooth_prepare(const void* K, const void* V, const vc_shape* shape, const vc_params* params,
+                            const vc_prep* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ExpCast-FP8 attention forward over prepped K/V (chooseai.io news 7051,
+ * ExpCast-FP8 section; theclarity.today: the mean goes back in during the
+ * online softmax, one pass over the values).
+ *   Q     bf16 [B,H,N,d] device input, original token order
+ *   prep  outputs of vc_smooth_prepare for the same shape and block
+ *   O     bf16 [B,H,N,d] device output, original token order
+ * Per query row: E4M3 Q with a per-token scale; FP8 QK^T on tensor cores;
+ * per tile an integer row reference M (raised online); each score maps to the
+ * E4M3 probability byte max(0, round(A*s + 56 + beta - 8M)) with one FMA;
+ * FP8 PV; row sums of the tile restore the block means; O = (v_scale * O_res +
+ * sum_b l_b mu_b) / l.  Non-causal; keys >= N are masked.
+ */
+vc_status vc_attn_fwd(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params, void* O,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* vc_smooth_prepare followed by vc_attn_fwd on the same stream: the drop-in
+ * attention call.  `scratch` receives the prep outputs. */
+vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_shape* shape, const vc_params* params,
+                       const vc_prep* scratch, void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the workspace status word, and
+ * returns VC_OK or the recorded device error (VC_ERR_DEVICE_TIMEOUT). */
+vc_status vc_check(void* workspace, void* stream);
+
+/* Element-wise E4M3 encode of fp32 values (round to nearest even, saturate to
+ * +-448), the encoder every quantiser above uses.  x fp32 [n] -> out uint8 [n]. */
+vc_status vc_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream);
+
+/* Element-wise ExpCast byte map used inside vc_attn_fwd:
+ * out[i] = max(0, round_half_even(A[i] * s[i] + cb[i])), one fp32 FMA with the
+ * rounding inside it.  cb must hold integers with |cb| < 2^22.
+ * A, s, cb fp32 [n] -> out uint8 [n]. */
+vc_status vc_expcast_bytes(const float* A, const float* s, const float* cb, uint8_t* out, int64_t n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VC_ATTENTION_H */
