@@ -18,6 +18,7 @@ method there is) on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -92,7 +93,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except OSError:
@@ -317,8 +318,12 @@ def main():
     ap.add_argument("--workload", default="mid_32k_d128", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only this many heads of the workload (profiling captures on a smaller case)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, name=f"{w.name}_h{args.heads}", H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
     else:
