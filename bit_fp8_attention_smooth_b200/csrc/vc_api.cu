@@ -20,7 +20,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct WsLayout {
     // offsets in bytes from the workspace base
     size_t status;
-    size_t labels, cent, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
+    size_t labels, c_hi, c_lo, cnorm, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
     size_t qfp8, sq;                                                      // attention region (aliases prep)
     size_t prep_end, attn_end, total;
 };
@@ -28,12 +28,15 @@ struct WsLayout {
 WsLayout ws_layout(const vc_shape& s, const vc_params& p) {
     const size_t BH = (size_t)s.B * s.H, N = (size_t)s.N, D = (size_t)s.d, C = (size_t)p.C;
     const size_t nblk = (N + 127) / 128;
+    const size_t Cp = (C + 15) & ~size_t(15);
     WsLayout w{};
     w.status = 0;
     size_t o = 256;
     const size_t region = o;
     w.labels = o; o = align256(o + 4 * BH * N);
-    w.cent = o; o = align256(o + 4 * BH * D * C);
+    w.c_hi = o; o = align256(o + 2 * BH * Cp * D);
+    w.c_lo = o; o = align256(o + 2 * BH * Cp * D);
+    w.cnorm = o; o = align256(o + 4 * BH * Cp);
     w.sums = o; o = align256(o + 8 * BH * C * D);
     w.cstart = o; o = align256(o + 4 * BH * C);
     w.ccount = o; o = align256(o + 4 * BH * C);
@@ -108,21 +111,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3-D uint8 tensor map: dims (d0 innermost, d1, d2), row strides in bytes.
-bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
-              uint64_t stride2, uint32_t box0, uint32_t box1) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {d0, d1, d2};
-    const cuuint64_t strides[2] = {stride1, stride2};
-    const cuuint32_t box[3] = {box0, box1, 1};
-    const cuuint32_t elem[3] = {1, 1, 1};
-    const CUtensorMapSwizzle sw = box0 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, elem,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc_params& p, const vc_prep& out,
                        uint8_t* ws, const WsLayout& L, cudaStream_t stream) {
     vc::PrepLaunch pl{};
@@ -142,7 +130,11 @@ vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc
     pl.v_mean = out.v_mean;
     pl.v_scale = out.v_scale;
     pl.labels = out.labels ? out.labels : reinterpret_cast<int32_t*>(ws + L.labels);
-    pl.cent_t = reinterpret_cast<float*>(ws + L.cent);
+    pl.c_hi = reinterpret_cast<__nv_bfloat16*>(ws + L.c_hi);
+    pl.c_lo = reinterpret_cast<__nv_bfloat16*>(ws + L.c_lo);
+    pl.cnorm = reinterpret_cast<float*>(ws + L.cnorm);
+    pl.ctl.status = reinterpret_cast<int*>(ws + L.status);
+    pl.ctl.limit_ns = p.wait_limit_ns > 0 ? p.wait_limit_ns : kDefaultWaitNs;
     pl.sums = reinterpret_cast<double*>(ws + L.sums);
     pl.cstart = reinterpret_cast<int32_t*>(ws + L.cstart);
     pl.ccount = reinterpret_cast<int32_t*>(ws + L.ccount);
@@ -163,9 +155,9 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
     if (vc::launch_quant_q(static_cast<const __nv_bfloat16*>(Q), qfp8, sq, (int64_t)BH * N, D, stream) != cudaSuccess)
         return VC_ERR_CUDA;
     CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, qfp8, D, N, BH, D, (uint64_t)N * D, D, 128) ||
-        !make_map(&tk, pr.k_fp8, D, Tp, BH, D, Tp * D, D, BK) ||
-        !make_map(&tv, pr.vt_fp8, Tp, D, BH, Tp, Tp * D, BK, D))
+    if (!vc::make_tmap_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qfp8, D, N, BH, D, 128) ||
+        !vc::make_tmap_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.k_fp8, D, Tp, BH, D, BK) ||
+        !vc::make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.vt_fp8, Tp, D, BH, BK, D))
         return VC_ERR_CUDA;
     vc::AttnArgs a{};
     a.sq = sq;
@@ -183,6 +175,24 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
 }
 
 }  // namespace
+
+namespace vc {
+bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t d0,
+                  uint64_t d1, uint64_t d2, uint32_t box0, uint32_t box1) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * elem_bytes, d1 * d0 * elem_bytes};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t elem[3] = {1, 1, 1};
+    const uint32_t row = box0 * elem_bytes;
+    const CUtensorMapSwizzle sw = row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : row == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_32B;
+    return fn(m, dtype, 3, const_cast<void*>(base), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace vc
 
 extern "C" {
 

@@ -271,9 +271,15 @@ __global__ void __launch_bounds__(320, 1)
                 for (int j = 0; j < BK; ++j)
                     if (j >= valid) s[j] = -INFINITY;
             }
-            float mx = s[0];
+            // row max: 8 independent 3-input max chains, then a short tree
+            float m8[8];
 #pragma unroll
-            for (int j = 1; j < BK; ++j) mx = fmaxf(mx, s[j]);
+            for (int a = 0; a < 8; ++a) m8[a] = fmaxf(s[2 * a], s[2 * a + 1]);
+#pragma unroll
+            for (int j = 16; j < BK; j += 16)
+#pragma unroll
+                for (int a = 0; a < 8; ++a) m8[a] = fmax3(m8[a], s[j + 2 * a], s[j + 2 * a + 1]);
+            const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
             const float A = __fmul_rn(aq, sk);
             const float Mc = ceilf(__fmul_rn(__fmul_rn(A, mx), 0.125f));
             const float Mnew = t == 0 ? Mc : fmaxf(M, Mc);
@@ -289,8 +295,9 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int j = ch * 16 + q * 4;
-                    w[q] = pack4_low_bytes(expcast_t(A, s[j], cbm), expcast_t(A, s[j + 1], cbm),
-                                           expcast_t(A, s[j + 2], cbm), expcast_t(A, s[j + 3], cbm));
+                    const float2 t01 = expcast_t2(A, s[j], s[j + 1], cbm);
+                    const float2 t23 = expcast_t2(A, s[j + 2], s[j + 3], cbm);
+                    w[q] = pack4_low_bytes(t01.x, t01.y, t23.x, t23.y);
                 }
                 *reinterpret_cast<uint4*>(prow + swz_offset(row, ch, BK)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
@@ -353,10 +360,14 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int c4 = 0; c4 < D / 4; ++c4) {
                 const float4 m = mu[c4];
-                acc[4 * c4 + 0] = __fmaf_rn(lb, m.x, acc[4 * c4 + 0]);
-                acc[4 * c4 + 1] = __fmaf_rn(lb, m.y, acc[4 * c4 + 1]);
-                acc[4 * c4 + 2] = __fmaf_rn(lb, m.z, acc[4 * c4 + 2]);
-                acc[4 * c4 + 3] = __fmaf_rn(lb, m.w, acc[4 * c4 + 3]);
+                const float2 a01 = ffma2(make_float2(lb, lb), make_float2(m.x, m.y),
+                                         make_float2(acc[4 * c4 + 0], acc[4 * c4 + 1]));
+                const float2 a23 = ffma2(make_float2(lb, lb), make_float2(m.z, m.w),
+                                         make_float2(acc[4 * c4 + 2], acc[4 * c4 + 3]));
+                acc[4 * c4 + 0] = a01.x;
+                acc[4 * c4 + 1] = a01.y;
+                acc[4 * c4 + 2] = a23.x;
+                acc[4 * c4 + 3] = a23.y;
             }
             l += lb;
             __syncwarp();
@@ -428,11 +439,13 @@ cudaError_t launch_attn(int D, int BK, const CUtensorMap& tq, const CUtensorMap&
     return cudaErrorInvalidValue;
 }
 
-// ExpCast byte map, element-wise (the same device function the kernel uses).
+// ExpCast byte map, element-wise (the same packed device function the kernel
+// uses; the second lane of the pair repeats the first).
 __global__ void vc_expcast_kernel(const float* A, const float* s, const float* cb, uint8_t* out, int64_t n) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const float cbm = cb[i] + kMagic;
-        out[i] = (uint8_t)(__float_as_uint(expcast_t(A[i], s[i], cbm)) & 0xFFu);
+        const float2 t = expcast_t2(A[i], s[i], s[i], cbm);
+        out[i] = (uint8_t)(__float_as_uint(t.x) & 0xFFu);
     }
 }
 

@@ -175,6 +175,37 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     return __uint_as_float(r);
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Instruction descriptor of kind::f16: D fp32, A and B bf16, both K-major,
+// M = 128, N = n (multiple of 16, 16..256).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
+    return (1u << 4)                          // D format: fp32
+           | (1u << 7) | (1u << 10)           // A, B format: bf16
+           | (uint32_t(n >> 3) << 17)         // N / 8
+           | (uint32_t(128 >> 4) << 24);      // M / 16
+}
+
 // Instruction descriptor of kind::f8f6f4: D fp32, A and B E4M3, both K-major,
 // M = 128, N = n (multiple of 16, 16..256).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n) {
@@ -217,10 +248,29 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 // (to nearest, ties to even) is the rounding to an integer.
 constexpr float kMagic = 12582912.0f;
 
-// One FMA: t = A*s + cbm with cbm = cb + 1.5*2^23 (cb an integer, |cb| < 2^22);
-// the max clamps negative t to 0; the byte is in the low 8 bits.
-__device__ __forceinline__ float expcast_t(float A, float s, float cbm) {
-    return fmaxf(__fmaf_rn(A, s, cbm), kMagic);
+// Packed fp32 pair FMA (two IEEE fma.rn lanes in one instruction).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// One FMA per score: t = A*s + cbm with cbm = cb + 1.5*2^23 (cb an integer,
+// |cb| < 2^22); the max clamps negative t to 0; the byte is in the low 8 bits.
+// Scores go in pairs through the packed FMA.
+__device__ __forceinline__ float2 expcast_t2(float A, float s0, float s1, float cbm) {
+    const float2 t = ffma2(make_float2(A, A), make_float2(s0, s1), make_float2(cbm, cbm));
+    return make_float2(fmaxf(t.x, kMagic), fmaxf(t.y, kMagic));
 }
 __device__ __forceinline__ uint32_t pack4_low_bytes(float a, float b, float c, float d) {
     const uint32_t lo = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);

@@ -37,7 +37,9 @@ struct PrepLaunch {
     float* v_scale;
     // workspace
     int32_t* labels;
-    float* cent_t;
+    __nv_bfloat16* c_hi;  // [BH, Cp, D] centroid high bf16 part
+    __nv_bfloat16* c_lo;  // [BH, Cp, D] centroid residual bf16 part
+    float* cnorm;         // [BH, Cp] squared centroid norms
     double* sums;
     int32_t* cstart;
     int32_t* ccount;
@@ -45,7 +47,13 @@ struct PrepLaunch {
     int32_t* offs;
     KmState* state;
     uint32_t* vamax;
+    DevCtl ctl;
 };
+
+// 3-D tensor map over a dense [d2][d1][d0] array of elem_bytes elements with
+// box {box0, box1, 1}; the swizzle matches box0 * elem_bytes (128, 64 or 32 B).
+bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t d0,
+                  uint64_t d1, uint64_t d2, uint32_t box0, uint32_t box1);
 
 cudaError_t launch_attn(int D, int BK, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const AttnArgs& a, int BH, cudaStream_t stream);

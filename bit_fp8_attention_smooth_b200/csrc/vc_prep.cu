@@ -30,138 +30,171 @@ __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float
 __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 // ------------------------------------------------------------------ k-means
-// cent_t: centroids channel-major [BH, D, C] fp32.
-__global__ void km_init(const __nv_bfloat16* __restrict__ V, float* __restrict__ cent_t, double* __restrict__ sums,
-                        KmState* __restrict__ state, uint32_t* __restrict__ vamax, int N, int C, int D) {
+// Centroids live as bf16 hi/lo pairs, row-major [BH, Cp, D] (Cp = C rounded up
+// to 16; pad rows are zero), plus fp32 squared norms [BH, Cp]: v.c is computed
+// on tensor cores as v.hi + v.lo (v is exact in bf16), so the distance
+// |c|^2 - 2 v.c carries about 2^-16 relative error in c.
+__device__ __forceinline__ void store_centroid(float c, __nv_bfloat16* hi, __nv_bfloat16* lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(c);
+    *hi = h;
+    *lo = __float2bfloat16_rn(c - __bfloat162float(h));
+}
+
+// Sum over the D threads of a block (D = blockDim.x, 64 or 128).
+__device__ __forceinline__ float block_sum_d(float x, float* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = x;
+    __syncthreads();
+    float t = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    return t;
+}
+
+__global__ void km_init(const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ c_hi,
+                        __nv_bfloat16* __restrict__ c_lo, float* __restrict__ cnorm, double* __restrict__ sums,
+                        KmState* __restrict__ state, uint32_t* __restrict__ vamax, int N, int C, int Cp, int D) {
+    __shared__ float red[4];
     const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-    if (c >= D) return;
-    const int64_t src = ((int64_t)k * N) / C;
-    cent_t[((size_t)bh * D + c) * C + k] = bf2f(V[((size_t)bh * N + src) * D + c]);
-    sums[((size_t)bh * C + k) * D + c] = 0.0;
+    const size_t row = ((size_t)bh * Cp + k) * D + c;
+    float x = 0.0f;
+    if (k < C) {
+        const int64_t src = ((int64_t)k * N) / C;
+        x = bf2f(V[((size_t)bh * N + src) * D + c]);
+        sums[((size_t)bh * C + k) * D + c] = 0.0;
+    }
+    c_hi[row] = __float2bfloat16_rn(x);
+    c_lo[row] = __float2bfloat16_rn(0.0f);
+    const float nrm = block_sum_d(x * x, red);
+    if (c == 0) cnorm[(size_t)bh * Cp + k] = nrm;
     if (k == 0) {
         vamax[(size_t)bh * D + c] = 0u;
         if (c == 0) state[bh] = KmState{0, 0, 0, 0};
     }
 }
 
-constexpr int KM_TOK = 128;  // tokens per assign block
+constexpr int KM_TOK = 128;  // tokens per assign block (the MMA's M)
 
+// Assignment pass on tensor cores: one CTA = 128 tokens of one head.
+//   S[token, k] = v . c_hi + v . c_lo   (kind::f16, bf16 x bf16 -> fp32 in TMEM)
+//   label = argmin_k (|c_k|^2 - 2 S[token, k]), ties to the lowest k.
 template <int D>
-__global__ void __launch_bounds__(256) km_assign(const __nv_bfloat16* __restrict__ V, const float* __restrict__ cent_t,
-                                                 int32_t* __restrict__ labels, int32_t* __restrict__ hist,
-                                                 KmState* __restrict__ state, int N, int C, int it) {
-    extern __shared__ float sm[];
+__global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtensorMap tm_v,
+                                                 const __grid_constant__ CUtensorMap tm_chi,
+                                                 const __grid_constant__ CUtensorMap tm_clo,
+                                                 const float* __restrict__ cnorm, int32_t* __restrict__ labels,
+                                                 int32_t* __restrict__ hist, KmState* __restrict__ state, int N, int C,
+                                                 int Cp, int it, DevCtl ctl) {
+    constexpr int A_BYTES = KM_TOK * D * 2;
     const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x;
-    if (state[bh].done) return;
-    const int Cpad = (C + 63) & ~63;
-    float* cent_s = sm;                      // [D][Cpad]
-    float* v_s = cent_s + D * Cpad;          // [D][KM_TOK]
-    float* cnorm = v_s + D * KM_TOK;         // [Cpad]
-    int* hist_s = reinterpret_cast<int*>(cnorm + Cpad);  // [C]
-    const int tid = threadIdx.x;
+    if (state[bh].done) return;  // uniform over the CTA, before any barrier or TMEM use
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_base);
+    const int B_BYTES = Cp * D * 2;
+    const uint32_t sA = base, sBh = base + A_BYTES, sBl = sBh + B_BYTES;
+    float* cn_s = reinterpret_cast<float*>(smem + A_BYTES + 2 * B_BYTES);
+    int* hist_s = reinterpret_cast<int*>(cn_s + 256);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(hist_s + 256);  // [0] loads, [1] mma
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int n0 = blk * KM_TOK;
-    const int valid = min(KM_TOK, N - n0);
+    const uint32_t ncols = Cp <= 32 ? 32 : (Cp <= 64 ? 64 : (Cp <= 128 ? 128 : 256));
+    const uint32_t bar_ld = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
 
-    for (int i = tid; i < D * Cpad; i += 256) {
-        const int c = i / Cpad, k = i % Cpad;
-        cent_s[i] = k < C ? cent_t[((size_t)bh * D + c) * C + k] : 0.0f;
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
     }
-    for (int i = tid; i < C; i += 256) hist_s[i] = 0;
-    for (int i = tid; i < KM_TOK * (D / 8); i += 256) {
-        const int r = i % KM_TOK, c8 = i / KM_TOK;
-        float f[8];
-        if (r < valid) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(V + ((size_t)bh * N + n0 + r) * D + 8 * c8);
-            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = bf2f(h[e]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = 0.0f;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v_s[(8 * c8 + e) * KM_TOK + r] = f[e];
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), ncols);
+        tmem_relinquish();
     }
+    for (int k = tid; k < Cp; k += 128) cn_s[k] = cnorm[(size_t)bh * Cp + k];
+    for (int k = tid; k < C; k += 128) hist_s[k] = 0;
+    tc_fence_before();
     __syncthreads();
-    for (int k = tid; k < Cpad; k += 256) {
-        float s = 0.0f;
-        for (int c = 0; c < D; ++c) s = fmaf(cent_s[c * Cpad + k], cent_s[c * Cpad + k], s);
-        cnorm[k] = s;
-    }
-    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
 
-    const int g = tid >> 3, h = tid & 7;  // tokens 4g..4g+3; centroids 8h..8h+7 of each 64-chunk
-    float best_d[4];
-    int best_k[4];
+    bool ok = true;
+    if (tid == 0) {
+        mbar_expect_tx_arrive(bar_ld, A_BYTES + 2 * B_BYTES);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        best_d[i] = INFINITY;
-        best_k[i] = 0;
-    }
-    for (int cc = 0; cc < Cpad; cc += 64) {
-        float acc[4][8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-#pragma unroll 4
-        for (int c = 0; c < D; ++c) {
-            const float4 vv = *reinterpret_cast<const float4*>(v_s + c * KM_TOK + 4 * g);
-            const float4 ca = *reinterpret_cast<const float4*>(cent_s + c * Cpad + cc + 8 * h);
-            const float4 cb = *reinterpret_cast<const float4*>(cent_s + c * Cpad + cc + 8 * h + 4);
-            const float v4[4] = {vv.x, vv.y, vv.z, vv.w};
-            const float c8[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(v4[i], c8[j], acc[i][j]);
+        for (int kc = 0; kc < D / 64; ++kc) {
+            tma_load_3d(sA + kc * (KM_TOK * 128), &tm_v, bar_ld, 64 * kc, n0, bh);
+            tma_load_3d(sBh + kc * (Cp * 128), &tm_chi, bar_ld, 64 * kc, 0, bh);
+            tma_load_3d(sBl + kc * (Cp * 128), &tm_clo, bar_ld, 64 * kc, 0, bh);
         }
+        ok = mbar_wait(bar_ld, 0, ctl, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(Cp);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int k = cc + 8 * h + j;
-            if (k < C) {
-                const float cn = cnorm[k];
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk & 3) * 32;
+                const uint64_t da = smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128);
+                const uint64_t dh = smem_desc(sBh + (kk >> 2) * (Cp * 128) + off, 128);
+                mma_bf16(tmem, da, dh, idesc, kk > 0);
+            }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float dist = cn - 2.0f * acc[i][j];
-                    if (dist < best_d[i]) {
-                        best_d[i] = dist;
-                        best_k[i] = k;
-                    }
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk & 3) * 32;
+                const uint64_t da = smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128);
+                const uint64_t dl = smem_desc(sBl + (kk >> 2) * (Cp * 128) + off, 128);
+                mma_bf16(tmem, da, dl, idesc, 1u);
+            }
+        }
+        mma_commit(bar_mma);  // also covers the case of no MMA issued
+    }
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_mma, 0, ctl, abort_flag));
+    int changed = 0;
+    if (ok && !*abort_flag) {
+        tc_fence_after();
+        const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
+        float best = INFINITY;
+        int bestk = 0;
+        for (int k0 = 0; k0 < Cp; k0 += 16) {
+            float dot[16];
+            tmem_ld16(lane_tmem + k0, dot);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int k = k0 + j;
+                const float dist = cn_s[k] - 2.0f * dot[j];
+                if (k < C && dist < best) {
+                    best = dist;
+                    bestk = k;
                 }
             }
         }
-    }
-    // reduce over the 8 lanes sharing a token group (lowest index on ties)
-#pragma unroll
-    for (int m = 1; m < 8; m <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float od = __shfl_xor_sync(0xffffffffu, best_d[i], m);
-            const int ok = __shfl_xor_sync(0xffffffffu, best_k[i], m);
-            if (od < best_d[i] || (od == best_d[i] && ok < best_k[i])) {
-                best_d[i] = od;
-                best_k[i] = ok;
-            }
-        }
-    }
-    int changed = 0;
-    if (h == 0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = 4 * g + i;
-            if (r < valid) {
-                int32_t* lp = labels + (size_t)bh * N + n0 + r;
-                if (it == 0 || *lp != best_k[i]) ++changed;
-                *lp = best_k[i];
-                atomicAdd(&hist_s[best_k[i]], 1);
-            }
+        if (n0 + tid < N) {
+            int32_t* lp = labels + (size_t)bh * N + n0 + tid;
+            if (it == 0 || *lp != bestk) changed = 1;
+            *lp = bestk;
+            atomicAdd(&hist_s[bestk], 1);
         }
     }
     changed = __reduce_add_sync(0xffffffffu, changed);
     if ((tid & 31) == 0 && changed) atomicAdd(&state[bh].changed, changed);
+    // The load barrier may still be pending after an abort: let the copies land.
+    if (tid == 0 && !ok) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar_ld, 0) && (int64_t)(globaltimer() - t0) < ctl.limit_ns) {
+        }
+    }
+    tc_fence_before();
     __syncthreads();
-    for (int k = tid; k < C; k += 256) hist[((size_t)bh * C + k) * nblk + blk] = hist_s[k];
+    for (int k = tid; k < C; k += 128) hist[((size_t)bh * C + k) * nblk + blk] = hist_s[k];
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
+    }
 }
 
 // Exclusive scan of hist[bh] in (cluster, block) order -> offs; cluster ranges.
@@ -250,14 +283,21 @@ __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict
     if (b > a) atomicAdd(&sums[((size_t)bh * C + k) * D + c], acc);
 }
 
-__global__ void km_finalize(float* __restrict__ cent_t, double* __restrict__ sums, const int32_t* __restrict__ ccount,
-                            const KmState* __restrict__ state, int C, int D) {
+__global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __restrict__ c_lo,
+                            float* __restrict__ cnorm, double* __restrict__ sums, const int32_t* __restrict__ ccount,
+                            const KmState* __restrict__ state, int C, int Cp, int D) {
+    __shared__ float red[4];
     const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-    if (c >= D || state[bh].done) return;
+    if (state[bh].done) return;
     const int cnt = ccount[(size_t)bh * C + k];
+    if (cnt == 0) return;  // an empty cluster keeps its centroid (sums are still 0)
     double* sp = &sums[((size_t)bh * C + k) * D + c];
-    if (cnt > 0) cent_t[((size_t)bh * D + c) * C + k] = (float)(*sp / (double)cnt);
+    const float x = (float)(*sp / (double)cnt);
     *sp = 0.0;
+    const size_t row = ((size_t)bh * Cp + k) * D + c;
+    store_centroid(x, c_hi + row, c_lo + row);
+    const float nrm = block_sum_d(x * x, red);
+    if (c == 0) cnorm[(size_t)bh * Cp + k] = nrm;
 }
 
 // ------------------------------------------------------------------ block quantisation
@@ -429,23 +469,30 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ x, uint8_t* __restr
 template <int D>
 static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     const int nblk = (p.N + KM_TOK - 1) / KM_TOK;
-    const int Cpad = (p.C + 63) & ~63;
-    const size_t smem = sizeof(float) * ((size_t)D * Cpad + (size_t)D * KM_TOK + Cpad) + sizeof(int) * p.C;
+    const int Cp = (p.C + 15) & ~15;
+    const size_t smem = 1024 + (size_t)KM_TOK * D * 2 + 2 * (size_t)Cp * D * 2 + 2 * 256 * 4 + 64;
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    km_init<<<dim3(p.C, p.BH), D, 0, s>>>(p.V, p.cent_t, p.sums, p.state, p.vamax, p.N, p.C, D);
+    CUtensorMap tv, th, tl;
+    if (!make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.V, D, p.N, p.BH, 64, KM_TOK) ||
+        !make_tmap_3d(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.c_hi, D, Cp, p.BH, 64, Cp) ||
+        !make_tmap_3d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.c_lo, D, Cp, p.BH, 64, Cp))
+        return cudaErrorInvalidValue;
+    km_init<<<dim3(Cp, p.BH), D, 0, s>>>(p.V, p.c_hi, p.c_lo, p.cnorm, p.sums, p.state, p.vamax, p.N, p.C, Cp, D);
     for (int it = 0; it < p.iters; ++it) {
-        km_assign<D><<<dim3(nblk, p.BH), 256, smem, s>>>(p.V, p.cent_t, p.labels, p.hist, p.state, p.N, p.C, it);
+        km_assign<D><<<dim3(nblk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.labels, p.hist, p.state, p.N, p.C,
+                                                          Cp, it, p.ctl);
         km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it);
         km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C);
         if (it + 1 < p.iters) {
             km_update<D><<<dim3(p.C, KM_SLICES, p.BH), 128, 0, s>>>(p.V, p.perm, p.cstart, p.ccount, p.sums, p.state,
                                                                     p.N, p.C);
-            km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.cent_t, p.sums, p.ccount, p.state, p.C, D);
+            km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.sums, p.ccount, p.state, p.C, Cp,
+                                                      D);
         }
     }
     return cudaGetLastError();
