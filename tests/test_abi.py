@@ -1,0 +1,66 @@
+"""The C ABI library builds for sm_100a, loads, and exports every function that
+include/*.h declares (no compute calls: this runs without a GPU)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(vc_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def libpath():
+    from bit_fp8_attention_smooth_b200 import build
+
+    return build.build()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("vc_smooth_prepare", "vc_attn_fwd", "vc_attention", "vc_workspace_bytes", "vc_prep_buffer_bytes",
+              "vc_check", "vc_status_string", "vc_abi_version", "vc_e4m3_encode", "vc_expcast_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(libpath):
+    out = subprocess.run(["nm", "-D", "--defined-only", libpath], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+
+
+def test_library_loads_and_answers_host_queries(libpath):
+    L = ctypes.CDLL(libpath)
+    assert L.vc_abi_version() == 1
+    L.vc_status_string.restype = ctypes.c_char_p
+    assert L.vc_status_string(0) == b"ok"
+    import bit_fp8_attention_smooth_b200 as vc
+
+    shape = (1, 40, 32768, 128)
+    params = vc.Params(C=64, iters=10, block=128)
+    sizes = vc.prep_sizes(shape, params)
+    assert sizes[2] == 40 * 32768 * 128 and sizes[4] == 40 * 128 * 32768
+    assert vc.workspace_bytes(shape, params) >= 40 * 32768 * 128
+    with pytest.raises(vc.VcError) as e:
+        vc.workspace_bytes((1, 1, 100, 96), params)
+    assert e.value.status == vc.VC_ERR_UNSUPPORTED
+
+
+def test_oracle_builds_independently():
+    import oracle
+
+    path = oracle.build()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    assert "vo_attn_emul" in out and "vc_" not in out
