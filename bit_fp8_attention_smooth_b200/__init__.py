@@ -66,6 +66,7 @@ def lib():
             "vc_attn_fwd": (ctypes.c_int, [P, PR, PS, PP, P, P, S, P]),
             "vc_attention": (ctypes.c_int, [P, P, P, PS, PP, PR, P, P, S, P]),
             "vc_check": (ctypes.c_int, [P, P]),
+            "vc_attn_fwd_noalloc": (ctypes.c_int, [P, PR, PS, PP, P, P]),
             "vc_e4m3_encode": (ctypes.c_int, [P, P, i64, P]),
             "vc_expcast_bytes": (ctypes.c_int, [P, P, P, P, i64, P]),
         }
@@ -205,6 +206,22 @@ def attention(Q, K, V, params: Params, out=None, prep=None, workspace=None, stre
                             ctypes.byref(params.c()), ctypes.byref(_prep_struct(prep)), out.data_ptr(),
                             ws.data_ptr(), ws.numel(), _stream(stream))
     _ok(st, "vc_attention")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def attn_fwd_noalloc(Q: torch.Tensor, prep, params: Params, out=None, stream=None) -> torch.Tensor:
+    """vc_attn_fwd without a workspace, for callers that cannot allocate at
+    call time: the library's static per-device scratch holds the quantised Q.
+    Problems larger than the scratch raise VcError(VC_ERR_WORKSPACE); calls
+    that overlap on the GPU race on the shared scratch."""
+    _check_input(Q, "Q")
+    out = torch.empty_like(Q) if out is None else out
+    st = lib().vc_attn_fwd_noalloc(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
+                                   ctypes.byref(params.c()), out.data_ptr(), _stream(stream))
+    _ok(st, "vc_attn_fwd_noalloc")
     return out
 
 

@@ -194,6 +194,29 @@ bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dtype, int elem_bytes, con
 }
 }  // namespace vc
 
+// Scratch of vc_attn_fwd_noalloc: status word, quantised Q and its scales.
+// In host code the symbol is only a handle; the device address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[VC_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {nullptr};
+
+vc_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return VC_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return VC_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return VC_OK;
+}
+}  // namespace
+
 extern "C" {
 
 int vc_abi_version(void) { return VC_ABI_VERSION; }
@@ -274,6 +297,22 @@ vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_sha
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((st = prepare_impl(K, V, *shape, *params, *scratch, ws, L, s)) != VC_OK) return st;
     return attn_impl(Q, *scratch, *shape, *params, O, ws, L, s);
+}
+
+vc_status vc_attn_fwd_noalloc(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params,
+                              void* O, void* stream) {
+    vc_status st = check_shape_params(shape, params);
+    if (st != VC_OK) return st;
+    if (!aligned16(Q) || !aligned16(O)) return VC_ERR_INVALID_ARG;
+    if ((st = check_prep_ptrs(prep, false)) != VC_OK) return st;
+    const WsLayout L = ws_layout(*shape, *params);  // the attention region only: status, Q fp8, Q scales
+    if (L.attn_end > VC_NOALLOC_SCRATCH_BYTES) return VC_ERR_WORKSPACE;
+    if ((st = check_device()) != VC_OK) return st;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != VC_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return VC_ERR_CUDA;  // status word starts at 0
+    return attn_impl(Q, *prep, *shape, *params, O, static_cast<uint8_t*>(scratch), L, s);
 }
 
 vc_status vc_check(void* workspace, void* stream) {

@@ -17,8 +17,9 @@
  *
  * Conventions for every entry point:
  *   - Tensors are dense, row-major, on the current CUDA device, and owned by
- *     the caller.  The library never allocates device or host memory and keeps
- *     no state beyond a cached driver entry point.
+ *     the caller.  The library never allocates device or host memory; its only
+ *     state is a cached driver entry point and the static scratch array of
+ *     vc_attn_fwd_noalloc.
  *   - All GPU work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and runs asynchronously.  No entry point synchronises,
  *     except vc_check.
@@ -144,6 +145,33 @@ vc_status vc_attn_fwd(const void* Q, const vc_prep* prep, const vc_shape* shape,
  * attention call.  `scratch` receives the prep outputs. */
 vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_shape* shape, const vc_params* params,
                        const vc_prep* scratch, void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Allocation-free variant of vc_attn_fwd, for callers that cannot allocate
+ * device memory at call time: a host runtime that hands the op only its
+ * input and output buffers and owns every other byte, or a real-time loop that
+ * cannot afford cudaMalloc's implicit device synchronisation or its failure
+ * under memory pressure.  The pages describe no such entry point; it is a
+ * property of this library, not of the method.
+ *
+ * Arguments and results are those of vc_attn_fwd without the workspace: the
+ * quantised Q, its scales and the status word live in a scratch array that
+ * the library reserves statically, VC_NOALLOC_SCRATCH_BYTES per device, held
+ * by every GPU that loads the library until the process exits.  The problem
+ * must fit: 768 + B*H*N*(d + 4) bytes (rounded up) <= VC_NOALLOC_SCRATCH_BYTES,
+ * else VC_ERR_WORKSPACE is returned before anything is launched.
+ *
+ * The first call on a device looks up the scratch address on that device
+ * (make that first call before any stream capture).  Every call shares the
+ * one array and clears its status word first, so calls that overlap on the
+ * GPU (other streams, or other host threads) race and must be serialised by
+ * the caller.  A device-side wait timeout is not reported by this entry
+ * point; O is then undefined.  No cudaMalloc, cudaFree or allocating library
+ * routine is called.
+ */
+#define VC_NOALLOC_SCRATCH_BYTES (16u << 20)
+vc_status vc_attn_fwd_noalloc(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params,
+                              void* O, void* stream);
 
 /* Synchronises `stream`, reads and clears the workspace status word, and
  * returns VC_OK or the recorded device error (VC_ERR_DEVICE_TIMEOUT). */
