@@ -30,7 +30,7 @@ def build(force: bool = False) -> str:
         os.makedirs(os.path.dirname(_SO), exist_ok=True)
         tmp = _SO + f".{os.getpid()}.tmp"
         subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
              "-Wall", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _SO)
     return _SO

@@ -161,22 +161,32 @@ VO_API void vo_kmeans(const uint16_t* v, int n, int d, int C, int iters, int32_t
         int64_t src = ((int64_t)k * n) / C;
         for (int c = 0; c < d; ++c) cent[(size_t)k * d + c] = vd[(size_t)src * d + c];
     }
+    double* ct = (double*)malloc(sizeof(double) * (size_t)C * d); /* centroids, channel-major */
     for (int it = 0; it < iters; ++it) {
-        for (int j = 0; j < n; ++j) {
-            int best = 0;
-            double bestd = INFINITY;
-            for (int k = 0; k < C; ++k) {
-                double dist = 0.0;
+        for (int k = 0; k < C; ++k)
+            for (int c = 0; c < d; ++c) ct[(size_t)c * C + k] = cent[(size_t)k * d + c];
+        /* assignment: tokens are independent, so they are split over threads;
+         * each token's distances are summed over channels in order */
+#pragma omp parallel
+        {
+            double* dist = (double*)malloc(sizeof(double) * (size_t)C);
+#pragma omp for schedule(static)
+            for (int j = 0; j < n; ++j) {
+                for (int k = 0; k < C; ++k) dist[k] = 0.0;
                 for (int c = 0; c < d; ++c) {
-                    double diff = vd[(size_t)j * d + c] - cent[(size_t)k * d + c];
-                    dist += diff * diff;
+                    const double x = vd[(size_t)j * d + c];
+                    const double* row = ct + (size_t)c * C;
+                    for (int k = 0; k < C; ++k) {
+                        const double diff = x - row[k];
+                        dist[k] += diff * diff;
+                    }
                 }
-                if (dist < bestd) { /* strict: ties keep the lowest k */
-                    bestd = dist;
-                    best = k;
-                }
+                int best = 0;
+                for (int k = 1; k < C; ++k)
+                    if (dist[k] < dist[best]) best = k; /* strict: ties keep the lowest k */
+                labels[j] = best;
             }
-            labels[j] = best;
+            free(dist);
         }
         if (it == iters - 1) break;
         memset(sums, 0, sizeof(double) * (size_t)C * d);
@@ -189,6 +199,7 @@ VO_API void vo_kmeans(const uint16_t* v, int n, int d, int C, int iters, int32_t
             if (cnt[k] > 0)
                 for (int c = 0; c < d; ++c) cent[(size_t)k * d + c] = sums[(size_t)k * d + c] / (double)cnt[k];
     }
+    free(ct);
     free(vd);
     free(sums);
     free(cnt);

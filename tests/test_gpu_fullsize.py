@@ -1,0 +1,90 @@
+"""Parity at the full sizes of the large workloads, in the launch configuration
+the benchmark times (vc_smooth_prepare + vc_attn_fwd over all heads at once),
+on sampled outputs the oracle computes one by one: heads 0 and H-1 (full
+k-means / regroup / quantisation of the head), 256 strided query rows per head
+over all keys, always including the ragged last row."""
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_fp8_attention_smooth_b200 import synth
+from gpu_common import BETA, COS_TOL, REL_L2_TOL, bits, check_perm, gpu_prep_head, metrics
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+ROWS = 256
+
+
+@pytest.fixture(scope="module")
+def vc():
+    import bit_fp8_attention_smooth_b200 as m
+
+    m.lib()
+    return m
+
+
+def _sample_rows(N):
+    rows = np.unique(np.concatenate([np.linspace(0, N - 1, ROWS).astype(np.int64), [N - 1]]))
+    return rows
+
+
+def _check_workload(vc, w, smooth=True):
+    shape = (w.B, w.H, w.N, w.d)
+    q = synth.tensor_bf16(w, "q").cuda()
+    k = synth.tensor_bf16(w, "k").cuda()
+    v = synth.tensor_bf16(w, "v").cuda()
+    params = vc.Params.for_workload(w, beta=BETA, smooth=smooth)
+    ws = vc.alloc_workspace(shape, params)
+    prep = vc.smooth_prepare(k, v, params, workspace=ws)
+    out = vc.attn_fwd(q, prep, params, workspace=ws)
+    vc.check(ws)
+    heads = [0, w.H - 1]
+    rows = _sample_rows(w.N)
+    gout = {h: out[0, h, rows].float().cpu().numpy() for h in heads}
+    gprep = {h: gpu_prep_head({kk: t[:, h:h + 1].cpu() for kk, t in prep.items()}, 0, 0, w.N, w.block)
+             for h in heads}
+    del q, k, v, out, prep, ws
+    torch.cuda.empty_cache()
+
+    def run(h):
+        qb, kb, vb = (synth.head_bits(w, t, 0, h) for t in "qkv")
+        r = oracle.forward_head(qb, kb, vb, rows, C=w.C, iters=w.iters, bk=w.block, beta=BETA, smooth=smooth,
+                                threads=8)
+        r["exact"] = oracle.attn_exact(qb, kb, vb, rows, threads=8)
+        return r
+
+    with ThreadPoolExecutor(len(heads)) as ex:
+        refs = dict(zip(heads, ex.map(run, heads)))
+    for h in heads:
+        ref, got = refs[h], gprep[h]
+        check_perm(got["perm"], got["labels"], w.N)
+        agree = (got["labels"] == ref["prep"]["labels"]).mean()
+        assert agree >= 0.999, (h, agree)
+        if np.array_equal(got["perm"], ref["prep"]["perm"]):
+            for key in ("khat", "ksc", "vmu", "vsc", "vhat"):
+                assert np.array_equal(got[key], ref["prep"][key]), (h, key)
+        rel, cos, _ = metrics(gout[h], ref["out"])
+        rel_x, _, psnr_x = metrics(gout[h], ref["exact"])
+        print(f"{w.name} smooth={smooth} head {h}: labels agree {agree:.5f}, "
+              f"vs emulation rel={rel:.2e} cos={cos:.6f}; vs exact rel={rel_x:.3e} psnr={psnr_x:.1f} dB")
+        assert rel <= REL_L2_TOL and cos >= COS_TOL, (h, rel, cos)
+
+
+def test_mid_32k(vc):
+    _check_workload(vc, synth.WORKLOADS["mid_32k_d128"])
+
+
+@pytest.mark.parametrize("smooth", [True, False], ids=["vsmooth", "plain"])
+def test_grid720p_ragged(vc, smooth):
+    _check_workload(vc, synth.WORKLOADS["grid720p_75600_d128"], smooth)
+
+
+def test_nvfp4_shape_with_e4m3_residual(vc):
+    _check_workload(vc, synth.WORKLOADS["nvfp4_32k_d128"])
+
+
+def test_longclip(vc):
+    _check_workload(vc, synth.WORKLOADS["longclip_245952_d128"])
