@@ -20,7 +20,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct WsLayout {
     // offsets in bytes from the workspace base
     size_t status;
-    size_t labels, c_hi, c_lo, cnorm, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
+    size_t labels, c_hi, c_lo, cnorm, cent64, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
     size_t qfp8, sq;                                                      // attention region (aliases prep)
     size_t prep_end, attn_end, total;
 };
@@ -37,6 +37,7 @@ WsLayout ws_layout(const vc_shape& s, const vc_params& p) {
     w.c_hi = o; o = align256(o + 2 * BH * Cp * D);
     w.c_lo = o; o = align256(o + 2 * BH * Cp * D);
     w.cnorm = o; o = align256(o + 4 * BH * Cp);
+    w.cent64 = o; o = align256(o + 8 * BH * C * D);
     w.sums = o; o = align256(o + 8 * BH * C * D);
     w.cstart = o; o = align256(o + 4 * BH * C);
     w.ccount = o; o = align256(o + 4 * BH * C);
@@ -133,6 +134,7 @@ vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc
     pl.c_hi = reinterpret_cast<__nv_bfloat16*>(ws + L.c_hi);
     pl.c_lo = reinterpret_cast<__nv_bfloat16*>(ws + L.c_lo);
     pl.cnorm = reinterpret_cast<float*>(ws + L.cnorm);
+    pl.cent64 = reinterpret_cast<double*>(ws + L.cent64);
     pl.ctl.status = reinterpret_cast<int*>(ws + L.status);
     pl.ctl.limit_ns = p.wait_limit_ns > 0 ? p.wait_limit_ns : kDefaultWaitNs;
     pl.sums = reinterpret_cast<double*>(ws + L.sums);
@@ -154,12 +156,12 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
     float* sq = reinterpret_cast<float*>(ws + L.sq);
     if (vc::launch_quant_q(static_cast<const __nv_bfloat16*>(Q), qfp8, sq, (int64_t)BH * N, D, stream) != cudaSuccess)
         return VC_ERR_CUDA;
-    CUtensorMap tq, tk, tv;
-    if (!vc::make_tmap_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qfp8, D, N, BH, D, 128) ||
-        !vc::make_tmap_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.k_fp8, D, Tp, BH, D, BK) ||
+    CUtensorMap tk, tv;
+    if (!vc::make_tmap_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.k_fp8, D, Tp, BH, D, BK) ||
         !vc::make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.vt_fp8, Tp, D, BH, BK, D))
         return VC_ERR_CUDA;
     vc::AttnArgs a{};
+    a.q_fp8 = qfp8;
     a.sq = sq;
     a.k_scale = pr.k_scale;
     a.v_mean = pr.v_mean;
@@ -171,7 +173,7 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
     a.beta = p.beta;
     a.ctl.status = reinterpret_cast<int*>(ws + L.status);
     a.ctl.limit_ns = p.wait_limit_ns > 0 ? p.wait_limit_ns : kDefaultWaitNs;
-    return vc::launch_attn(D, BK, tq, tk, tv, a, BH, stream) == cudaSuccess ? VC_OK : VC_ERR_CUDA;
+    return vc::launch_attn(D, BK, tk, tv, a, BH, stream) == cudaSuccess ? VC_OK : VC_ERR_CUDA;
 }
 
 }  // namespace

@@ -8,72 +8,74 @@
 // softmax (same page, V-Smooth section; theclarity.today: restored during the
 // online softmax, one pass over the values).
 //
-// One CTA computes a 128-row query tile of one (b, h) against all T key tiles:
-//   warp 0       TMA producer: Q tile once; K tile, V^T tile and block mean per
-//                key tile through a STAGES-deep ring.
-//   warp 1       TMEM owner and MMA issuer (one thread):
-//                  S[t%2]  = Q K_t^T                       (kind::f8f6f4, TMEM fp32)
-//                  O      += P_t V_t                       (accumulates over t)
-//                  L[t%2]  = P_t 1   (row sums of the bytes' values, N = 16)
-//   warps 2..5   softmax, one thread per query row: row max of S, integer row
-//                reference M (raised online; a rise by k rescales O by 2^-k,
-//                exactly), ExpCast bytes into shared memory as the A operand of
-//                the PV MMA.
-//   warps 6..9   correction, one thread per row: acc += l_t * mu_t (the block-
-//                mean restore) and l += l_t, both rescaled with O; epilogue
-//                O = (v_scale * O + acc) / l in bf16, original token order.
+// One CTA computes a 128-row query tile of one (b, h) against all T key tiles.
+// The A operands of every MMA live in tensor memory, so shared memory only
+// feeds the B operands (K tile, V^T tile, a constant tile of ones):
+//   TMEM (columns): S0, S1 [BK each] | O [D + 16] | Q [D/4] | P0, P1 [BK/4 each]
+//                   (E4M3 A operands: 4 values a column).  O's column D
+//                   accumulates the running row sum l: the PV B operand is the
+//                   V^T tile followed by 16 rows of E4M3 ones.
+//   warp 0       TMA producer: K tile, V^T tile and block mean per key tile
+//                through a STAGES-deep ring.
+//   warp 1       TMEM owner and MMA issuer (one thread), kind::f8f6f4:
+//                  S[t%2] = Q K_t^T     (A = Q in TMEM)
+//                  [O|l] += P_t [V_t|1] (A = P_t in TMEM; N = D + 16)
+//   warps 2..9   softmax, two warps per query row (each half of the tile's
+//                scores): they first write the row's E4M3 Q into TMEM; per
+//                tile: row max of S, integer row reference M (raised online;
+//                a rise by k rescales O by 2^-k, exactly), ExpCast bytes
+//                stored to TMEM as the A operand of the PV MMA.
+//   warps 10..17 correction, two warps per row (each half of the channels):
+//                the tile's row sum l_t = l(t) - 2^-k l(t-1) from O's column D,
+//                acc += l_t * mu_t (the block-mean restore), rescaled with O;
+//                epilogue O = (v_scale * O + acc) / l in bf16, original token
+//                order.
 // Every wait is bounded (DevCtl); on a timeout the CTA drains its copies and
 // MMAs, frees TMEM and exits with the status word set.
 #include "vc_launch.cuh"
 
 namespace vc {
 
-
 template <int D, int BK>
 struct AttnCfg {
     static constexpr int BM = 128;
-    static constexpr int STAGES = 3;
-    static constexpr int THREADS = 320;
-    static constexpr int Q_BYTES = BM * D;
+    static constexpr int STAGES = 4;
+    static constexpr int THREADS = 576;  // 18 warps
     static constexpr int K_BYTES = BK * D;
-    static constexpr int V_BYTES = D * BK;
-    static constexpr int P_BYTES = BM * BK;
-    static constexpr int ONES_BYTES = 16 * BK;
+    static constexpr int V_BYTES = D * BK;            // the TMA-loaded V^T tile
+    static constexpr int VX_BYTES = (D + 16) * BK;    // + 16 rows of ones (the l column)
     static constexpr int MU_BYTES = D * 4;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
-    static constexpr int OFF_P = OFF_V + STAGES * V_BYTES;
-    static constexpr int OFF_ONES = OFF_P + 2 * P_BYTES;
-    static constexpr int OFF_MU = OFF_ONES + ONES_BYTES;
+    static constexpr int OFF_MU = OFF_V + STAGES * VX_BYTES;
     static constexpr int OFF_KINC = OFF_MU + STAGES * MU_BYTES;
-    static constexpr int OFF_BAR = OFF_KINC + 4 * BM * 4;
+    static constexpr int OFF_MXEX = OFF_KINC + 4 * BM * 4;
+    static constexpr int OFF_BAR = OFF_MXEX + 2 * 2 * BM * 4;
     // barrier slots
-    static constexpr int B_QFULL = 0;
+    static constexpr int B_QREADY = 0;
     static constexpr int B_KFULL = 1;
     static constexpr int B_KEMPTY = B_KFULL + STAGES;
     static constexpr int B_VFULL = B_KEMPTY + STAGES;
     static constexpr int B_VEMPTY = B_VFULL + STAGES;
     static constexpr int B_SFULL = B_VEMPTY + STAGES;
-    static constexpr int B_SFREE = B_SFULL + 2;
-    static constexpr int B_PFULL = B_SFREE + 2;
+    static constexpr int B_PFULL = B_SFULL + 2;
     static constexpr int B_PVDONE = B_PFULL + 2;
-    static constexpr int B_LFREE = B_PVDONE + 2;
-    static constexpr int B_KINC = B_LFREE + 2;
+    static constexpr int B_LREAD = B_PVDONE + 2;  // correction has read O's l column for the tile
+    static constexpr int B_KINC = B_LREAD + 2;
     static constexpr int B_MMADONE = B_KINC + 4;
     static constexpr int NBAR = B_MMADONE + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
     // TMEM columns
-    static constexpr int O_COL = 0;
-    static constexpr int S_COL0 = D;
-    static constexpr int L_COL0 = D + 2 * BK;
-    static constexpr int TMEM_USED = D + 2 * BK + 32;
+    static constexpr int S_COL0 = 0;
+    static constexpr int O_COL = 2 * BK;
+    static constexpr int L_COL = O_COL + D;  // running row sum l
+    static constexpr int Q_COL = O_COL + D + 16;
+    static constexpr int P_COL0 = Q_COL + D / 4;
+    static constexpr int TMEM_USED = P_COL0 + 2 * (BK / 4);
     static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
     static_assert(TMEM_USED <= 512, "TMEM budget");
-    static_assert((Q_BYTES % 1024) == 0 && (K_BYTES % 1024) == 0 && (P_BYTES % 1024) == 0 &&
-                      (ONES_BYTES % 1024) == 0,
-                  "swizzled tiles stay 1024-byte aligned");
+    static_assert((K_BYTES % 1024) == 0 && (VX_BYTES % 1024) == 0, "swizzled tiles stay 1024-byte aligned");
 };
 
 __device__ __forceinline__ float exp2_neg_int(int k) {
@@ -101,9 +103,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, const 
 }
 
 template <int D, int BK>
-__global__ void __launch_bounds__(320, 1)
-    vc_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
+__global__ void __launch_bounds__(576, 1)
+    vc_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const AttnArgs args) {
     using Cfg = AttnCfg<D, BK>;
     constexpr int STAGES = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -125,21 +127,20 @@ __global__ void __launch_bounds__(320, 1)
 
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
-        mbar_init(bar(Cfg::B_QFULL), 1);
+        mbar_init(bar(Cfg::B_QREADY), 8);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar(Cfg::B_KFULL + s), 1);
             mbar_init(bar(Cfg::B_KEMPTY + s), 1);
             mbar_init(bar(Cfg::B_VFULL + s), 1);
-            mbar_init(bar(Cfg::B_VEMPTY + s), 1 + 4);
+            mbar_init(bar(Cfg::B_VEMPTY + s), 1 + 8);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(Cfg::B_SFULL + i), 1);
-            mbar_init(bar(Cfg::B_SFREE + i), 4);
-            mbar_init(bar(Cfg::B_PFULL + i), 4);
+            mbar_init(bar(Cfg::B_PFULL + i), 8);
             mbar_init(bar(Cfg::B_PVDONE + i), 1);
-            mbar_init(bar(Cfg::B_LFREE + i), 4);
+            mbar_init(bar(Cfg::B_LREAD + i), 8);
         }
-        for (int i = 0; i < 4; ++i) mbar_init(bar(Cfg::B_KINC + i), 4);
+        for (int i = 0; i < 4; ++i) mbar_init(bar(Cfg::B_KINC + i), 8);
         mbar_init(bar(Cfg::B_MMADONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -148,10 +149,11 @@ __global__ void __launch_bounds__(320, 1)
         tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
         tmem_relinquish();
     }
-    {  // the constant "ones" B operand of the row-sum MMA: every byte is E4M3 1.0
-        uint4* ones = reinterpret_cast<uint4*>(smem + Cfg::OFF_ONES);
+    {  // rows D..D+15 of every V stage: E4M3 1.0, so the PV MMA also sums P
         const uint4 v = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
-        for (int i = threadIdx.x; i < Cfg::ONES_BYTES / 16; i += Cfg::THREADS) ones[i] = v;
+        constexpr int PER = 16 * BK / 16;  // uint4 per stage
+        for (int i = threadIdx.x; i < STAGES * PER; i += Cfg::THREADS)
+            reinterpret_cast<uint4*>(smem + Cfg::OFF_V + (i / PER) * Cfg::VX_BYTES + Cfg::V_BYTES)[i % PER] = v;
         fence_proxy_async_smem();
     }
     tc_fence_before();
@@ -163,11 +165,8 @@ __global__ void __launch_bounds__(320, 1)
     if (warp == 0) {
         // -------------------------------------------------------- producer
         if (lane == 0) {
-            prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_expect_tx_arrive(bar(Cfg::B_QFULL), Cfg::Q_BYTES);
-            tma_load_3d(base + Cfg::OFF_Q, &tm_q, bar(Cfg::B_QFULL), 0, q0, bh);
             int issued_k = 0, issued_v = 0;
             for (int t = 0; t < T; ++t) {
                 const int st = t % STAGES;
@@ -178,14 +177,13 @@ __global__ void __launch_bounds__(320, 1)
                 issued_k = t + 1;
                 if (n > 0 && !mbar_wait(bar(Cfg::B_VEMPTY + st), (n - 1) & 1, ctl, abort_flag)) break;
                 mbar_expect_tx_arrive(bar(Cfg::B_VFULL + st), Cfg::V_BYTES + Cfg::MU_BYTES);
-                tma_load_3d(base + Cfg::OFF_V + st * Cfg::V_BYTES, &tm_v, bar(Cfg::B_VFULL + st), t * BK, 0, bh);
+                tma_load_3d(base + Cfg::OFF_V + st * Cfg::VX_BYTES, &tm_v, bar(Cfg::B_VFULL + st), t * BK, 0, bh);
                 bulk_load(base + Cfg::OFF_MU + st * Cfg::MU_BYTES, args.v_mean + ((size_t)bh * T + t) * D,
                           Cfg::MU_BYTES, bar(Cfg::B_VFULL + st));
                 issued_v = t + 1;
             }
             // Drain: every copy issued has landed before the CTA may exit.  Only
             // the last STAGES tiles of each ring can still be in flight.
-            drain_wait(bar(Cfg::B_QFULL), 0, ctl);
             for (int t = issued_k - STAGES < 0 ? 0 : issued_k - STAGES; t < issued_k; ++t)
                 drain_wait(bar(Cfg::B_KFULL + t % STAGES), (t / STAGES) & 1, ctl);
             for (int t = issued_v - STAGES < 0 ? 0 : issued_v - STAGES; t < issued_v; ++t)
@@ -193,62 +191,82 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t id_qk = idesc_e4m3_f32(BK);
-            const uint32_t id_pv = idesc_e4m3_f32(D);
-            const uint32_t id_l = idesc_e4m3_f32(16);
-            const uint64_t dq = smem_desc(base + Cfg::OFF_Q, D);
-            const uint64_t dones = smem_desc(base + Cfg::OFF_ONES, BK);
-            bool ok = mbar_wait(bar(Cfg::B_QFULL), 0, ctl, abort_flag);
-            auto issue_qk = [&](int t) -> bool {
-                const int st = t % STAGES, sb = t & 1;
-                if (!mbar_wait(bar(Cfg::B_KFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
-                if (t >= 2 && !mbar_wait(bar(Cfg::B_SFREE + sb), ((t - 2) >> 1) & 1, ctl, abort_flag)) return false;
-                tc_fence_after();
-                const uint64_t dk = smem_desc(base + Cfg::OFF_K + st * Cfg::K_BYTES, D);
+        // The whole warp runs the loop (warp-uniform operands); one elected
+        // lane issues each MMA and commit.  S buffer (t+2)%2 is free once the
+        // softmax has posted P(t): it reads S(t) before it writes P(t), and
+        // QK(t+2) is issued after this warp waited for p_full(t).
+        const uint32_t id_qk = idesc_e4m3_f32(BK);
+        const uint32_t id_pv = idesc_e4m3_f32(D + 16);
+        bool ok = warp_wait(bar(Cfg::B_QREADY), 0, ctl, abort_flag);
+        auto issue_qk = [&](int t) -> bool {
+            const int st = t % STAGES, sb = t & 1;
+            if (!warp_wait(bar(Cfg::B_KFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
+            tc_fence_after();
+            const uint64_t dk = smem_desc(base + Cfg::OFF_K + st * Cfg::K_BYTES, D);
 #pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk)
-                    mma_f8(tmem + Cfg::S_COL0 + sb * BK, dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0);
-                mma_commit(bar(Cfg::B_SFULL + sb));
-                mma_commit(bar(Cfg::B_KEMPTY + st));
-                return true;
-            };
-            auto issue_pv = [&](int t) -> bool {
-                const int st = t % STAGES, pb = t & 1;
-                if (!mbar_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
-                if (!mbar_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
-                if (t >= 2 && !mbar_wait(bar(Cfg::B_LFREE + pb), ((t - 2) >> 1) & 1, ctl, abort_flag)) return false;
-                tc_fence_after();
-                const uint64_t dp = smem_desc(base + Cfg::OFF_P + pb * Cfg::P_BYTES, BK);
-                const uint64_t dv = smem_desc(base + Cfg::OFF_V + st * Cfg::V_BYTES, BK);
+            for (int kk = 0; kk < D / 32; ++kk)
+                mma_f8_ts_warp(tmem + Cfg::S_COL0 + sb * BK, tmem + Cfg::Q_COL + 8 * kk, dk + 2 * kk, id_qk, kk > 0);
+            mma_commit_warp(bar(Cfg::B_SFULL + sb));
+            mma_commit_warp(bar(Cfg::B_KEMPTY + st));
+            return true;
+        };
+        auto issue_pv = [&](int t) -> bool {
+            const int st = t % STAGES, pb = t & 1;
+            if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
+            if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
+            tc_fence_after();
+            const uint32_t ap = tmem + Cfg::P_COL0 + pb * (BK / 4);
+            const uint64_t dv = smem_desc(base + Cfg::OFF_V + st * Cfg::VX_BYTES, BK);
 #pragma unroll
-                for (int kk = 0; kk < BK / 32; ++kk)
-                    mma_f8(tmem + Cfg::O_COL, dp + 2 * kk, dv + 2 * kk, id_pv, (t > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < BK / 32; ++kk)
-                    mma_f8(tmem + Cfg::L_COL0 + 16 * pb, dp + 2 * kk, dones + 2 * kk, id_l, kk > 0);
-                mma_commit(bar(Cfg::B_PVDONE + pb));
-                mma_commit(bar(Cfg::B_VEMPTY + st));
-                return true;
-            };
-            if (ok) ok = issue_qk(0);
-            for (int t = 0; ok && t < T; ++t) {
-                if (t + 1 < T && !issue_qk(t + 1)) break;
-                if (!issue_pv(t)) break;
-            }
-            mma_commit(bar(Cfg::B_MMADONE));
-            drain_wait(bar(Cfg::B_MMADONE), 0, ctl);
+            for (int kk = 0; kk < BK / 32; ++kk)
+                mma_f8_ts_warp(tmem + Cfg::O_COL, ap + 8 * kk, dv + 2 * kk, id_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_warp(bar(Cfg::B_PVDONE + pb));
+            mma_commit_warp(bar(Cfg::B_VEMPTY + st));
+            return true;
+        };
+        if (ok) ok = issue_qk(0);
+        for (int t = 0; ok && t < T; ++t) {
+            if (t + 1 < T && !issue_qk(t + 1)) break;
+            if (!issue_pv(t)) break;
         }
-    } else if (warp < 6) {
+        mma_commit_warp(bar(Cfg::B_MMADONE));
+        drain_wait(bar(Cfg::B_MMADONE), 0, ctl);
+    } else if (warp < 10) {
         // -------------------------------------------------------- softmax
+        // Two warps per TMEM lane quadrant: warp (qd, hf) handles rows
+        // 32qd..32qd+31, score columns [hf*BK/2, (hf+1)*BK/2).  The pair
+        // exchanges half-row maxima through shared memory.
+        constexpr int HB = BK / 2;
+        constexpr int HD = D / 2;
         const int qd = warp & 3;
+        const int hf = (warp - 2) >> 2;
         const int row = qd * 32 + lane;
         const uint32_t lane_tmem = tmem + ((uint32_t)(qd * 32) << 16);
         const int qrow = q0 + row;
+        {   // this warp's half of the row's E4M3 Q into TMEM (zeros past N)
+            uint32_t qw[HD / 4];
+            const uint4* src = reinterpret_cast<const uint4*>(args.q_fp8 + ((size_t)bh * N + qrow) * D + hf * HD);
+#pragma unroll
+            for (int i = 0; i < HD / 16; ++i) {
+                const uint4 v = qrow < N ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+                qw[4 * i + 0] = v.x;
+                qw[4 * i + 1] = v.y;
+                qw[4 * i + 2] = v.z;
+                qw[4 * i + 3] = v.w;
+            }
+            if constexpr (HD / 4 == 16)
+                tmem_st16(lane_tmem + Cfg::Q_COL + hf * (HD / 4), qw);
+            else
+                tmem_st8(lane_tmem + Cfg::Q_COL + hf * (HD / 4), qw);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(Cfg::B_QREADY));
+        }
         const float sqv = qrow < N ? args.sq[(size_t)bh * N + qrow] : 0.0f;
         const float aq = __fmul_rn(args.kappa, sqv);
         const float c0 = 56.0f + (float)args.beta;
-        uint8_t* pbuf = smem + Cfg::OFF_P;
+        float* mx_ex = reinterpret_cast<float*>(smem + Cfg::OFF_MXEX);  // [tile parity][half][row]
         float M = 0.0f;
         float sk_next = args.k_scale[(size_t)bh * T];
         for (int t = 0; t < T; ++t) {
@@ -257,69 +275,79 @@ __global__ void __launch_bounds__(320, 1)
             if (t + 1 < T) sk_next = args.k_scale[(size_t)bh * T + t + 1];
             if (!warp_wait(bar(Cfg::B_SFULL + sb), (t >> 1) & 1, ctl, abort_flag)) break;
             tc_fence_after();
-            float s[BK];
+            float s[HB];
 #pragma unroll
-            for (int c = 0; c < BK / 32; ++c) tmem_ld32(lane_tmem + Cfg::S_COL0 + sb * BK + 32 * c, s + 32 * c);
+            for (int c = 0; c < HB / 32; ++c)
+                tmem_ld32(lane_tmem + Cfg::S_COL0 + sb * BK + hf * HB + 32 * c, s + 32 * c);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(Cfg::B_SFREE + sb));
 
-            const int valid = N - t * BK;
-            if (valid < BK) {
+            const int valid = N - t * BK - hf * HB;
+            if (valid < HB) {
 #pragma unroll
-                for (int j = 0; j < BK; ++j)
+                for (int j = 0; j < HB; ++j)
                     if (j >= valid) s[j] = -INFINITY;
             }
-            // row max: 8 independent 3-input max chains, then a short tree
+            // half-row max: 8 independent 3-input max chains, then a short tree
             float m8[8];
 #pragma unroll
             for (int a = 0; a < 8; ++a) m8[a] = fmaxf(s[2 * a], s[2 * a + 1]);
 #pragma unroll
-            for (int j = 16; j < BK; j += 16)
+            for (int j = 16; j < HB; j += 16)
 #pragma unroll
                 for (int a = 0; a < 8; ++a) m8[a] = fmax3(m8[a], s[j + 2 * a], s[j + 2 * a + 1]);
-            const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+            const float mh =
+                fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+            mx_ex[((t & 1) * 2 + hf) * Cfg::BM + row] = mh;
+            named_barrier_sync(1 + qd, 64);
+            const float mx = fmaxf(mh, mx_ex[((t & 1) * 2 + (1 - hf)) * Cfg::BM + row]);
             const float A = __fmul_rn(aq, sk);
             const float Mc = ceilf(__fmul_rn(__fmul_rn(A, mx), 0.125f));
             const float Mnew = t == 0 ? Mc : fmaxf(M, Mc);
             const int kinc = t == 0 ? 0 : (int)(Mnew - M);
             M = Mnew;
             const float cbm = (c0 - 8.0f * M) + kMagic;
-            // P buffer sb was last read by the PV MMA of tile t-2.
-            if (t >= 2 && !warp_wait(bar(Cfg::B_PVDONE + sb), ((t - 2) >> 1) & 1, ctl, abort_flag)) break;
-            uint8_t* prow = pbuf + sb * Cfg::P_BYTES;
+            uint32_t pw[HB / 4];
 #pragma unroll
-            for (int ch = 0; ch < BK / 16; ++ch) {
-                uint32_t w[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int j = ch * 16 + q * 4;
-                    const float2 t01 = expcast_t2(A, s[j], s[j + 1], cbm);
-                    const float2 t23 = expcast_t2(A, s[j + 2], s[j + 3], cbm);
-                    w[q] = pack4_low_bytes(t01.x, t01.y, t23.x, t23.y);
-                }
-                *reinterpret_cast<uint4*>(prow + swz_offset(row, ch, BK)) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int q = 0; q < HB / 4; ++q) {
+                const float2 t01 = expcast_t2(A, s[4 * q], s[4 * q + 1], cbm);
+                const float2 t23 = expcast_t2(A, s[4 * q + 2], s[4 * q + 3], cbm);
+                pw[q] = pack4_low_bytes(t01.x, t01.y, t23.x, t23.y);
             }
+            // P slot sb was last read by the PV MMA of tile t-2.
+            if (t >= 2 && !warp_wait(bar(Cfg::B_PVDONE + sb), ((t - 2) >> 1) & 1, ctl, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t pcol = lane_tmem + Cfg::P_COL0 + sb * (BK / 4) + hf * (HB / 4);
+            if constexpr (HB / 4 == 16)
+                tmem_st16(pcol, pw);
+            else
+                tmem_st8(pcol, pw);
             if (t > 0 && __any_sync(0xffffffffu, kinc > 0)) {
-                // O holds PV of tiles < t: wait for it, then scale by 2^-kinc
-                // (before this tile's PV, which waits on p_full below).
+                // O holds PV of tiles < t: wait for it, then scale this warp's
+                // half of the O columns by 2^-kinc (before this tile's PV,
+                // which waits on p_full below).
                 if (!warp_wait(bar(Cfg::B_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) break;
+                // ... and for the correction warps to have read l after PV(t-1)
+                if (!warp_wait(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) break;
                 tc_fence_after();
                 const float f = exp2_neg_int(kinc);
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
                     float o[32];
-                    tmem_ld32(lane_tmem + Cfg::O_COL + 32 * c, o);
+                    tmem_ld32(lane_tmem + Cfg::O_COL + hf * HD + 32 * c, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= f;
-                    tmem_st32(lane_tmem + Cfg::O_COL + 32 * c, o);
+                    tmem_st32(lane_tmem + Cfg::O_COL + hf * HD + 32 * c, o);
                 }
-                tmem_wait_st();
+                if (hf == 1) {  // the running row sum l, column D
+                    float lv = tmem_ld1(lane_tmem + Cfg::L_COL);
+                    tmem_wait_ld();
+                    lv *= f;
+                    tmem_st1(lane_tmem + Cfg::L_COL, lv);
+                }
             }
-            fence_proxy_async_smem();
-            kinc_ring[(t & 3) * Cfg::BM + row] = kinc;
+            tmem_wait_st();
+            if (hf == 0) kinc_ring[(t & 3) * Cfg::BM + row] = kinc;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -329,14 +357,18 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else {
         // -------------------------------------------------------- correction + epilogue
+        // Two warps per lane quadrant: warp (qd, hf) owns output channels
+        // [hf*D/2, (hf+1)*D/2) of rows 32qd..32qd+31.
+        constexpr int HD = D / 2;
         const int qd = warp & 3;
+        const int hf = (warp - 10) >> 2;
         const int row = qd * 32 + lane;
         const uint32_t lane_tmem = tmem + ((uint32_t)(qd * 32) << 16);
         const int qrow = q0 + row;
-        float acc[D];
+        float acc[HD];
 #pragma unroll
-        for (int c = 0; c < D; ++c) acc[c] = 0.0f;
-        float l = 0.0f;
+        for (int c = 0; c < HD; ++c) acc[c] = 0.0f;
+        float l = 0.0f;  // running row sum after the last tile seen
         bool ok = true;
         for (int t = 0; t < T; ++t) {
             const int st = t % STAGES;
@@ -344,21 +376,26 @@ __global__ void __launch_bounds__(320, 1)
             const int kinc = kinc_ring[(t & 3) * Cfg::BM + row];
             if (!(ok = warp_wait(bar(Cfg::B_PVDONE + (t & 1)), (t >> 1) & 1, ctl, abort_flag))) break;
             tc_fence_after();
-            const float lb = tmem_ld1(lane_tmem + Cfg::L_COL0 + 16 * (t & 1));
+            const float lt = tmem_ld1(lane_tmem + Cfg::L_COL);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(Cfg::B_LFREE + (t & 1)));
+            if (lane == 0) mbar_arrive(bar(Cfg::B_LREAD + (t & 1)));
             if (!(ok = warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag))) break;
+            float lb;
             if (kinc > 0) {
                 const float f = exp2_neg_int(kinc);
 #pragma unroll
-                for (int c = 0; c < D; ++c) acc[c] *= f;
-                l *= f;
+                for (int c = 0; c < HD; ++c) acc[c] *= f;
+                lb = lt - l * f;
+            } else {
+                lb = lt - l;
             }
-            const float4* mu = reinterpret_cast<const float4*>(smem + Cfg::OFF_MU + st * Cfg::MU_BYTES);
+            l = lt;
+            const float4* mu =
+                reinterpret_cast<const float4*>(smem + Cfg::OFF_MU + st * Cfg::MU_BYTES) + hf * (HD / 4);
 #pragma unroll
-            for (int c4 = 0; c4 < D / 4; ++c4) {
+            for (int c4 = 0; c4 < HD / 4; ++c4) {
                 const float4 m = mu[c4];
                 const float2 a01 = ffma2(make_float2(lb, lb), make_float2(m.x, m.y),
                                          make_float2(acc[4 * c4 + 0], acc[4 * c4 + 1]));
@@ -369,7 +406,6 @@ __global__ void __launch_bounds__(320, 1)
                 acc[4 * c4 + 2] = a23.x;
                 acc[4 * c4 + 3] = a23.y;
             }
-            l += lb;
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(Cfg::B_VEMPTY + st));
         }
@@ -377,27 +413,26 @@ __global__ void __launch_bounds__(320, 1)
             // The last PV (tile T-1) has completed, so O is final.
             tc_fence_after();
             const float inv_l = 1.0f / l;
-            const float* vsc = args.v_scale + (size_t)bh * D;
-            __nv_bfloat16* orow = args.out + ((size_t)bh * N + qrow) * D;
+            const float* vsc = args.v_scale + (size_t)bh * D + hf * HD;
+            __nv_bfloat16* orow = args.out + ((size_t)bh * N + qrow) * D + hf * HD;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                float o[32];
-                tmem_ld32(lane_tmem + Cfg::O_COL + 32 * c, o);
+            for (int c = 0; c < HD / 16; ++c) {
+                float o[16];
+                tmem_ld16(lane_tmem + Cfg::O_COL + hf * HD + 16 * c, o);
                 tmem_wait_ld();
-                uint32_t packed[16];
+                uint32_t packed[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int c0i = 32 * c + 2 * i;
+                for (int i = 0; i < 8; ++i) {
+                    const int c0i = 16 * c + 2 * i;
                     const float x0 = (vsc[c0i] * o[2 * i] + acc[c0i]) * inv_l;
                     const float x1 = (vsc[c0i + 1] * o[2 * i + 1] + acc[c0i + 1]) * inv_l;
                     const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
                     packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
                 if (qrow < N) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
+                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                 }
             }
         }
@@ -415,8 +450,8 @@ __global__ void __launch_bounds__(320, 1)
 
 // ---------------------------------------------------------------- host side
 template <int D, int BK>
-cudaError_t launch_attn_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
-                          int BH, cudaStream_t stream) {
+cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int BH,
+                          cudaStream_t stream) {
     using Cfg = AttnCfg<D, BK>;
     static bool configured = false;
     if (!configured) {
@@ -426,16 +461,16 @@ cudaError_t launch_attn_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
         configured = true;
     }
     dim3 grid((a.N + Cfg::BM - 1) / Cfg::BM, BH);
-    vc_attn_kernel<D, BK><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+    vc_attn_kernel<D, BK><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tk, tv, a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_attn(int D, int BK, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnArgs& a, int BH, cudaStream_t stream) {
-    if (D == 128 && BK == 128) return launch_attn_t<128, 128>(tq, tk, tv, a, BH, stream);
-    if (D == 128 && BK == 64) return launch_attn_t<128, 64>(tq, tk, tv, a, BH, stream);
-    if (D == 64 && BK == 128) return launch_attn_t<64, 128>(tq, tk, tv, a, BH, stream);
-    if (D == 64 && BK == 64) return launch_attn_t<64, 64>(tq, tk, tv, a, BH, stream);
+cudaError_t launch_attn(int D, int BK, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int BH,
+                        cudaStream_t stream) {
+    if (D == 128 && BK == 128) return launch_attn_t<128, 128>(tk, tv, a, BH, stream);
+    if (D == 128 && BK == 64) return launch_attn_t<128, 64>(tk, tv, a, BH, stream);
+    if (D == 64 && BK == 128) return launch_attn_t<64, 128>(tk, tv, a, BH, stream);
+    if (D == 64 && BK == 64) return launch_attn_t<64, 64>(tk, tv, a, BH, stream);
     return cudaErrorInvalidValue;
 }
 

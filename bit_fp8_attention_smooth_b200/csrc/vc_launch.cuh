@@ -7,6 +7,7 @@
 namespace vc {
 
 struct AttnArgs {
+    const uint8_t* q_fp8;  // [BH, N, D] E4M3 Q
     const float* sq;       // [BH, N] per-token Q scale
     const float* k_scale;  // [BH, T]
     const float* v_mean;   // [BH, T, D]
@@ -40,6 +41,7 @@ struct PrepLaunch {
     __nv_bfloat16* c_hi;  // [BH, Cp, D] centroid high bf16 part
     __nv_bfloat16* c_lo;  // [BH, Cp, D] centroid residual bf16 part
     float* cnorm;         // [BH, Cp] squared centroid norms
+    double* cent64;       // [BH, C, D] fp64 centroids (the exact near-tie decision)
     double* sums;
     int32_t* cstart;
     int32_t* ccount;
@@ -55,8 +57,8 @@ struct PrepLaunch {
 bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t d0,
                   uint64_t d1, uint64_t d2, uint32_t box0, uint32_t box1);
 
-cudaError_t launch_attn(int D, int BK, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnArgs& a, int BH, cudaStream_t stream);
+cudaError_t launch_attn(int D, int BK, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int BH,
+                        cudaStream_t stream);
 cudaError_t launch_prep(const PrepLaunch& p, cudaStream_t s);
 cudaError_t launch_quant_q(const __nv_bfloat16* Q, uint8_t* q_fp8, float* sq, int64_t tokens, int D,
                            cudaStream_t s);

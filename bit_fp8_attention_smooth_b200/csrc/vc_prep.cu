@@ -52,8 +52,9 @@ __device__ __forceinline__ float block_sum_d(float x, float* red) {
 }
 
 __global__ void km_init(const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ c_hi,
-                        __nv_bfloat16* __restrict__ c_lo, float* __restrict__ cnorm, double* __restrict__ sums,
-                        KmState* __restrict__ state, uint32_t* __restrict__ vamax, int N, int C, int Cp, int D) {
+                        __nv_bfloat16* __restrict__ c_lo, float* __restrict__ cnorm, double* __restrict__ cent64,
+                        double* __restrict__ sums, KmState* __restrict__ state, uint32_t* __restrict__ vamax, int N,
+                        int C, int Cp, int D) {
     __shared__ float red[4];
     const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
     const size_t row = ((size_t)bh * Cp + k) * D + c;
@@ -62,6 +63,7 @@ __global__ void km_init(const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __re
         const int64_t src = ((int64_t)k * N) / C;
         x = bf2f(V[((size_t)bh * N + src) * D + c]);
         sums[((size_t)bh * C + k) * D + c] = 0.0;
+        cent64[((size_t)bh * C + k) * D + c] = (double)x;
     }
     c_hi[row] = __float2bfloat16_rn(x);
     c_lo[row] = __float2bfloat16_rn(0.0f);
@@ -82,7 +84,8 @@ template <int D>
 __global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtensorMap tm_v,
                                                  const __grid_constant__ CUtensorMap tm_chi,
                                                  const __grid_constant__ CUtensorMap tm_clo,
-                                                 const float* __restrict__ cnorm, int32_t* __restrict__ labels,
+                                                 const float* __restrict__ cnorm, const double* __restrict__ cent64,
+                                                 const __nv_bfloat16* __restrict__ V, int32_t* __restrict__ labels,
                                                  int32_t* __restrict__ hist, KmState* __restrict__ state, int N, int C,
                                                  int Cp, int it, DevCtl ctl) {
     constexpr int A_BYTES = KM_TOK * D * 2;
@@ -156,7 +159,8 @@ __global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtenso
     if (ok && !*abort_flag) {
         tc_fence_after();
         const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
-        float best = INFINITY;
+        // pass 1: tensor-core distances |c|^2 - 2 v.c; best and runner-up
+        float best = INFINITY, second = INFINITY;
         int bestk = 0;
         for (int k0 = 0; k0 < Cp; k0 += 16) {
             float dot[16];
@@ -166,11 +170,102 @@ __global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtenso
             for (int j = 0; j < 16; ++j) {
                 const int k = k0 + j;
                 const float dist = cn_s[k] - 2.0f * dot[j];
-                if (k < C && dist < best) {
-                    best = dist;
-                    bestk = k;
+                if (k < C) {
+                    if (dist < best) {
+                        second = best;
+                        best = dist;
+                        bestk = k;
+                    } else if (dist < second) {
+                        second = dist;
+                    }
                 }
             }
+        }
+        // Error bound of the tensor-core distance: bf16 hi/lo centroids carry
+        // 2^-18 relative error and the fp32 accumulation at most 2^-15 of
+        // sum |v_c c_c|, so |err| <= 2^-14 (|v| + |c|)^2.  Candidates within
+        // the margin are decided again in fp64, exactly as the Lloyd step
+        // defines the distance (sum over channels, in order, of (v - c)^2).
+        float vn2 = 0.0f;
+        {
+            const uint8_t* arow = smem + tid * 128;
+#pragma unroll
+            for (int kc = 0; kc < D / 64; ++kc)
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 raw = *reinterpret_cast<const uint4*>(arow + kc * (KM_TOK * 128) + ((ch ^ (tid & 7)) << 4));
+                    const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) vn2 = fmaf(bf2f(hv[e]), bf2f(hv[e]), vn2);
+                }
+        }
+        float cmax2 = 0.0f;
+        for (int k = 0; k < C; ++k) cmax2 = fmaxf(cmax2, cn_s[k]);
+        const float rad = sqrtf(vn2) + sqrtf(cmax2);
+        const float margin = ldexpf(rad * rad, -12);
+        const bool valid_tok = n0 + tid < N;
+        const bool refine = valid_tok && C > 1 && (second - best) <= margin;
+        if (__any_sync(0xffffffffu, refine)) {
+            // The warp evaluates each candidate of each refining lane together:
+            // every lane sums (v - c)^2 over D/32 channels in fp64, then a
+            // butterfly adds the lanes.  Candidates go in ascending k with a
+            // strict comparison, so ties keep the lowest k.
+            constexpr int CPL = D / 32;  // channels per lane
+            const int lane = tid & 31;
+            const float lim = best + margin;
+            double dbest = INFINITY;
+            int kbest = bestk;
+            for (int k0 = 0; k0 < Cp; k0 += 16) {
+                float dot[16];
+                tmem_ld16(lane_tmem + k0, dot);
+                tmem_wait_ld();
+                uint32_t cm = 0;
+                if (refine) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (k0 + j < C && cn_s[k0 + j] - 2.0f * dot[j] <= lim) cm |= 1u << j;
+                }
+                uint32_t lanes = __ballot_sync(0xffffffffu, cm != 0);
+                while (lanes) {
+                    const int src = __ffs(lanes) - 1;
+                    lanes &= lanes - 1;
+                    uint32_t m = __shfl_sync(0xffffffffu, cm, src);
+                    const int r = warp * 32 + src;  // the source lane's token row in the tile
+                    const int c0 = lane * CPL;
+                    const uint8_t* vp = smem + (c0 / 64) * (KM_TOK * 128) + r * 128 +
+                                        ((((c0 % 64) / 8) ^ (r & 7)) << 4) + (c0 % 8) * 2;
+                    float vx[CPL];
+                    if constexpr (CPL == 4) {
+                        const uint2 raw = *reinterpret_cast<const uint2*>(vp);
+                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) vx[e] = bf2f(hv[e]);
+                    } else {
+                        const uint32_t raw = *reinterpret_cast<const uint32_t*>(vp);
+                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                        for (int e = 0; e < CPL; ++e) vx[e] = bf2f(hv[e]);
+                    }
+                    while (m) {
+                        const int k = k0 + __ffs(m) - 1;
+                        m &= m - 1;
+                        const double* crow = cent64 + ((size_t)bh * C + k) * D + c0;
+                        double part = 0.0;
+#pragma unroll
+                        for (int e = 0; e < CPL; ++e) {
+                            const double diff = __dsub_rn((double)vx[e], crow[e]);
+                            part = __dadd_rn(part, __dmul_rn(diff, diff));
+                        }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+                        if (lane == src && part < dbest) {
+                            dbest = part;
+                            kbest = k;
+                        }
+                    }
+                }
+            }
+            if (refine) bestk = kbest;
         }
         if (n0 + tid < N) {
             int32_t* lp = labels + (size_t)bh * N + n0 + tid;
@@ -284,18 +379,23 @@ __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict
 }
 
 __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __restrict__ c_lo,
-                            float* __restrict__ cnorm, double* __restrict__ sums, const int32_t* __restrict__ ccount,
-                            const KmState* __restrict__ state, int C, int Cp, int D) {
+                            float* __restrict__ cnorm, double* __restrict__ cent64, double* __restrict__ sums,
+                            const int32_t* __restrict__ ccount, const KmState* __restrict__ state, int C, int Cp,
+                            int D) {
     __shared__ float red[4];
     const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
     if (state[bh].done) return;
     const int cnt = ccount[(size_t)bh * C + k];
     if (cnt == 0) return;  // an empty cluster keeps its centroid (sums are still 0)
     double* sp = &sums[((size_t)bh * C + k) * D + c];
-    const float x = (float)(*sp / (double)cnt);
+    const double mean = *sp / (double)cnt;  // the fp64 member mean (the sum of bf16 values is exact)
     *sp = 0.0;
+    cent64[((size_t)bh * C + k) * D + c] = mean;
     const size_t row = ((size_t)bh * Cp + k) * D + c;
-    store_centroid(x, c_hi + row, c_lo + row);
+    const __nv_bfloat16 h = __double2bfloat16(mean);
+    c_hi[row] = h;
+    c_lo[row] = __double2bfloat16(mean - (double)__bfloat162float(h));
+    const float x = (float)mean;
     const float nrm = block_sum_d(x * x, red);
     if (c == 0) cnorm[(size_t)bh * Cp + k] = nrm;
 }
@@ -482,17 +582,18 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
         !make_tmap_3d(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.c_hi, D, Cp, p.BH, 64, Cp) ||
         !make_tmap_3d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.c_lo, D, Cp, p.BH, 64, Cp))
         return cudaErrorInvalidValue;
-    km_init<<<dim3(Cp, p.BH), D, 0, s>>>(p.V, p.c_hi, p.c_lo, p.cnorm, p.sums, p.state, p.vamax, p.N, p.C, Cp, D);
+    km_init<<<dim3(Cp, p.BH), D, 0, s>>>(p.V, p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.state, p.vamax, p.N, p.C,
+                                         Cp, D);
     for (int it = 0; it < p.iters; ++it) {
-        km_assign<D><<<dim3(nblk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.labels, p.hist, p.state, p.N, p.C,
-                                                          Cp, it, p.ctl);
+        km_assign<D><<<dim3(nblk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.labels, p.hist,
+                                                          p.state, p.N, p.C, Cp, it, p.ctl);
         km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it);
         km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C);
         if (it + 1 < p.iters) {
             km_update<D><<<dim3(p.C, KM_SLICES, p.BH), 128, 0, s>>>(p.V, p.perm, p.cstart, p.ccount, p.sums, p.state,
                                                                     p.N, p.C);
-            km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.sums, p.ccount, p.state, p.C, Cp,
-                                                      D);
+            km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.ccount, p.state,
+                                                      p.C, Cp, D);
         }
     }
     return cudaGetLastError();
