@@ -31,7 +31,8 @@
 //                epilogue O = (v_scale * O + acc) / l in bf16, original token
 //                order.
 // Every wait is bounded (DevCtl); on a timeout the CTA drains its copies and
-// MMAs, frees TMEM and exits with the status word set.
+// MMAs, frees TMEM and exits with the status word set.  A CTA does nothing
+// when the status word already holds an error.
 #include "vc_launch.cuh"
 
 namespace vc {
@@ -50,7 +51,8 @@ struct AttnCfg {
     static constexpr int OFF_MU = OFF_V + STAGES * VX_BYTES;
     static constexpr int OFF_KINC = OFF_MU + STAGES * MU_BYTES;
     static constexpr int OFF_MXEX = OFF_KINC + 4 * BM * 4;
-    static constexpr int OFF_BAR = OFF_MXEX + 2 * 2 * BM * 4;
+    static constexpr int OFF_PAIRCNT = OFF_MXEX + 2 * 2 * BM * 4;  // pair-barrier arrivals per softmax warp
+    static constexpr int OFF_BAR = OFF_PAIRCNT + 8 * 4;
     // barrier slots
     static constexpr int B_QREADY = 0;
     static constexpr int B_KFULL = 1;
@@ -95,7 +97,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, const DevCtl& ctl) {
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
-        if ((int64_t)(globaltimer() - t0) > ctl.limit_ns) {
+        if ((int64_t)(globaltimer() - t0) > kDrainNs) {
             record_error(ctl, VC_ERR_DEVICE_TIMEOUT);
             return;
         }
@@ -108,6 +110,8 @@ __global__ void __launch_bounds__(576, 1)
                    const AttnArgs args) {
     using Cfg = AttnCfg<D, BK>;
     constexpr int STAGES = Cfg::STAGES;
+    // The prep outputs are undefined after a recorded device error.
+    if (ctl_failed(args.ctl.status)) return;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -161,6 +165,7 @@ __global__ void __launch_bounds__(576, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const DevCtl ctl = args.ctl;
+    int pair_arrivals = 0;  // softmax warps: arrivals on the pair's named barrier
 
     if (warp == 0) {
         // -------------------------------------------------------- producer
@@ -269,7 +274,9 @@ __global__ void __launch_bounds__(576, 1)
         float* mx_ex = reinterpret_cast<float*>(smem + Cfg::OFF_MXEX);  // [tile parity][half][row]
         float M = 0.0f;
         float sk_next = args.k_scale[(size_t)bh * T];
+        bool done = true;
         for (int t = 0; t < T; ++t) {
+            done = false;
             const int sb = t & 1;
             const float sk = sk_next;
             if (t + 1 < T) sk_next = args.k_scale[(size_t)bh * T + t + 1];
@@ -279,6 +286,9 @@ __global__ void __launch_bounds__(576, 1)
 #pragma unroll
             for (int c = 0; c < HB / 32; ++c)
                 tmem_ld32(lane_tmem + Cfg::S_COL0 + sb * BK + hf * HB + 32 * c, s + 32 * c);
+            // read after this warp's last pair barrier, in the shadow of the
+            // TMEM load: enough to stop before the next one (below)
+            const int abort_seen = *abort_flag;
             tmem_wait_ld();
 
             const int valid = N - t * BK - hf * HB;
@@ -298,7 +308,15 @@ __global__ void __launch_bounds__(576, 1)
             const float mh =
                 fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
             mx_ex[((t & 1) * 2 + hf) * Cfg::BM + row] = mh;
+            // The pair meets on named barrier 1 + qd.  A warp never enters it
+            // once it has seen the CTA abort (its partner may have left); a
+            // warp that leaves early arrives once more instead, which frees a
+            // partner already waiting there (see the teardown for the balance).
+            // An abort that frees a waiting partner is visible to it through
+            // the barrier, so the partner stops before its next meeting.
+            if (__any_sync(0xffffffffu, abort_seen != 0)) break;
             named_barrier_sync(1 + qd, 64);
+            ++pair_arrivals;
             const float mx = fmaxf(mh, mx_ex[((t & 1) * 2 + (1 - hf)) * Cfg::BM + row]);
             const float A = __fmul_rn(aq, sk);
             const float Mc = ceilf(__fmul_rn(__fmul_rn(A, mx), 0.125f));
@@ -354,6 +372,11 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive(bar(Cfg::B_PFULL + sb));
                 mbar_arrive(bar(Cfg::B_KINC + (t & 3)));
             }
+            done = true;
+        }
+        if (!done) {
+            named_barrier_arrive(1 + qd, 64);
+            ++pair_arrivals;
         }
     } else {
         // -------------------------------------------------------- correction + epilogue
@@ -439,8 +462,17 @@ __global__ void __launch_bounds__(576, 1)
     }
 
     // ------------------------------------------------------------ teardown
+    int* pair_cnt = reinterpret_cast<int*>(smem + Cfg::OFF_PAIRCNT);
+    if (warp >= 2 && warp < 10) {
+        tmem_wait_st();  // an aborted softmax warp may hold a pending store
+        if (lane == 0) pair_cnt[warp - 2] = pair_arrivals;
+    }
     tc_fence_before();
     __syncthreads();
+    // After an abort one generation of a pair barrier may hold a single
+    // warp's arrival: complete it, so no barrier is left half-way.
+    if (warp >= 2 && warp < 6 && ((pair_cnt[warp - 2] + pair_cnt[warp + 2]) & 1))
+        named_barrier_arrive(1 + (warp & 3), 64);
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();

@@ -29,6 +29,14 @@ __device__ __forceinline__ void record_error(const DevCtl& ctl, int code) {
     atomicCAS(ctl.status, 0, code);
 }
 
+// True, for every thread of the CTA, when an earlier kernel on the same
+// workspace recorded a device error: its outputs are undefined, so a kernel
+// that would index memory with them does nothing instead.  Call at the top of
+// the kernel, by all threads.
+__device__ __forceinline__ bool ctl_failed(const int* status) {
+    return __syncthreads_or(threadIdx.x == 0 && *reinterpret_cast<const volatile int*>(status) != 0) != 0;
+}
+
 // ---------------------------------------------------------------- smem
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -62,6 +70,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+
+// Bound on draining a CTA's own in-flight copies and MMAs after an abort; it
+// does not depend on the (possibly tiny) wait limit.
+constexpr int64_t kDrainNs = 2000000000LL;
 
 // Waits for the phase of parity `parity` to complete.  Gives up when the CTA
 // abort flag is raised by another warp, or after ctl.limit_ns, in which case
@@ -106,6 +118,10 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 // Barrier `id` (1..15) over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void named_barrier_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core).
@@ -318,11 +334,17 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 // One FMA per score: t = A*s + cbm with cbm = cb + 1.5*2^23 (cb an integer,
-// |cb| < 2^22); the max clamps negative t to 0; the byte is in the low 8 bits.
-// Scores go in pairs through the packed FMA.
+// |cb| < 2^22) rounds A*s + cb to the integer n in t's low mantissa bits.  The
+// clamp n -> max(n, 0) stays on the FMA pipe and is exact:
+// sat(t * 2^-23 - 1.5) = max(n, 0) * 2^-23 (saturation also sends -inf and
+// NaN to 0), and w * 2^23 + 1.5*2^23 puts max(n, 0) back into the low bits.
+// The byte is the low 8 bits.  Scores go in pairs through the packed FMA.
 __device__ __forceinline__ float2 expcast_t2(float A, float s0, float s1, float cbm) {
     const float2 t = ffma2(make_float2(A, A), make_float2(s0, s1), make_float2(cbm, cbm));
-    return make_float2(fmaxf(t.x, kMagic), fmaxf(t.y, kMagic));
+    float w0, w1;
+    asm("fma.rn.sat.f32 %0, %1, 0f34000000, 0fBFC00000;" : "=f"(w0) : "f"(t.x));
+    asm("fma.rn.sat.f32 %0, %1, 0f34000000, 0fBFC00000;" : "=f"(w1) : "f"(t.y));
+    return ffma2(make_float2(w0, w1), make_float2(8388608.0f, 8388608.0f), make_float2(kMagic, kMagic));
 }
 __device__ __forceinline__ uint32_t pack4_low_bytes(float a, float b, float c, float d) {
     const uint32_t lo = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);

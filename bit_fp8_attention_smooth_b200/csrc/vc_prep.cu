@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtenso
                                                  int Cp, int it, DevCtl ctl) {
     constexpr int A_BYTES = KM_TOK * D * 2;
     const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x;
-    if (state[bh].done) return;  // uniform over the CTA, before any barrier or TMEM use
+    // both uniform over the CTA, before any barrier or TMEM use
+    if (ctl_failed(ctl.status) || state[bh].done) return;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -276,10 +277,14 @@ __global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtenso
     }
     changed = __reduce_add_sync(0xffffffffu, changed);
     if ((tid & 31) == 0 && changed) atomicAdd(&state[bh].changed, changed);
-    // The load barrier may still be pending after an abort: let the copies land.
+    // After an abort the copies and MMAs of thread 0 may still be in flight:
+    // let them land before TMEM and shared memory are released.  Thread 0
+    // always committed bar_mma, so both barriers complete.
     if (tid == 0 && !ok) {
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(bar_ld, 0) && (int64_t)(globaltimer() - t0) < ctl.limit_ns) {
+        while (!mbar_try_wait(bar_ld, 0) && (int64_t)(globaltimer() - t0) < kDrainNs) {
+        }
+        while (!mbar_try_wait(bar_mma, 0) && (int64_t)(globaltimer() - t0) < kDrainNs) {
         }
     }
     tc_fence_before();
@@ -295,9 +300,11 @@ __global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtenso
 // Exclusive scan of hist[bh] in (cluster, block) order -> offs; cluster ranges.
 __global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist, int32_t* __restrict__ offs,
                                                 int32_t* __restrict__ cstart, int32_t* __restrict__ ccount,
-                                                KmState* __restrict__ state, int N, int C, int nblk, int it) {
+                                                KmState* __restrict__ state, int N, int C, int nblk, int it,
+                                                const int* __restrict__ status) {
     __shared__ int s_part[1024];
     __shared__ int s_skip;
+    if (ctl_failed(status)) return;
     const int bh = blockIdx.x, tid = threadIdx.x;
     if (tid == 0) {
         int skip = state[bh].done;
@@ -341,10 +348,11 @@ __global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist
 
 __global__ void __launch_bounds__(KM_TOK) km_scatter(const int32_t* __restrict__ labels,
                                                      const int32_t* __restrict__ offs, int32_t* __restrict__ perm,
-                                                     const KmState* __restrict__ state, int N, int C) {
+                                                     const KmState* __restrict__ state, int N, int C,
+                                                     const int* __restrict__ status) {
     __shared__ int lab_s[KM_TOK];
     const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x, r = threadIdx.x;
-    if (state[bh].done) return;
+    if (ctl_failed(status) || state[bh].done) return;
     const int j = blk * KM_TOK + r;
     const int L = j < N ? labels[(size_t)bh * N + j] : -1;
     lab_s[r] = L;
@@ -361,9 +369,10 @@ template <int D>
 __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ perm,
                                                  const int32_t* __restrict__ cstart,
                                                  const int32_t* __restrict__ ccount, double* __restrict__ sums,
-                                                 const KmState* __restrict__ state, int N, int C) {
+                                                 const KmState* __restrict__ state, int N, int C,
+                                                 const int* __restrict__ status) {
     const int k = blockIdx.x, sl = blockIdx.y, bh = blockIdx.z;
-    if (state[bh].done) return;
+    if (ctl_failed(status) || state[bh].done) return;
     const int cnt = ccount[(size_t)bh * C + k];
     if (cnt == 0) return;
     const int st = cstart[(size_t)bh * C + k];
@@ -381,10 +390,10 @@ __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict
 __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __restrict__ c_lo,
                             float* __restrict__ cnorm, double* __restrict__ cent64, double* __restrict__ sums,
                             const int32_t* __restrict__ ccount, const KmState* __restrict__ state, int C, int Cp,
-                            int D) {
+                            int D, const int* __restrict__ status) {
     __shared__ float red[4];
     const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-    if (state[bh].done) return;
+    if (ctl_failed(status) || state[bh].done) return;
     const int cnt = ccount[(size_t)bh * C + k];
     if (cnt == 0) return;  // an empty cluster keeps its centroid (sums are still 0)
     double* sp = &sums[((size_t)bh * C + k) * D + c];
@@ -411,12 +420,13 @@ __global__ void __launch_bounds__(128) prep_kv_block(const __nv_bfloat16* __rest
                                                      const int32_t* __restrict__ perm, int smooth,
                                                      uint8_t* __restrict__ k_fp8, float* __restrict__ k_scale,
                                                      float* __restrict__ v_mean, uint32_t* __restrict__ vamax, int N,
-                                                     int T) {
+                                                     int T, const int* __restrict__ status) {
     constexpr int RG = 128 / D;  // row groups
     __shared__ int tok_s[BK];
     __shared__ double vsum_s[RG][D];
     __shared__ float kmax_s[128];
     __shared__ float vmax_s[RG][D];
+    if (ctl_failed(status)) return;  // perm is undefined
     const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int c = tid % D, rg = tid / D;
     const int valid = min(BK, N - b * BK);
@@ -481,11 +491,13 @@ __global__ void __launch_bounds__(128) prep_v_quant(const __nv_bfloat16* __restr
                                                     const int32_t* __restrict__ perm, int smooth,
                                                     const float* __restrict__ v_mean,
                                                     const uint32_t* __restrict__ vamax, uint8_t* __restrict__ vt_fp8,
-                                                    float* __restrict__ v_scale, int N, int T) {
+                                                    float* __restrict__ v_scale, int N, int T,
+                                                    const int* __restrict__ status) {
     constexpr int RG = 128 / D;
     constexpr int STRIDE = BK + 4;  // bytes per channel row in smem (conflict-free word stores)
     __shared__ int tok_s[BK];
     __shared__ uint32_t cs[D * STRIDE / 4];
+    if (ctl_failed(status)) return;  // perm is undefined
     const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int c = tid % D, rg = tid / D;
     const int valid = min(BK, N - b * BK);
@@ -587,13 +599,15 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     for (int it = 0; it < p.iters; ++it) {
         km_assign<D><<<dim3(nblk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.labels, p.hist,
                                                           p.state, p.N, p.C, Cp, it, p.ctl);
-        km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it);
-        km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C);
+        km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it,
+                                      p.ctl.status);
+        km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C,
+                                                       p.ctl.status);
         if (it + 1 < p.iters) {
             km_update<D><<<dim3(p.C, KM_SLICES, p.BH), 128, 0, s>>>(p.V, p.perm, p.cstart, p.ccount, p.sums, p.state,
-                                                                    p.N, p.C);
+                                                                    p.N, p.C, p.ctl.status);
             km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.ccount, p.state,
-                                                      p.C, Cp, D);
+                                                      p.C, Cp, D, p.ctl.status);
         }
     }
     return cudaGetLastError();
@@ -610,9 +624,9 @@ static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     prep_kv_block<D, BK><<<dim3(T, p.BH), 128, 0, s>>>(p.K, p.V, p.perm, p.smooth, p.k_fp8, p.k_scale, p.v_mean,
-                                                       p.vamax, p.N, T);
+                                                       p.vamax, p.N, T, p.ctl.status);
     prep_v_quant<D, BK><<<dim3(T, p.BH), 128, 0, s>>>(p.V, p.perm, p.smooth, p.v_mean, p.vamax, p.vt_fp8, p.v_scale,
-                                                      p.N, T);
+                                                      p.N, T, p.ctl.status);
     return cudaGetLastError();
 }
 

@@ -28,8 +28,11 @@
  *   - Return values: VC_OK, or an error code.  Argument errors are detected on
  *     the host before any launch.  Launch failures return VC_ERR_CUDA.
  *     A kernel whose internal wait exceeds params->wait_limit_ns records
- *     VC_ERR_DEVICE_TIMEOUT in the workspace status word, stops cleanly and
- *     leaves its outputs undefined; vc_check reports it.
+ *     VC_ERR_DEVICE_TIMEOUT in the workspace status word, lets its own copies
+ *     and tensor-core work land, frees its tensor memory and returns; its
+ *     outputs are undefined.  While the status word holds an error, every
+ *     later kernel that reads the workspace returns without work (its outputs
+ *     stay as they were) until vc_check reports and clears the error.
  *
  * Shapes: B batches, H heads, N tokens, head dim d (64 or 128).  The hardware
  * block is `block` tokens (64 or 128) and equals the key/value tile of the
