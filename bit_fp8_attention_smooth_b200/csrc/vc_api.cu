@@ -20,7 +20,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct WsLayout {
     // offsets in bytes from the workspace base
     size_t status;
-    size_t labels, c_hi, c_lo, cnorm, cent64, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
+    size_t labels, c_hi, c_lo, cnorm, cent64, vnorm2, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
     size_t qfp8, sq;                                                      // attention region (aliases prep)
     size_t prep_end, attn_end, total;
 };
@@ -38,6 +38,7 @@ WsLayout ws_layout(const vc_shape& s, const vc_params& p) {
     w.c_lo = o; o = align256(o + 2 * BH * Cp * D);
     w.cnorm = o; o = align256(o + 4 * BH * Cp);
     w.cent64 = o; o = align256(o + 8 * BH * C * D);
+    w.vnorm2 = o; o = align256(o + 4 * BH * N);
     w.sums = o; o = align256(o + 8 * BH * C * D);
     w.cstart = o; o = align256(o + 4 * BH * C);
     w.ccount = o; o = align256(o + 4 * BH * C);
@@ -135,9 +136,10 @@ vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc
     pl.c_lo = reinterpret_cast<__nv_bfloat16*>(ws + L.c_lo);
     pl.cnorm = reinterpret_cast<float*>(ws + L.cnorm);
     pl.cent64 = reinterpret_cast<double*>(ws + L.cent64);
+    pl.vnorm2 = reinterpret_cast<float*>(ws + L.vnorm2);
+    pl.sums = reinterpret_cast<double*>(ws + L.sums);
     pl.ctl.status = reinterpret_cast<int*>(ws + L.status);
     pl.ctl.limit_ns = p.wait_limit_ns > 0 ? p.wait_limit_ns : kDefaultWaitNs;
-    pl.sums = reinterpret_cast<double*>(ws + L.sums);
     pl.cstart = reinterpret_cast<int32_t*>(ws + L.cstart);
     pl.ccount = reinterpret_cast<int32_t*>(ws + L.ccount);
     pl.hist = reinterpret_cast<int32_t*>(ws + L.hist);

@@ -42,7 +42,8 @@ struct PrepLaunch {
     __nv_bfloat16* c_lo;  // [BH, Cp, D] centroid residual bf16 part
     float* cnorm;         // [BH, Cp] squared centroid norms
     double* cent64;       // [BH, C, D] fp64 centroids (the exact near-tie decision)
-    double* sums;
+    double* sums;         // [BH, C, D] fp64 member sums of the Lloyd update
+    float* vnorm2;        // [BH, N] |v|^2 of every token (bounds the tensor-core distance error)
     int32_t* cstart;
     int32_t* ccount;
     int32_t* hist;

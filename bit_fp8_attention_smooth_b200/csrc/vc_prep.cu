@@ -13,7 +13,7 @@
 //             km_scan         exclusive scan -> stable positions; a head whose labels
 //                             did not change is final (its later passes would repeat)
 //             km_scatter      perm[position] = token (stable within a cluster)
-//             km_update       fp64 member sums over each cluster's contiguous range
+//             km_update       fp64 member sums over fixed slices of the stable order
 //             km_finalize     c_k = sum / count (empty clusters keep c_k)
 //   prep_kv_block             per block: K amax scale + E4M3 K, V block mean (fp64 sum),
 //                             residual channel amax
@@ -75,42 +75,71 @@ __global__ void km_init(const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __re
     }
 }
 
-constexpr int KM_TOK = 128;  // tokens per assign block (the MMA's M)
+constexpr int KM_TOK = 128;  // tokens per tile (the MMA's M)
 
-// Assignment pass on tensor cores: one CTA = 128 tokens of one head.
+// Shared-memory plan of km_assign, from a 1024-byte aligned base:
+//   V tile x2 | centroid hi | centroid lo | |c|^2 | histograms x2 | scratch | barriers
+constexpr int KM_PCAP = 64;  // near-tie (token, candidate) pairs a warp decides together
+
+struct KmLayout {
+    uint32_t v_bytes, c_bytes, off_v, off_chi, off_clo, off_cn, off_hist, off_pk, off_red, off_bar, off_misc, bytes;
+    __host__ __device__ KmLayout(int D, int Cp) {
+        v_bytes = KM_TOK * D * 2;
+        c_bytes = Cp * D * 2;
+        off_v = 0;
+        off_chi = 2 * v_bytes;
+        off_clo = off_chi + c_bytes;
+        off_cn = off_clo + c_bytes;            // [256] |c_k|^2
+        off_hist = off_cn + 256 * 4;           // [2][256] per-tile cluster counts
+        off_pk = off_hist + 2 * 256 * 4;       // [4 warps][KM_PCAP] near-tie pairs
+        off_red = off_pk + 4 * KM_PCAP * 4;
+        off_bar = off_red + 64;
+        off_misc = off_bar + 64;
+        bytes = off_misc + 16 + 1024;  // + alignment slack
+    }
+};
+
+// Assignment pass on tensor cores.  One CTA takes `tpc` consecutive 128-token
+// tiles of one head; the centroids are loaded once, the V tiles stream through
+// a double buffer, and the MMA of tile j+1 runs while the CUDA cores finish
+// tile j:
 //   S[token, k] = v . c_hi + v . c_lo   (kind::f16, bf16 x bf16 -> fp32 in TMEM)
-//   label = argmin_k (|c_k|^2 - 2 S[token, k]), ties to the lowest k.
+//   label = argmin_k (|c_k|^2 - 2 S[token, k]), ties to the lowest k,
+// with near-ties decided again in fp64.  Per tile: labels, the per-cluster
+// histogram of the tile (for the stable regroup) and the change count.
 template <int D>
-__global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtensorMap tm_v,
+__global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUtensorMap tm_v,
                                                  const __grid_constant__ CUtensorMap tm_chi,
                                                  const __grid_constant__ CUtensorMap tm_clo,
                                                  const float* __restrict__ cnorm, const double* __restrict__ cent64,
-                                                 const __nv_bfloat16* __restrict__ V, int32_t* __restrict__ labels,
-                                                 int32_t* __restrict__ hist, KmState* __restrict__ state, int N, int C,
-                                                 int Cp, int it, DevCtl ctl) {
-    constexpr int A_BYTES = KM_TOK * D * 2;
-    const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x;
+                                                 const __nv_bfloat16* __restrict__ V, float* __restrict__ vnorm2,
+                                                 int32_t* __restrict__ labels, int32_t* __restrict__ hist,
+                                                 KmState* __restrict__ state, int N, int C, int Cp, int it, int tpc,
+                                                 DevCtl ctl) {
+    const int bh = blockIdx.y, nblk = (N + KM_TOK - 1) / KM_TOK;
+    const int blk0 = blockIdx.x * tpc;
+    const int nt = min(tpc, nblk - blk0);
     // both uniform over the CTA, before any barrier or TMEM use
-    if (ctl_failed(ctl.status) || state[bh].done) return;
+    if (ctl_failed(ctl.status) || state[bh].done || nt <= 0) return;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
-    const int B_BYTES = Cp * D * 2;
-    const uint32_t sA = base, sBh = base + A_BYTES, sBl = sBh + B_BYTES;
-    float* cn_s = reinterpret_cast<float*>(smem + A_BYTES + 2 * B_BYTES);
-    int* hist_s = reinterpret_cast<int*>(cn_s + 256);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(hist_s + 256);  // [0] loads, [1] mma
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int n0 = blk * KM_TOK;
-    const uint32_t ncols = Cp <= 32 ? 32 : (Cp <= 64 ? 64 : (Cp <= 128 ? 128 : 256));
-    const uint32_t bar_ld = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
+    const KmLayout L(D, Cp);
+    float* cn_s = reinterpret_cast<float*>(smem + L.off_cn);
+    int* hist_s = reinterpret_cast<int*>(smem + L.off_hist);  // [2][256]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.off_misc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc + 4);
+    const uint32_t bar_c = base + L.off_bar, bar_v0 = bar_c + 8, bar_mma0 = bar_c + 24;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t ncols = 2 * Cp <= 32 ? 32 : (2 * Cp <= 64 ? 64 : (2 * Cp <= 128 ? 128 : (2 * Cp <= 256 ? 256 : 512)));
 
     if (tid == 0) {
-        mbar_init(bar_ld, 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(bar_c, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_v0 + 8 * i, 1);
+            mbar_init(bar_mma0 + 8 * i, 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -118,178 +147,294 @@ __global__ void __launch_bounds__(128) km_assign(const __grid_constant__ CUtenso
         tmem_alloc(smem_u32(tmem_slot), ncols);
         tmem_relinquish();
     }
-    for (int k = tid; k < Cp; k += 128) cn_s[k] = cnorm[(size_t)bh * Cp + k];
-    for (int k = tid; k < C; k += 128) hist_s[k] = 0;
+    // |c_k|^2 (pad clusters +inf, never chosen) and max_k |c_k|^2 of the head
+    uint32_t* red_s = reinterpret_cast<uint32_t*>(smem + L.off_red);
+    uint32_t cmax_bits = 0;
+    for (int k = tid; k < Cp; k += 128) {
+        const float x = k < C ? cnorm[(size_t)bh * Cp + k] : INFINITY;
+        cn_s[k] = x;
+        if (k < C) cmax_bits = max(cmax_bits, __float_as_uint(x));  // x >= 0: bit order is value order
+    }
+    cmax_bits = __reduce_max_sync(0xffffffffu, cmax_bits);
+    if (lane == 0) red_s[warp] = cmax_bits;
+    for (int k = tid; k < 2 * 256; k += 128) hist_s[k] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const float cmax_r = sqrtf(__uint_as_float(max(max(red_s[0], red_s[1]), max(red_s[2], red_s[3]))));
 
+    const uint32_t sV = base + L.off_v, sCh = base + L.off_chi, sCl = base + L.off_clo;
+    auto load_v = [&](int j) {  // thread 0
+        const uint32_t b = j & 1, bar = bar_v0 + 8 * b;
+        mbar_expect_tx_arrive(bar, L.v_bytes);
+#pragma unroll
+        for (int kc = 0; kc < D / 64; ++kc)
+            tma_load_3d(sV + b * L.v_bytes + kc * (KM_TOK * 128), &tm_v, bar, 64 * kc, (blk0 + j) * KM_TOK, bh);
+    };
+    const uint32_t idesc = idesc_bf16_f32(Cp);
+    auto issue_mma = [&](int j) {  // thread 0, after V tile j (and the centroids) landed
+        const uint32_t b = j & 1;
+        const uint32_t sA = sV + b * L.v_bytes, acc = tmem + b * Cp;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            mma_bf16(acc, smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128),
+                     smem_desc(sCh + (kk >> 2) * (Cp * 128) + off, 128), idesc, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            mma_bf16(acc, smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128),
+                     smem_desc(sCl + (kk >> 2) * (Cp * 128) + off, 128), idesc, 1u);
+        }
+        mma_commit(bar_mma0 + 8 * b);
+    };
+
+    int v_issued = 0, mma_issued = 0;  // thread 0's in-flight bookkeeping
     bool ok = true;
     if (tid == 0) {
-        mbar_expect_tx_arrive(bar_ld, A_BYTES + 2 * B_BYTES);
+        mbar_expect_tx_arrive(bar_c, 2 * L.c_bytes);
 #pragma unroll
         for (int kc = 0; kc < D / 64; ++kc) {
-            tma_load_3d(sA + kc * (KM_TOK * 128), &tm_v, bar_ld, 64 * kc, n0, bh);
-            tma_load_3d(sBh + kc * (Cp * 128), &tm_chi, bar_ld, 64 * kc, 0, bh);
-            tma_load_3d(sBl + kc * (Cp * 128), &tm_clo, bar_ld, 64 * kc, 0, bh);
+            tma_load_3d(sCh + kc * (Cp * 128), &tm_chi, bar_c, 64 * kc, 0, bh);
+            tma_load_3d(sCl + kc * (Cp * 128), &tm_clo, bar_c, 64 * kc, 0, bh);
         }
-        ok = mbar_wait(bar_ld, 0, ctl, abort_flag);
+        load_v(0);
+        v_issued = 1;
+        if (nt > 1) {
+            load_v(1);
+            v_issued = 2;
+        }
+        ok = mbar_wait(bar_c, 0, ctl, abort_flag) && mbar_wait(bar_v0, 0, ctl, abort_flag);
         if (ok) {
-            tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(Cp);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk & 3) * 32;
-                const uint64_t da = smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128);
-                const uint64_t dh = smem_desc(sBh + (kk >> 2) * (Cp * 128) + off, 128);
-                mma_bf16(tmem, da, dh, idesc, kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk & 3) * 32;
-                const uint64_t da = smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128);
-                const uint64_t dl = smem_desc(sBl + (kk >> 2) * (Cp * 128) + off, 128);
-                mma_bf16(tmem, da, dl, idesc, 1u);
-            }
+            issue_mma(0);
+            mma_issued = 1;
         }
-        mma_commit(bar_mma);  // also covers the case of no MMA issued
     }
-    ok = __all_sync(0xffffffffu, mbar_wait(bar_mma, 0, ctl, abort_flag));
     int changed = 0;
-    if (ok && !*abort_flag) {
+    for (int j = 0; j < nt; ++j) {
+        const int b = j & 1;
+        const int n0 = (blk0 + j) * KM_TOK;
+        if (j >= 1) {  // the previous tile's histogram is complete (barrier below)
+            int* hp = hist_s + (b ^ 1) * 256;
+            for (int k = tid; k < C; k += 128) {
+                hist[((size_t)bh * C + k) * nblk + blk0 + j - 1] = hp[k];
+                hp[k] = 0;
+            }
+        }
+        if (tid == 0 && ok && j + 1 < nt) {  // MMA j+1 into the other accumulator, read out by tile j-1
+            ok = mbar_wait(bar_v0 + 8 * (b ^ 1), ((j + 1) >> 1) & 1, ctl, abort_flag);
+            if (ok) {
+                issue_mma(j + 1);
+                mma_issued = j + 2;
+            }
+        }
+        bool okj = __all_sync(0xffffffffu, ok && mbar_wait(bar_mma0 + 8 * b, (j >> 1) & 1, ctl, abort_flag));
         tc_fence_after();
-        const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
-        // pass 1: tensor-core distances |c|^2 - 2 v.c; best and runner-up
-        float best = INFINITY, second = INFINITY;
-        int bestk = 0;
-        for (int k0 = 0; k0 < Cp; k0 += 16) {
-            float dot[16];
-            tmem_ld16(lane_tmem + k0, dot);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int k = k0 + j;
-                const float dist = cn_s[k] - 2.0f * dot[j];
-                if (k < C) {
-                    if (dist < best) {
-                        second = best;
-                        best = dist;
-                        bestk = k;
-                    } else if (dist < second) {
-                        second = dist;
-                    }
-                }
-            }
-        }
-        // Error bound of the tensor-core distance: bf16 hi/lo centroids carry
-        // 2^-18 relative error and the fp32 accumulation at most 2^-15 of
-        // sum |v_c c_c|, so |err| <= 2^-14 (|v| + |c|)^2.  Candidates within
-        // the margin are decided again in fp64, exactly as the Lloyd step
-        // defines the distance (sum over channels, in order, of (v - c)^2).
+        const int n = n0 + tid;
+        const bool valid = n < N;
         float vn2 = 0.0f;
-        {
-            const uint8_t* arow = smem + tid * 128;
+        if (it == 0) {  // |v|^2 once per prep, from the V tile before it is overwritten
+            if (okj) {
+                const uint8_t* arow = smem + L.off_v + b * L.v_bytes + tid * 128;
 #pragma unroll
-            for (int kc = 0; kc < D / 64; ++kc)
+                for (int kc = 0; kc < D / 64; ++kc)
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(arow + kc * (KM_TOK * 128) + ((ch ^ (tid & 7)) << 4));
-                    const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) vn2 = fmaf(bf2f(hv[e]), bf2f(hv[e]), vn2);
-                }
-        }
-        float cmax2 = 0.0f;
-        for (int k = 0; k < C; ++k) cmax2 = fmaxf(cmax2, cn_s[k]);
-        const float rad = sqrtf(vn2) + sqrtf(cmax2);
-        const float margin = ldexpf(rad * rad, -12);
-        const bool valid_tok = n0 + tid < N;
-        const bool refine = valid_tok && C > 1 && (second - best) <= margin;
-        if (__any_sync(0xffffffffu, refine)) {
-            // The warp evaluates each candidate of each refining lane together:
-            // every lane sums (v - c)^2 over D/32 channels in fp64, then a
-            // butterfly adds the lanes.  Candidates go in ascending k with a
-            // strict comparison, so ties keep the lowest k.
-            constexpr int CPL = D / 32;  // channels per lane
-            const int lane = tid & 31;
-            const float lim = best + margin;
-            double dbest = INFINITY;
-            int kbest = bestk;
-            for (int k0 = 0; k0 < Cp; k0 += 16) {
-                float dot[16];
-                tmem_ld16(lane_tmem + k0, dot);
-                tmem_wait_ld();
-                uint32_t cm = 0;
-                if (refine) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (k0 + j < C && cn_s[k0 + j] - 2.0f * dot[j] <= lim) cm |= 1u << j;
-                }
-                uint32_t lanes = __ballot_sync(0xffffffffu, cm != 0);
-                while (lanes) {
-                    const int src = __ffs(lanes) - 1;
-                    lanes &= lanes - 1;
-                    uint32_t m = __shfl_sync(0xffffffffu, cm, src);
-                    const int r = warp * 32 + src;  // the source lane's token row in the tile
-                    const int c0 = lane * CPL;
-                    const uint8_t* vp = smem + (c0 / 64) * (KM_TOK * 128) + r * 128 +
-                                        ((((c0 % 64) / 8) ^ (r & 7)) << 4) + (c0 % 8) * 2;
-                    float vx[CPL];
-                    if constexpr (CPL == 4) {
-                        const uint2 raw = *reinterpret_cast<const uint2*>(vp);
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 raw =
+                            *reinterpret_cast<const uint4*>(arow + kc * (KM_TOK * 128) + ((ch ^ (tid & 7)) << 4));
                         const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) vx[e] = bf2f(hv[e]);
-                    } else {
-                        const uint32_t raw = *reinterpret_cast<const uint32_t*>(vp);
-                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-                        for (int e = 0; e < CPL; ++e) vx[e] = bf2f(hv[e]);
+                        for (int e = 0; e < 8; ++e) vn2 = fmaf(bf2f(hv[e]), bf2f(hv[e]), vn2);
                     }
-                    while (m) {
-                        const int k = k0 + __ffs(m) - 1;
-                        m &= m - 1;
-                        const double* crow = cent64 + ((size_t)bh * C + k) * D + c0;
-                        double part = 0.0;
+                if (valid) vnorm2[(size_t)bh * N + n] = vn2;
+            }
+            __syncthreads();
+        } else if (okj && valid) {
+            vn2 = vnorm2[(size_t)bh * N + n];
+        }
+        if (tid == 0 && okj && j + 2 < nt) {  // MMA j has read V buffer b
+            load_v(j + 2);
+            v_issued = j + 3;
+        }
+        if (okj) {
+            const uint32_t lane_tmem = tmem + b * Cp + ((uint32_t)(warp * 32) << 16);
+            // Pass 1: best and runner-up of the tensor-core distances
+            // d_k = |c_k|^2 - 2 v.c_k.  With Cp <= 64 the distances stay in
+            // registers for the near-tie masks below.
+            float best = INFINITY, second = INFINITY;
+            int bestk = 0;
+            float dk[64];
+            for (int g = 0; g < Cp; g += 64) {
 #pragma unroll
-                        for (int e = 0; e < CPL; ++e) {
-                            const double diff = __dsub_rn((double)vx[e], crow[e]);
-                            part = __dadd_rn(part, __dmul_rn(diff, diff));
-                        }
+                for (int q = 0; q < 4; ++q)
+                    if (g + 16 * q < Cp) tmem_ld16(lane_tmem + g + 16 * q, dk + 16 * q);
+                tmem_wait_ld();
 #pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
-                        if (lane == src && part < dbest) {
-                            dbest = part;
-                            kbest = k;
+                for (int q4 = 0; q4 < 16; ++q4) {
+                    if (g + 4 * q4 < Cp) {
+                        const float4 cn = reinterpret_cast<const float4*>(cn_s + g)[q4];
+                        const float cv[4] = {cn.x, cn.y, cn.z, cn.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float d = fmaf(-2.0f, dk[4 * q4 + e], cv[e]);
+                            dk[4 * q4 + e] = d;
+                            const bool lt = d < best;
+                            second = fminf(second, fmaxf(best, d));
+                            best = fminf(best, d);
+                            bestk = lt ? g + 4 * q4 + e : bestk;
                         }
                     }
                 }
             }
-            if (refine) bestk = kbest;
+            // Error bound of the tensor-core distance: bf16 hi/lo centroids carry
+            // 2^-16 relative error, the products are exact and the fp32
+            // accumulation of the 2 D products errs by at most 2^-15 of
+            // sum |v_c c_c|, so |err| <= 2^-14 (|v| + max|c|)^2 with room to
+            // spare.  Clusters within twice that of the best are decided again
+            // in fp64 from the fp64 centroids, as the Lloyd step defines the
+            // distance (sum over channels of (v - c)^2).
+            const float rad = sqrtf(vn2) + cmax_r;
+            const float margin = ldexpf(rad * rad, -12);
+            const bool refine = valid && C > 1 && (second - best) <= margin;
+            if (__any_sync(0xffffffffu, refine)) {
+                int* pk = reinterpret_cast<int*>(smem + L.off_pk) + warp * KM_PCAP;
+                const float lim = best + margin;
+                double dbest = INFINITY;
+                int kbest = bestk;
+                for (int g = 0; g < Cp; g += 64) {
+                    if (Cp > 64) {  // the group's distances again, from TMEM
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)  // warp-collective: every lane loads
+                            if (g + 16 * q < Cp) tmem_ld16(lane_tmem + g + 16 * q, dk + 16 * q);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int jj = 0; jj < 64; ++jj)
+                            if (g + jj < Cp) dk[jj] = fmaf(-2.0f, dk[jj], cn_s[g + jj]);
+                    }
+                    uint32_t m0 = 0, m1 = 0;  // candidates g..g+31 and g+32..g+63
+                    if (refine) {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            if (g + jj < Cp && dk[jj] <= lim) m0 |= 1u << jj;
+                            if (g + 32 + jj < Cp && dk[32 + jj] <= lim) m1 |= 1u << jj;
+                        }
+                    }
+                    const int cnt = __popc(m0) + __popc(m1);
+                    int incl = cnt;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += t;
+                    }
+                    const int total = __shfl_sync(0xffffffffu, incl, 31);
+                    // The warp's (lane, cluster) pairs, lane by lane and in
+                    // ascending k, KM_PCAP at a time.
+                    for (int base = 0; base < total; base += KM_PCAP) {
+                        int p = incl - cnt;
+                        for (int h = 0; h < 2; ++h)
+                            for (uint32_t m = h ? m1 : m0; m; m &= m - 1, ++p)
+                                if (p >= base && p < base + KM_PCAP)
+                                    pk[p - base] = (lane << 16) | (g + 32 * h + __ffs(m) - 1);
+                        __syncwarp();
+                        const int np = min(KM_PCAP, total - base);
+                        // Each pair's distance is computed by the whole warp (D/32
+                        // channels a lane, then a butterfly), four pairs at a time
+                        // with all their loads issued first.
+                        constexpr int CPL = D / 32;
+                        const int c0 = lane * CPL;
+                        for (int q0 = 0; q0 < np; q0 += 4) {
+                            float vx[4][CPL];
+                            double cx[4][CPL];
+                            int pid[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                pid[u] = q0 + u < np ? pk[q0 + u] : -1;
+                                if (pid[u] >= 0) {
+                                    const int t = pid[u] >> 16, k = pid[u] & 0xFFFF;
+                                    const __nv_bfloat16* vp = V + ((size_t)bh * N + n0 + warp * 32 + t) * D + c0;
+                                    const double* cp = cent64 + ((size_t)bh * C + k) * D + c0;
+                                    if constexpr (CPL == 4) {
+                                        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(vp));
+                                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+                                        const double2 a = __ldg(reinterpret_cast<const double2*>(cp));
+                                        const double2 b2 = __ldg(reinterpret_cast<const double2*>(cp) + 1);
+#pragma unroll
+                                        for (int e = 0; e < 4; ++e) vx[u][e] = bf2f(hv[e]);
+                                        cx[u][0] = a.x;
+                                        cx[u][1] = a.y;
+                                        cx[u][2] = b2.x;
+                                        cx[u][3] = b2.y;
+                                    } else {
+                                        const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(vp));
+                                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+                                        const double2 a = __ldg(reinterpret_cast<const double2*>(cp));
+#pragma unroll
+                                        for (int e = 0; e < CPL; ++e) vx[u][e] = bf2f(hv[e]);
+                                        cx[u][0] = a.x;
+                                        cx[u][CPL - 1] = a.y;
+                                    }
+                                }
+                            }
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                if (pid[u] < 0) break;  // uniform: pid comes from shared memory
+                                double part = 0.0;
+#pragma unroll
+                                for (int e = 0; e < CPL; ++e) {
+                                    const double diff = __dsub_rn((double)vx[u][e], cx[u][e]);
+                                    part = __dadd_rn(part, __dmul_rn(diff, diff));
+                                }
+#pragma unroll
+                                for (int o = 16; o > 0; o >>= 1)
+                                    part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+                                // strict: of equal distances the lowest k stays
+                                if (lane == (pid[u] >> 16) && part < dbest) {
+                                    dbest = part;
+                                    kbest = pid[u] & 0xFFFF;
+                                }
+                            }
+                        }
+                        __syncwarp();
+                    }
+                }
+                if (refine) bestk = kbest;
+            }
+            const int label = bestk;
+            if (valid) {
+                int32_t* lp = labels + (size_t)bh * N + n;
+                if (it == 0 || *lp != label) ++changed;
+                *lp = label;
+                atomicAdd(&hist_s[b * 256 + label], 1);
+            }
         }
-        if (n0 + tid < N) {
-            int32_t* lp = labels + (size_t)bh * N + n0 + tid;
-            if (it == 0 || *lp != bestk) changed = 1;
-            *lp = bestk;
-            atomicAdd(&hist_s[bestk], 1);
-        }
+        tc_fence_before();
+        ok = __syncthreads_and(okj) != 0;  // also frees accumulator b and histogram b^1
+        if (!ok) break;
+    }
+    if (ok) {
+        const int j = nt - 1;
+        const int* hp = hist_s + (j & 1) * 256;
+        for (int k = tid; k < C; k += 128) hist[((size_t)bh * C + k) * nblk + blk0 + j] = hp[k];
     }
     changed = __reduce_add_sync(0xffffffffu, changed);
-    if ((tid & 31) == 0 && changed) atomicAdd(&state[bh].changed, changed);
-    // After an abort the copies and MMAs of thread 0 may still be in flight:
-    // let them land before TMEM and shared memory are released.  Thread 0
-    // always committed bar_mma, so both barriers complete.
+    if (lane == 0 && changed) atomicAdd(&state[bh].changed, changed);
+    // After an abort thread 0's last copies and MMAs may still be in flight:
+    // let them land before shared memory and TMEM are released.
     if (tid == 0 && !ok) {
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(bar_ld, 0) && (int64_t)(globaltimer() - t0) < kDrainNs) {
-        }
-        while (!mbar_try_wait(bar_mma, 0) && (int64_t)(globaltimer() - t0) < kDrainNs) {
-        }
+        auto drain = [&](uint32_t bar, uint32_t parity) {
+            while (!mbar_try_wait(bar, parity) && (int64_t)(globaltimer() - t0) < kDrainNs) {
+            }
+        };
+        drain(bar_c, 0);
+        for (int t = max(0, v_issued - 2); t < v_issued; ++t) drain(bar_v0 + 8 * (t & 1), (t >> 1) & 1);
+        for (int t = max(0, mma_issued - 2); t < mma_issued; ++t) drain(bar_mma0 + 8 * (t & 1), (t >> 1) & 1);
     }
     tc_fence_before();
     __syncthreads();
-    for (int k = tid; k < C; k += 128) hist[((size_t)bh * C + k) * nblk + blk] = hist_s[k];
     if (warp == 0) {
         __syncwarp();
         tc_fence_after();
@@ -363,28 +508,74 @@ __global__ void __launch_bounds__(KM_TOK) km_scatter(const int32_t* __restrict__
     perm[(size_t)bh * N + offs[((size_t)bh * C + L) * nblk + blk] + rank] = j;
 }
 
-constexpr int KM_SLICES = 8;
+// fp64 member sums for the Lloyd update.  The stable order lists the members
+// of cluster 0, then cluster 1, ...; one CTA takes a fixed slice of KM_UPD_ROWS
+// positions of it (so large clusters spread over many CTAs) and walks the
+// cluster segments inside the slice: a row is read as D/8 16-byte pieces (8
+// channels a thread), the row groups are added in shared memory, and each
+// segment adds its sum to `sums` with one fp64 atomic per channel.
+constexpr int KM_UPD_ROWS = 256;
 
 template <int D>
 __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ perm,
-                                                 const int32_t* __restrict__ cstart,
-                                                 const int32_t* __restrict__ ccount, double* __restrict__ sums,
+                                                 const int32_t* __restrict__ cstart, double* __restrict__ sums,
                                                  const KmState* __restrict__ state, int N, int C,
                                                  const int* __restrict__ status) {
-    const int k = blockIdx.x, sl = blockIdx.y, bh = blockIdx.z;
+    constexpr int TPR = D / 8;    // threads per row
+    constexpr int R = 128 / TPR;  // rows per pass
+    __shared__ double red[R][D];
+    __shared__ int seg_s;
+    const int bh = blockIdx.y;
     if (ctl_failed(status) || state[bh].done) return;
-    const int cnt = ccount[(size_t)bh * C + k];
-    if (cnt == 0) return;
-    const int st = cstart[(size_t)bh * C + k];
-    const int a = st + (int)(((int64_t)cnt * sl) / KM_SLICES);
-    const int b = st + (int)(((int64_t)cnt * (sl + 1)) / KM_SLICES);
-    constexpr int RG = 128 / D;
-    const int c = threadIdx.x % D, rg = threadIdx.x / D;
-    double acc = 0.0;
+    const int r0 = blockIdx.x * KM_UPD_ROWS, r1 = min(N, r0 + KM_UPD_ROWS);
+    const int tid = threadIdx.x, cg = tid % TPR, rr = tid / TPR;
+    const int32_t* cs = cstart + (size_t)bh * C;
+    if (tid == 0) {  // the cluster holding position r0: the last k with cstart[k] <= r0
+        int lo = 0, hi = C - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (cs[mid] <= r0) lo = mid; else hi = mid - 1;
+        }
+        seg_s = lo;
+    }
+    __syncthreads();
     const int32_t* pp = perm + (size_t)bh * N;
-    const __nv_bfloat16* vb = V + (size_t)bh * N * D;
-    for (int i = a + rg; i < b; i += RG) acc += (double)bf2f(vb[(size_t)pp[i] * D + c]);
-    if (b > a) atomicAdd(&sums[((size_t)bh * C + k) * D + c], acc);
+    const uint4* vb = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D) + cg;
+    for (int k = seg_s; k < C; ++k) {
+        const int a = max(r0, cs[k]);
+        const int b = min(r1, k + 1 < C ? cs[k + 1] : N);
+        if (a >= r1) break;
+        if (b <= a) continue;  // empty cluster (uniform over the CTA)
+        double acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+        auto add = [&](const uint4& x) {
+            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __dadd_rn(acc[e], (double)bf2f(h[e]));
+        };
+        int i = a + rr;
+        for (; i + 3 * R < b; i += 4 * R) {
+            const int t0 = pp[i], t1 = pp[i + R], t2 = pp[i + 2 * R], t3 = pp[i + 3 * R];
+            const uint4 x0 = __ldg(vb + (size_t)t0 * TPR), x1 = __ldg(vb + (size_t)t1 * TPR);
+            const uint4 x2 = __ldg(vb + (size_t)t2 * TPR), x3 = __ldg(vb + (size_t)t3 * TPR);
+            add(x0);
+            add(x1);
+            add(x2);
+            add(x3);
+        }
+        for (; i < b; i += R) add(__ldg(vb + (size_t)pp[i] * TPR));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[rr][cg * 8 + e] = acc[e];
+        __syncthreads();
+        for (int c = tid; c < D; c += 128) {
+            double t = 0.0;
+#pragma unroll
+            for (int q = 0; q < R; ++q) t = __dadd_rn(t, red[q][c]);
+            atomicAdd(&sums[((size_t)bh * C + k) * D + c], t);
+        }
+        __syncthreads();
+    }
 }
 
 __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __restrict__ c_lo,
@@ -397,7 +588,7 @@ __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __r
     const int cnt = ccount[(size_t)bh * C + k];
     if (cnt == 0) return;  // an empty cluster keeps its centroid (sums are still 0)
     double* sp = &sums[((size_t)bh * C + k) * D + c];
-    const double mean = *sp / (double)cnt;  // the fp64 member mean (the sum of bf16 values is exact)
+    const double mean = __ddiv_rn(*sp, (double)cnt);  // the fp64 member mean
     *sp = 0.0;
     cent64[((size_t)bh * C + k) * D + c] = mean;
     const size_t row = ((size_t)bh * Cp + k) * D + c;
@@ -410,63 +601,98 @@ __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __r
 }
 
 // ------------------------------------------------------------------ block quantisation
-// One CTA per (block of BK regrouped tokens, head).  K: amax over the block,
-// inv = 448/amax, code = E4M3(k * inv), k_scale = amax/448.  V: block mean
-// (fp64 sum / valid, rounded to fp32; zero when smooth == 0), residual channel
-// amax folded into vamax with an integer max on the fp32 bits (all >= 0).
+// One CTA per (block of BK regrouped tokens, head), 256 threads.  The block's
+// gathered K and V rows are read once, 16 bytes a thread, into shared memory;
+// every pass below works from there.  K: amax over the block, inv = 448/amax,
+// code = E4M3(k * inv), k_scale = amax/448.  V: block mean (fp64 sum / valid,
+// rounded to fp32; zero when smooth == 0), residual channel amax folded into
+// vamax with an integer max on the fp32 bits (all >= 0).
+constexpr int PREP_THREADS = 256;
+
 template <int D, int BK>
-__global__ void __launch_bounds__(128) prep_kv_block(const __nv_bfloat16* __restrict__ K,
-                                                     const __nv_bfloat16* __restrict__ V,
-                                                     const int32_t* __restrict__ perm, int smooth,
-                                                     uint8_t* __restrict__ k_fp8, float* __restrict__ k_scale,
-                                                     float* __restrict__ v_mean, uint32_t* __restrict__ vamax, int N,
-                                                     int T, const int* __restrict__ status) {
-    constexpr int RG = 128 / D;  // row groups
+constexpr int kv_block_smem() {
+    return 2 * BK * D * 2;
+}
+
+template <int D, int BK>
+__global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat16* __restrict__ K,
+                                                              const __nv_bfloat16* __restrict__ V,
+                                                              const int32_t* __restrict__ perm, int smooth,
+                                                              uint8_t* __restrict__ k_fp8, float* __restrict__ k_scale,
+                                                              float* __restrict__ v_mean, uint32_t* __restrict__ vamax,
+                                                              int N, int T, const int* __restrict__ status) {
+    constexpr int NT = PREP_THREADS;
+    constexpr int RG = NT / D;  // row groups of the per-channel passes
+    constexpr int CH = D / 8;   // 16-byte pieces per row
+    extern __shared__ uint4 kv_s[];  // K rows [BK][CH], then V rows [BK][CH]
     __shared__ int tok_s[BK];
+    __shared__ uint32_t red_s[NT / 32];
     __shared__ double vsum_s[RG][D];
-    __shared__ float kmax_s[128];
     __shared__ float vmax_s[RG][D];
     if (ctl_failed(status)) return;  // perm is undefined
     const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    const int c = tid % D, rg = tid / D;
     const int valid = min(BK, N - b * BK);
-    for (int r = tid; r < BK; r += 128) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
     __syncthreads();
-    const __nv_bfloat16* kb = K + (size_t)bh * N * D + c;
-    const __nv_bfloat16* vb = V + (size_t)bh * N * D + c;
-    float kmax = 0.0f;
-    double vsum = 0.0;
-    for (int r = rg; r < valid; r += RG) {
-        const size_t row = (size_t)tok_s[r] * D;
-        kmax = fmaxf(kmax, fabsf(bf2f(kb[row])));
-        vsum += (double)bf2f(vb[row]);
+    uint4* ks = kv_s;
+    uint4* vs = kv_s + BK * CH;
+    const uint4* kg = reinterpret_cast<const uint4*>(K + (size_t)bh * N * D);
+    const uint4* vg = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D);
+    uint32_t kmax_bits = 0;  // |k| >= 0: the fp32 bit order is the value order
+#pragma unroll
+    for (int u = 0; u < BK * CH / NT; ++u) {
+        const int i = tid + u * NT;
+        const int r = i / CH, q = i % CH;
+        if (r < valid) {
+            const size_t src = (size_t)tok_s[r] * CH + q;
+            const uint4 kx = __ldg(kg + src);
+            const uint4 vx = __ldg(vg + src);
+            ks[i] = kx;
+            vs[i] = vx;
+            const uint32_t w[4] = {kx.x, kx.y, kx.z, kx.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)  // bf16 -> fp32 bits of |k|: the high half, sign cleared
+                kmax_bits = max(kmax_bits, max((w[e] << 16) & 0x7FFFFFFFu, w[e] & 0x7FFF0000u));
+        }
     }
-    kmax_s[tid] = kmax;
-    vsum_s[rg][c] = vsum;
+    kmax_bits = __reduce_max_sync(0xffffffffu, kmax_bits);
+    if ((tid & 31) == 0) red_s[tid >> 5] = kmax_bits;
     __syncthreads();
-    for (int s = 64; s > 0; s >>= 1) {
-        if (tid < s) kmax_s[tid] = fmaxf(kmax_s[tid], kmax_s[tid + s]);
-        __syncthreads();
-    }
-    const float amax = kmax_s[0];
+    uint32_t am = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) am = max(am, red_s[w]);
+    const float amax = __uint_as_float(am);
     const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
     if (tid == 0) k_scale[(size_t)bh * T + b] = __fdiv_rn(amax, 448.0f);
+
+    const __nv_bfloat16* ksh = reinterpret_cast<const __nv_bfloat16*>(ks);
+    const __nv_bfloat16* vsh = reinterpret_cast<const __nv_bfloat16*>(vs);
+    const int c = tid % D, rg = tid / D;
+    double vsum = 0.0;
+    for (int r = rg; r < valid; r += RG) vsum += (double)bf2f(vsh[r * D + c]);
+    vsum_s[rg][c] = vsum;
+    // K codes, four channels a thread (one 32-bit store); padding rows are 0
+    uint32_t* kout = reinterpret_cast<uint32_t*>(k_fp8 + ((size_t)bh * T * BK + (size_t)b * BK) * D);
+#pragma unroll 4
+    for (int i = tid; i < BK * D / 4; i += NT) {
+        const int r = i / (D / 4);
+        uint32_t w = 0;
+        if (r < valid) {
+            const uint2 raw = reinterpret_cast<const uint2*>(ksh)[i];
+            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+            w = (uint32_t)e4m3x2(__fmul_rn(bf2f(h[0]), inv), __fmul_rn(bf2f(h[1]), inv)) |
+                ((uint32_t)e4m3x2(__fmul_rn(bf2f(h[2]), inv), __fmul_rn(bf2f(h[3]), inv)) << 16);
+        }
+        kout[i] = w;
+    }
+    __syncthreads();
     double tot = 0.0;
 #pragma unroll
     for (int q = 0; q < RG; ++q) tot += vsum_s[q][c];
     const float mu = smooth ? (float)(tot / (double)valid) : 0.0f;
     if (rg == 0) v_mean[((size_t)bh * T + b) * D + c] = mu;
-    uint8_t* kout = k_fp8 + ((size_t)bh * T * BK + (size_t)b * BK) * D;
     float vmax = 0.0f;
-    for (int r = rg; r < BK; r += RG) {
-        uint8_t code = 0;
-        if (r < valid) {
-            const size_t row = (size_t)tok_s[r] * D;  // second read of the gathered rows hits L2
-            code = (uint8_t)(e4m3x2(__fmul_rn(bf2f(kb[row]), inv), 0.0f) & 0xFF);
-            vmax = fmaxf(vmax, fabsf(__fsub_rn(bf2f(vb[row]), mu)));
-        }
-        kout[(size_t)r * D + c] = code;
-    }
+    for (int r = rg; r < valid; r += RG) vmax = fmaxf(vmax, fabsf(__fsub_rn(bf2f(vsh[r * D + c]), mu)));
     vmax_s[rg][c] = vmax;
     __syncthreads();
     if (rg == 0) {
@@ -486,46 +712,60 @@ __global__ void identity_order(int32_t* __restrict__ perm, int32_t* __restrict__
 }
 
 // E4M3 residual with per-channel scales, written transposed: vt[bh][c][token].
+// The block's gathered V rows are read once, 16 bytes a thread, into shared
+// memory; codes are built per channel and leave as 16-byte pieces of vt rows.
 template <int D, int BK>
-__global__ void __launch_bounds__(128) prep_v_quant(const __nv_bfloat16* __restrict__ V,
-                                                    const int32_t* __restrict__ perm, int smooth,
-                                                    const float* __restrict__ v_mean,
-                                                    const uint32_t* __restrict__ vamax, uint8_t* __restrict__ vt_fp8,
-                                                    float* __restrict__ v_scale, int N, int T,
-                                                    const int* __restrict__ status) {
-    constexpr int RG = 128 / D;
-    constexpr int STRIDE = BK + 4;  // bytes per channel row in smem (conflict-free word stores)
+constexpr int v_quant_smem() {
+    return BK * D * 2;
+}
+
+template <int D, int BK>
+__global__ void __launch_bounds__(PREP_THREADS) prep_v_quant(const __nv_bfloat16* __restrict__ V,
+                                                             const int32_t* __restrict__ perm, int smooth,
+                                                             const float* __restrict__ v_mean,
+                                                             const uint32_t* __restrict__ vamax,
+                                                             uint8_t* __restrict__ vt_fp8, float* __restrict__ v_scale,
+                                                             int N, int T, const int* __restrict__ status) {
+    constexpr int NT = PREP_THREADS;
+    constexpr int RG = NT / D;
+    constexpr int CH = D / 8;
+    constexpr int STRIDE = BK + 4;  // bytes per channel row of codes (conflict-free word stores)
+    extern __shared__ uint4 v_s[];  // [BK][CH]
     __shared__ int tok_s[BK];
     __shared__ uint32_t cs[D * STRIDE / 4];
     if (ctl_failed(status)) return;  // perm is undefined
     const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    const int c = tid % D, rg = tid / D;
     const int valid = min(BK, N - b * BK);
     const int Tp = T * BK;
-    for (int r = tid; r < BK; r += 128) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    __syncthreads();
+    const uint4* vg = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D);
+#pragma unroll
+    for (int u = 0; u < BK * CH / NT; ++u) {
+        const int i = tid + u * NT;
+        const int r = i / CH;
+        if (r < valid) v_s[i] = __ldg(vg + (size_t)tok_s[r] * CH + i % CH);
+    }
+    const int c = tid % D, rg = tid / D;
     const float amax = __uint_as_float(vamax[(size_t)bh * D + c]);
     const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
     if (b == 0 && rg == 0) v_scale[(size_t)bh * D + c] = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
     const float mu = v_mean[((size_t)bh * T + b) * D + c];
     __syncthreads();
+    const __nv_bfloat16* vsh = reinterpret_cast<const __nv_bfloat16*>(v_s);
     for (int r4 = rg; r4 < BK / 4; r4 += RG) {
         float x[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = 4 * r4 + e;
-            x[e] = 0.0f;
-            if (r < valid) {
-                const float v = bf2f(V[((size_t)bh * N + tok_s[r]) * D + c]);
-                x[e] = __fmul_rn(__fsub_rn(v, mu), inv);
-            }
+            // padding tokens must be code 0 (x = +0 encodes to 0x00)
+            x[e] = r < valid ? __fmul_rn(__fsub_rn(bf2f(vsh[r * D + c]), mu), inv) : 0.0f;
         }
-        const uint32_t w = (uint32_t)e4m3x2(x[0], x[1]) | ((uint32_t)e4m3x2(x[2], x[3]) << 16);
-        // padding tokens must be code 0 (x = +0 encodes to 0x00)
-        cs[(c * STRIDE) / 4 + r4] = w;
+        cs[(c * STRIDE) / 4 + r4] = (uint32_t)e4m3x2(x[0], x[1]) | ((uint32_t)e4m3x2(x[2], x[3]) << 16);
     }
     __syncthreads();
     constexpr int CHUNKS = BK / 16;
-    for (int i = tid; i < D * CHUNKS; i += 128) {
+    for (int i = tid; i < D * CHUNKS; i += NT) {
         const int cc = i / CHUNKS, ch = i % CHUNKS;
         const uint32_t* src = cs + (cc * STRIDE) / 4 + ch * 4;
         *reinterpret_cast<uint4*>(vt_fp8 + ((size_t)bh * D + cc) * Tp + (size_t)b * BK + 16 * ch) =
@@ -582,7 +822,17 @@ template <int D>
 static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     const int nblk = (p.N + KM_TOK - 1) / KM_TOK;
     const int Cp = (p.C + 15) & ~15;
-    const size_t smem = 1024 + (size_t)KM_TOK * D * 2 + 2 * (size_t)Cp * D * 2 + 2 * 256 * 4 + 64;
+    // Two CTAs share an SM when both fit in shared memory and TMEM (2 Cp columns
+    // each); otherwise ask for enough shared memory to keep one CTA per SM, so
+    // no CTA waits in tcgen05.alloc.
+    const KmLayout lay(D, Cp);
+    const bool pair = lay.bytes <= 113 * 1024 && 2 * Cp <= 128;
+    const size_t smem = pair ? lay.bytes : (lay.bytes > 120 * 1024 ? lay.bytes : 120 * 1024);
+    // Tiles per CTA: about four waves of CTAs over the 148 SMs.
+    const int64_t tiles = (int64_t)nblk * p.BH;
+    const int64_t slots = 148LL * (pair ? 2 : 1) * 4;
+    const int tpc = (int)imin64(16, (tiles + slots - 1) / slots);
+    const int nchunk = (nblk + tpc - 1) / tpc;
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -597,15 +847,15 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     km_init<<<dim3(Cp, p.BH), D, 0, s>>>(p.V, p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.state, p.vamax, p.N, p.C,
                                          Cp, D);
     for (int it = 0; it < p.iters; ++it) {
-        km_assign<D><<<dim3(nblk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.labels, p.hist,
-                                                          p.state, p.N, p.C, Cp, it, p.ctl);
+        km_assign<D><<<dim3(nchunk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.vnorm2, p.labels,
+                                                            p.hist, p.state, p.N, p.C, Cp, it, tpc, p.ctl);
         km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it,
                                       p.ctl.status);
         km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C,
                                                        p.ctl.status);
         if (it + 1 < p.iters) {
-            km_update<D><<<dim3(p.C, KM_SLICES, p.BH), 128, 0, s>>>(p.V, p.perm, p.cstart, p.ccount, p.sums, p.state,
-                                                                    p.N, p.C, p.ctl.status);
+            km_update<D><<<dim3((p.N + KM_UPD_ROWS - 1) / KM_UPD_ROWS, p.BH), 128, 0, s>>>(
+                p.V, p.perm, p.cstart, p.sums, p.state, p.N, p.C, p.ctl.status);
             km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.ccount, p.state,
                                                       p.C, Cp, D, p.ctl.status);
         }
@@ -623,10 +873,20 @@ static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
         cudaError_t e = cudaMemsetAsync(p.vamax, 0, sizeof(uint32_t) * (size_t)p.BH * D, s);
         if (e != cudaSuccess) return e;
     }
-    prep_kv_block<D, BK><<<dim3(T, p.BH), 128, 0, s>>>(p.K, p.V, p.perm, p.smooth, p.k_fp8, p.k_scale, p.v_mean,
-                                                       p.vamax, p.N, T, p.ctl.status);
-    prep_v_quant<D, BK><<<dim3(T, p.BH), 128, 0, s>>>(p.V, p.perm, p.smooth, p.v_mean, p.vamax, p.vt_fp8, p.v_scale,
-                                                      p.N, T, p.ctl.status);
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(prep_kv_block<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kv_block_smem<D, BK>());
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(prep_v_quant<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 v_quant_smem<D, BK>());
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    prep_kv_block<D, BK><<<dim3(T, p.BH), PREP_THREADS, kv_block_smem<D, BK>(), s>>>(
+        p.K, p.V, p.perm, p.smooth, p.k_fp8, p.k_scale, p.v_mean, p.vamax, p.N, T, p.ctl.status);
+    prep_v_quant<D, BK><<<dim3(T, p.BH), PREP_THREADS, v_quant_smem<D, BK>(), s>>>(
+        p.V, p.perm, p.smooth, p.v_mean, p.vamax, p.vt_fp8, p.v_scale, p.N, T, p.ctl.status);
     return cudaGetLastError();
 }
 
