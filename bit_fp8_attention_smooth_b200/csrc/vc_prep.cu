@@ -87,7 +87,7 @@ struct KmLayout {
         v_bytes = KM_TOK * D * 2;
         c_bytes = Cp * D * 2;
         off_v = 0;
-        off_chi = 2 * v_bytes;
+        off_chi = v_bytes;  // one V tile: the next is loaded while the CUDA cores work
         off_clo = off_chi + c_bytes;
         off_cn = off_clo + c_bytes;            // [256] |c_k|^2
         off_hist = off_cn + 256 * 4;           // [2][256] per-tile cluster counts
@@ -108,7 +108,7 @@ struct KmLayout {
 // with near-ties decided again in fp64.  Per tile: labels, the per-cluster
 // histogram of the tile (for the stable regroup) and the change count.
 template <int D>
-__global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUtensorMap tm_v,
+__global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUtensorMap tm_v,
                                                  const __grid_constant__ CUtensorMap tm_chi,
                                                  const __grid_constant__ CUtensorMap tm_clo,
                                                  const float* __restrict__ cnorm, const double* __restrict__ cent64,
@@ -165,17 +165,16 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
     const float cmax_r = sqrtf(__uint_as_float(max(max(red_s[0], red_s[1]), max(red_s[2], red_s[3]))));
 
     const uint32_t sV = base + L.off_v, sCh = base + L.off_chi, sCl = base + L.off_clo;
-    auto load_v = [&](int j) {  // thread 0
-        const uint32_t b = j & 1, bar = bar_v0 + 8 * b;
-        mbar_expect_tx_arrive(bar, L.v_bytes);
+    auto load_v = [&](int j) {  // thread 0; tile j completes phase j & 1 of bar_v0
+        mbar_expect_tx_arrive(bar_v0, L.v_bytes);
 #pragma unroll
         for (int kc = 0; kc < D / 64; ++kc)
-            tma_load_3d(sV + b * L.v_bytes + kc * (KM_TOK * 128), &tm_v, bar, 64 * kc, (blk0 + j) * KM_TOK, bh);
+            tma_load_3d(sV + kc * (KM_TOK * 128), &tm_v, bar_v0, 64 * kc, (blk0 + j) * KM_TOK, bh);
     };
     const uint32_t idesc = idesc_bf16_f32(Cp);
     auto issue_mma = [&](int j) {  // thread 0, after V tile j (and the centroids) landed
         const uint32_t b = j & 1;
-        const uint32_t sA = sV + b * L.v_bytes, acc = tmem + b * Cp;
+        const uint32_t sA = sV, acc = tmem + b * Cp;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -203,10 +202,6 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
         }
         load_v(0);
         v_issued = 1;
-        if (nt > 1) {
-            load_v(1);
-            v_issued = 2;
-        }
         ok = mbar_wait(bar_c, 0, ctl, abort_flag) && mbar_wait(bar_v0, 0, ctl, abort_flag);
         if (ok) {
             issue_mma(0);
@@ -224,13 +219,6 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
                 hp[k] = 0;
             }
         }
-        if (tid == 0 && ok && j + 1 < nt) {  // MMA j+1 into the other accumulator, read out by tile j-1
-            ok = mbar_wait(bar_v0 + 8 * (b ^ 1), ((j + 1) >> 1) & 1, ctl, abort_flag);
-            if (ok) {
-                issue_mma(j + 1);
-                mma_issued = j + 2;
-            }
-        }
         bool okj = __all_sync(0xffffffffu, ok && mbar_wait(bar_mma0 + 8 * b, (j >> 1) & 1, ctl, abort_flag));
         tc_fence_after();
         const int n = n0 + tid;
@@ -238,7 +226,7 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
         float vn2 = 0.0f;
         if (it == 0) {  // |v|^2 once per prep, from the V tile before it is overwritten
             if (okj) {
-                const uint8_t* arow = smem + L.off_v + b * L.v_bytes + tid * 128;
+                const uint8_t* arow = smem + L.off_v + tid * 128;
 #pragma unroll
                 for (int kc = 0; kc < D / 64; ++kc)
 #pragma unroll
@@ -255,17 +243,17 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
         } else if (okj && valid) {
             vn2 = vnorm2[(size_t)bh * N + n];
         }
-        if (tid == 0 && okj && j + 2 < nt) {  // MMA j has read V buffer b
-            load_v(j + 2);
-            v_issued = j + 3;
+        if (tid == 0 && okj && j + 1 < nt) {  // MMA j has read the V tile
+            load_v(j + 1);
+            v_issued = j + 2;
         }
         if (okj) {
             const uint32_t lane_tmem = tmem + b * Cp + ((uint32_t)(warp * 32) << 16);
             // Pass 1: best and runner-up of the tensor-core distances
             // d_k = |c_k|^2 - 2 v.c_k.  With Cp <= 64 the distances stay in
             // registers for the near-tie masks below.
-            float best = INFINITY, second = INFINITY;
-            int bestk = 0;
+            float b4[4] = {INFINITY, INFINITY, INFINITY, INFINITY}, s4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+            int k4[4] = {0, 0, 0, 0};  // four independent chains: candidate k goes to chain k % 4
             float dk[64];
             for (int g = 0; g < Cp; g += 64) {
 #pragma unroll
@@ -281,12 +269,23 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
                         for (int e = 0; e < 4; ++e) {
                             const float d = fmaf(-2.0f, dk[4 * q4 + e], cv[e]);
                             dk[4 * q4 + e] = d;
-                            const bool lt = d < best;
-                            second = fminf(second, fmaxf(best, d));
-                            best = fminf(best, d);
-                            bestk = lt ? g + 4 * q4 + e : bestk;
+                            const bool lt = d < b4[e];
+                            s4[e] = fminf(s4[e], fmaxf(b4[e], d));
+                            b4[e] = fminf(b4[e], d);
+                            k4[e] = lt ? g + 4 * q4 + e : k4[e];
                         }
                     }
+                }
+            }
+            // merge the chains: best (ties to the lowest k) and runner-up
+            float best = b4[0], second = s4[0];
+            int bestk = k4[0];
+#pragma unroll
+            for (int e = 1; e < 4; ++e) {
+                second = fminf(fminf(second, s4[e]), fmaxf(best, b4[e]));
+                if (b4[e] < best || (b4[e] == best && k4[e] < bestk)) {
+                    best = b4[e];
+                    bestk = k4[e];
                 }
             }
             // Error bound of the tensor-core distance: bf16 hi/lo centroids carry
@@ -410,8 +409,17 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
                 atomicAdd(&hist_s[b * 256 + label], 1);
             }
         }
+        if (tid == 0 && ok && okj && j + 1 < nt) {
+            // MMA j+1 into the other accumulator (read out by tile j-1) while
+            // the other warps finish tile j
+            ok = mbar_wait(bar_v0, (j + 1) & 1, ctl, abort_flag);
+            if (ok) {
+                issue_mma(j + 1);
+                mma_issued = j + 2;
+            }
+        }
         tc_fence_before();
-        ok = __syncthreads_and(okj) != 0;  // also frees accumulator b and histogram b^1
+        ok = __syncthreads_and(okj && ok) != 0;  // also frees accumulator b and histogram b^1
         if (!ok) break;
     }
     if (ok) {
@@ -430,7 +438,7 @@ __global__ void __launch_bounds__(128, 2) km_assign(const __grid_constant__ CUte
             }
         };
         drain(bar_c, 0);
-        for (int t = max(0, v_issued - 2); t < v_issued; ++t) drain(bar_v0 + 8 * (t & 1), (t >> 1) & 1);
+        if (v_issued > 0) drain(bar_v0, (v_issued - 1) & 1);  // earlier tiles landed before the next was issued
         for (int t = max(0, mma_issued - 2); t < mma_issued; ++t) drain(bar_mma0 + 8 * (t & 1), (t >> 1) & 1);
     }
     tc_fence_before();
@@ -825,12 +833,18 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     // Two CTAs share an SM when both fit in shared memory and TMEM (2 Cp columns
     // each); otherwise ask for enough shared memory to keep one CTA per SM, so
     // no CTA waits in tcgen05.alloc.
+    // CTAs per SM: as many as shared memory (228 KB an SM) and TMEM (512
+    // columns, 2 Cp a CTA) allow, at most three; the request is padded so no
+    // more CTAs than that share an SM and none waits in tcgen05.alloc.
     const KmLayout lay(D, Cp);
-    const bool pair = lay.bytes <= 113 * 1024 && 2 * Cp <= 128;
-    const size_t smem = pair ? lay.bytes : (lay.bytes > 120 * 1024 ? lay.bytes : 120 * 1024);
+    const int ncols = 2 * Cp <= 32 ? 32 : (2 * Cp <= 64 ? 64 : (2 * Cp <= 128 ? 128 : (2 * Cp <= 256 ? 256 : 512)));
+    int cps = 3;
+    while (cps > 1 && ((size_t)cps * lay.bytes > 227 * 1024 || cps * ncols > 512)) --cps;
+    const size_t smem = lay.bytes > (size_t)(228 * 1024 / (cps + 1) + 1024) ? lay.bytes
+                                                                             : (size_t)(228 * 1024 / (cps + 1) + 1024);
     // Tiles per CTA: about four waves of CTAs over the 148 SMs.
     const int64_t tiles = (int64_t)nblk * p.BH;
-    const int64_t slots = 148LL * (pair ? 2 : 1) * 4;
+    const int64_t slots = 148LL * cps * 4;
     const int tpc = (int)imin64(16, (tiles + slots - 1) / slots);
     const int nchunk = (nblk + tpc - 1) / tpc;
     static bool configured = false;
