@@ -20,7 +20,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct WsLayout {
     // offsets in bytes from the workspace base
     size_t status;
-    size_t labels, c_hi, c_lo, cnorm, cent64, vnorm2, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
+    size_t labels, c_hi, c_lo, cnorm, cent64, vnorm2, ties, tie_count, sums, cstart, ccount, hist, offs, state, vamax;  // prep region
     size_t qfp8, sq;                                                      // attention region (aliases prep)
     size_t prep_end, attn_end, total;
 };
@@ -39,6 +39,8 @@ WsLayout ws_layout(const vc_shape& s, const vc_params& p) {
     w.cnorm = o; o = align256(o + 4 * BH * Cp);
     w.cent64 = o; o = align256(o + 8 * BH * C * D);
     w.vnorm2 = o; o = align256(o + 4 * BH * N);
+    w.ties = o; o = align256(o + sizeof(vc::KmTie) * BH * N);
+    w.tie_count = o; o = align256(o + 2 * sizeof(int));
     w.sums = o; o = align256(o + 8 * BH * C * D);
     w.cstart = o; o = align256(o + 4 * BH * C);
     w.ccount = o; o = align256(o + 4 * BH * C);
@@ -137,6 +139,8 @@ vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc
     pl.cnorm = reinterpret_cast<float*>(ws + L.cnorm);
     pl.cent64 = reinterpret_cast<double*>(ws + L.cent64);
     pl.vnorm2 = reinterpret_cast<float*>(ws + L.vnorm2);
+    pl.ties = reinterpret_cast<vc::KmTie*>(ws + L.ties);
+    pl.tie_count = reinterpret_cast<int*>(ws + L.tie_count);
     pl.sums = reinterpret_cast<double*>(ws + L.sums);
     pl.ctl.status = reinterpret_cast<int*>(ws + L.status);
     pl.ctl.limit_ns = p.wait_limit_ns > 0 ? p.wait_limit_ns : kDefaultWaitNs;

@@ -25,6 +25,14 @@ struct KmState {  // per (b, h), 16 bytes of workspace
     int pad0, pad1;
 };
 
+// A k-means near tie: a token whose tensor-core distances leave more than one
+// cluster within the error bound; km_refine decides it in fp64.
+struct KmTie {
+    int32_t bh, n;       // head, token
+    int32_t old, prov;   // label before this pass (-1 on the first), tensor-core label
+    uint32_t mask[8];    // candidate clusters (bit k of word k / 32)
+};
+
 struct PrepLaunch {
     const __nv_bfloat16* K;
     const __nv_bfloat16* V;
@@ -43,7 +51,9 @@ struct PrepLaunch {
     float* cnorm;         // [BH, Cp] squared centroid norms
     double* cent64;       // [BH, C, D] fp64 centroids (the exact near-tie decision)
     double* sums;         // [BH, C, D] fp64 member sums of the Lloyd update
-    float* vnorm2;        // [BH, N] |v|^2 of every token (bounds the tensor-core distance error)
+    float* vnorm2;
+    KmTie* ties;          // [BH * N] near-tie list of the current pass
+    int* tie_count;       // [2] list lengths, by pass parity        // [BH, N] |v|^2 of every token (bounds the tensor-core distance error)
     int32_t* cstart;
     int32_t* ccount;
     int32_t* hist;

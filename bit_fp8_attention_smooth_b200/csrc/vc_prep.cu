@@ -53,7 +53,8 @@ __device__ __forceinline__ float block_sum_d(float x, float* red) {
 
 __global__ void km_init(const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ c_hi,
                         __nv_bfloat16* __restrict__ c_lo, float* __restrict__ cnorm, double* __restrict__ cent64,
-                        double* __restrict__ sums, KmState* __restrict__ state, uint32_t* __restrict__ vamax, int N,
+                        double* __restrict__ sums, KmState* __restrict__ state, uint32_t* __restrict__ vamax,
+                        int* __restrict__ tie_count, int N,
                         int C, int Cp, int D) {
     __shared__ float red[4];
     const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
@@ -69,6 +70,7 @@ __global__ void km_init(const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __re
     c_lo[row] = __float2bfloat16_rn(0.0f);
     const float nrm = block_sum_d(x * x, red);
     if (c == 0) cnorm[(size_t)bh * Cp + k] = nrm;
+    if (k == 0 && bh == 0 && c < 2) tie_count[c] = 0;
     if (k == 0) {
         vamax[(size_t)bh * D + c] = 0u;
         if (c == 0) state[bh] = KmState{0, 0, 0, 0};
@@ -79,10 +81,8 @@ constexpr int KM_TOK = 128;  // tokens per tile (the MMA's M)
 
 // Shared-memory plan of km_assign, from a 1024-byte aligned base:
 //   V tile x2 | centroid hi | centroid lo | |c|^2 | histograms x2 | scratch | barriers
-constexpr int KM_PCAP = 64;  // near-tie (token, candidate) pairs a warp decides together
-
 struct KmLayout {
-    uint32_t v_bytes, c_bytes, off_v, off_chi, off_clo, off_cn, off_hist, off_pk, off_red, off_bar, off_misc, bytes;
+    uint32_t v_bytes, c_bytes, off_v, off_chi, off_clo, off_cn, off_hist, off_red, off_bar, off_misc, bytes;
     __host__ __device__ KmLayout(int D, int Cp) {
         v_bytes = KM_TOK * D * 2;
         c_bytes = Cp * D * 2;
@@ -91,8 +91,7 @@ struct KmLayout {
         off_clo = off_chi + c_bytes;
         off_cn = off_clo + c_bytes;            // [256] |c_k|^2
         off_hist = off_cn + 256 * 4;           // [2][256] per-tile cluster counts
-        off_pk = off_hist + 2 * 256 * 4;       // [4 warps][KM_PCAP] near-tie pairs
-        off_red = off_pk + 4 * KM_PCAP * 4;
+        off_red = off_hist + 2 * 256 * 4;
         off_bar = off_red + 64;
         off_misc = off_bar + 64;
         bytes = off_misc + 16 + 1024;  // + alignment slack
@@ -114,6 +113,7 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
                                                  const float* __restrict__ cnorm, const double* __restrict__ cent64,
                                                  const __nv_bfloat16* __restrict__ V, float* __restrict__ vnorm2,
                                                  int32_t* __restrict__ labels, int32_t* __restrict__ hist,
+                                                 KmTie* __restrict__ ties, int* __restrict__ tie_count,
                                                  KmState* __restrict__ state, int N, int C, int Cp, int it, int tpc,
                                                  DevCtl ctl) {
     const int bh = blockIdx.y, nblk = (N + KM_TOK - 1) / KM_TOK;
@@ -298,11 +298,16 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
             const float rad = sqrtf(vn2) + cmax_r;
             const float margin = ldexpf(rad * rad, -12);
             const bool refine = valid && C > 1 && (second - best) <= margin;
-            if (__any_sync(0xffffffffu, refine)) {
-                int* pk = reinterpret_cast<int*>(smem + L.off_pk) + warp * KM_PCAP;
+            // Near ties go to the list that km_refine decides in fp64; the
+            // label written now is the tensor-core choice.
+            const int32_t old_label = valid && it > 0 ? labels[(size_t)bh * N + n] : -1;
+            const uint32_t rmask = __ballot_sync(0xffffffffu, refine);
+            if (rmask != 0) {
+                int first = 0;
+                if (lane == 0) first = atomicAdd(tie_count + (it & 1), __popc(rmask));
+                first = __shfl_sync(0xffffffffu, first, 0);
+                KmTie* e = ties + first + __popc(rmask & ((1u << lane) - 1));
                 const float lim = best + margin;
-                double dbest = INFINITY;
-                int kbest = bestk;
                 for (int g = 0; g < Cp; g += 64) {
                     if (Cp > 64) {  // the group's distances again, from TMEM
 #pragma unroll
@@ -313,99 +318,23 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
                         for (int jj = 0; jj < 64; ++jj)
                             if (g + jj < Cp) dk[jj] = fmaf(-2.0f, dk[jj], cn_s[g + jj]);
                     }
-                    uint32_t m0 = 0, m1 = 0;  // candidates g..g+31 and g+32..g+63
                     if (refine) {
+                        uint32_t m0 = 0, m1 = 0;  // candidates g..g+31 and g+32..g+63
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) {
                             if (g + jj < Cp && dk[jj] <= lim) m0 |= 1u << jj;
                             if (g + 32 + jj < Cp && dk[32 + jj] <= lim) m1 |= 1u << jj;
                         }
-                    }
-                    const int cnt = __popc(m0) + __popc(m1);
-                    int incl = cnt;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += t;
-                    }
-                    const int total = __shfl_sync(0xffffffffu, incl, 31);
-                    // The warp's (lane, cluster) pairs, lane by lane and in
-                    // ascending k, KM_PCAP at a time.
-                    for (int base = 0; base < total; base += KM_PCAP) {
-                        int p = incl - cnt;
-                        for (int h = 0; h < 2; ++h)
-                            for (uint32_t m = h ? m1 : m0; m; m &= m - 1, ++p)
-                                if (p >= base && p < base + KM_PCAP)
-                                    pk[p - base] = (lane << 16) | (g + 32 * h + __ffs(m) - 1);
-                        __syncwarp();
-                        const int np = min(KM_PCAP, total - base);
-                        // Each pair's distance is computed by the whole warp (D/32
-                        // channels a lane, then a butterfly), four pairs at a time
-                        // with all their loads issued first.
-                        constexpr int CPL = D / 32;
-                        const int c0 = lane * CPL;
-                        for (int q0 = 0; q0 < np; q0 += 4) {
-                            float vx[4][CPL];
-                            double cx[4][CPL];
-                            int pid[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                pid[u] = q0 + u < np ? pk[q0 + u] : -1;
-                                if (pid[u] >= 0) {
-                                    const int t = pid[u] >> 16, k = pid[u] & 0xFFFF;
-                                    const __nv_bfloat16* vp = V + ((size_t)bh * N + n0 + warp * 32 + t) * D + c0;
-                                    const double* cp = cent64 + ((size_t)bh * C + k) * D + c0;
-                                    if constexpr (CPL == 4) {
-                                        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(vp));
-                                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-                                        const double2 a = __ldg(reinterpret_cast<const double2*>(cp));
-                                        const double2 b2 = __ldg(reinterpret_cast<const double2*>(cp) + 1);
-#pragma unroll
-                                        for (int e = 0; e < 4; ++e) vx[u][e] = bf2f(hv[e]);
-                                        cx[u][0] = a.x;
-                                        cx[u][1] = a.y;
-                                        cx[u][2] = b2.x;
-                                        cx[u][3] = b2.y;
-                                    } else {
-                                        const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(vp));
-                                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-                                        const double2 a = __ldg(reinterpret_cast<const double2*>(cp));
-#pragma unroll
-                                        for (int e = 0; e < CPL; ++e) vx[u][e] = bf2f(hv[e]);
-                                        cx[u][0] = a.x;
-                                        cx[u][CPL - 1] = a.y;
-                                    }
-                                }
-                            }
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                if (pid[u] < 0) break;  // uniform: pid comes from shared memory
-                                double part = 0.0;
-#pragma unroll
-                                for (int e = 0; e < CPL; ++e) {
-                                    const double diff = __dsub_rn((double)vx[u][e], cx[u][e]);
-                                    part = __dadd_rn(part, __dmul_rn(diff, diff));
-                                }
-#pragma unroll
-                                for (int o = 16; o > 0; o >>= 1)
-                                    part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
-                                // strict: of equal distances the lowest k stays
-                                if (lane == (pid[u] >> 16) && part < dbest) {
-                                    dbest = part;
-                                    kbest = pid[u] & 0xFFFF;
-                                }
-                            }
-                        }
-                        __syncwarp();
+                        e->mask[g >> 5] = m0;
+                        if ((g >> 5) + 1 < 8) e->mask[(g >> 5) + 1] = m1;
                     }
                 }
-                if (refine) bestk = kbest;
+                if (refine) *reinterpret_cast<int4*>(e) = make_int4(bh, n, old_label, bestk);
             }
             const int label = bestk;
             if (valid) {
-                int32_t* lp = labels + (size_t)bh * N + n;
-                if (it == 0 || *lp != label) ++changed;
-                *lp = label;
+                if (it == 0 || old_label != label) ++changed;
+                labels[(size_t)bh * N + n] = label;
                 atomicAdd(&hist_s[b * 256 + label], 1);
             }
         }
@@ -447,6 +376,82 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, ncols);
+    }
+}
+
+// fp64 decision of the near ties km_assign listed: one warp a token, each
+// candidate's squared distance summed over D/32 channels a lane in fp64 and
+// added across the warp; candidates in ascending cluster order with a strict
+// comparison, so equal distances keep the lowest cluster (as the Lloyd step's
+// argmin).  When the decision differs from the tensor-core label, the label,
+// the tile's cluster counts and the head's change count are corrected.
+template <int D>
+__global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties, int* __restrict__ tie_count,
+                                                 const __nv_bfloat16* __restrict__ V,
+                                                 const double* __restrict__ cent64, int32_t* __restrict__ labels,
+                                                 int32_t* __restrict__ hist, KmState* __restrict__ state, int N,
+                                                 int C, int Cp, int it, const int* __restrict__ status) {
+    if (ctl_failed(status)) return;
+    constexpr int CPL = D / 32;  // channels a lane
+    const int count = tie_count[it & 1];
+    if (blockIdx.x == 0 && threadIdx.x == 0) tie_count[(it + 1) & 1] = 0;  // the next pass's list starts empty
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nblk = (N + KM_TOK - 1) / KM_TOK;
+    const int words = (Cp + 31) >> 5;
+    for (int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; e < count; e += nwarps) {
+        const int4 hd = *reinterpret_cast<const int4*>(ties + e);  // bh, n, old, prov
+        const int bh = hd.x, n = hd.y;
+        float vx[CPL];
+        {
+            const __nv_bfloat16* vp = V + ((size_t)bh * N + n) * D + lane * CPL;
+            if constexpr (CPL == 4) {
+                const uint2 raw = __ldg(reinterpret_cast<const uint2*>(vp));
+                const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) vx[i] = bf2f(h[i]);
+            } else {
+                const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(vp));
+                const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) vx[i] = bf2f(h[i]);
+            }
+        }
+        double dbest = INFINITY;
+        int kbest = hd.w;
+        for (int w = 0; w < words; ++w) {
+            for (uint32_t m = ties[e].mask[w]; m; m &= m - 1) {
+                const int k = 32 * w + __ffs(m) - 1;
+                const double2* cp = reinterpret_cast<const double2*>(cent64 + ((size_t)bh * C + k) * D + lane * CPL);
+                double cx[CPL];
+#pragma unroll
+                for (int i = 0; i < CPL / 2; ++i) {
+                    const double2 c2 = __ldg(cp + i);
+                    cx[2 * i] = c2.x;
+                    cx[2 * i + 1] = c2.y;
+                }
+                double part = 0.0;
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) {
+                    const double diff = __dsub_rn((double)vx[i], cx[i]);
+                    part = __dadd_rn(part, __dmul_rn(diff, diff));
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+                if (part < dbest) {
+                    dbest = part;
+                    kbest = k;
+                }
+            }
+        }
+        if (lane == 0 && kbest != hd.w) {
+            labels[(size_t)bh * N + n] = kbest;
+            const int tile = n / KM_TOK;
+            atomicSub(&hist[((size_t)bh * C + hd.w) * nblk + tile], 1);
+            atomicAdd(&hist[((size_t)bh * C + kbest) * nblk + tile], 1);
+            const int dchg = (kbest != hd.z) - (hd.w != hd.z);
+            if (dchg != 0) atomicAdd(&state[bh].changed, dchg);
+        }
     }
 }
 
@@ -858,11 +863,14 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
         !make_tmap_3d(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.c_hi, D, Cp, p.BH, 64, Cp) ||
         !make_tmap_3d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.c_lo, D, Cp, p.BH, 64, Cp))
         return cudaErrorInvalidValue;
-    km_init<<<dim3(Cp, p.BH), D, 0, s>>>(p.V, p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.state, p.vamax, p.N, p.C,
+    km_init<<<dim3(Cp, p.BH), D, 0, s>>>(p.V, p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.state, p.vamax, p.tie_count, p.N, p.C,
                                          Cp, D);
     for (int it = 0; it < p.iters; ++it) {
         km_assign<D><<<dim3(nchunk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.vnorm2, p.labels,
-                                                            p.hist, p.state, p.N, p.C, Cp, it, tpc, p.ctl);
+                                                            p.hist, p.ties, p.tie_count, p.state, p.N, p.C, Cp,
+                                                            it, tpc, p.ctl);
+        km_refine<D><<<148 * 8, 256, 0, s>>>(p.ties, p.tie_count, p.V, p.cent64, p.labels, p.hist, p.state, p.N,
+                                              p.C, Cp, it, p.ctl.status);
         km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it,
                                       p.ctl.status);
         km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C,
