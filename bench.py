@@ -50,6 +50,29 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def attn_traffic_bytes(heads: int):
+    """DRAM bytes (read + write) of one attention-kernel launch over `heads`
+    heads, from the ncu capture summarised in profiles/; None when the kernel
+    sources have changed since that capture (its counters no longer apply)."""
+    import hashlib
+    import re
+
+    prof = os.path.join(ROOT, "profiles", "vc_attn_kernel_mid_32k_h8.md")
+    csrc = os.path.join(ROOT, "bit_fp8_attention_smooth_b200", "csrc")
+    try:
+        text = open(prof).read()
+        h = hashlib.sha256()
+        for name in ("vc_attn.cu", "vc_device.cuh"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    except OSError:
+        return None
+    m = re.search(r"roofline-traffic: kernel=\S+ sources_sha256_16=([0-9a-f]{16}) dram_bytes_per_head=(\d+)", text)
+    if not m or m.group(1) != h.hexdigest()[:16]:
+        return None
+    return int(m.group(2)) * heads
+
+
 # ----------------------------------------------------------------- distributed
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -287,7 +310,8 @@ def run_ours(args, w):
                 "bound": "tensor", "kernel": "vc_attn_fwd (Q quantise + vc_attn_kernel)",
                 "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
                 "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16)",
-                "traffic": None,
+                "traffic": attn_traffic_bytes(w.B * w.H),
+                "traffic_unit": "bytes per launch (ncu capture on 8 heads, scaled by heads)",
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": e2e.h2d_bytes, "d2h_bytes_per_step": e2e.d2h_bytes},

@@ -8,8 +8,10 @@
 //
 // Kernels, per call, for all (b, h) at once:
 //   km_init                   strided centroid init c_k = v[floor(k N / C)]
-//   per pass: km_assign       labels = argmin_k |v - c_k|^2 (fp32, ties -> lowest k),
-//                             per-(cluster, 128-token block) histogram, change count
+//   per pass: km_assign       labels = argmin_k |c_k|^2 - 2 v.c_k on tensor cores (ties ->
+//                             lowest k), per-(cluster, 128-token block) histogram, change
+//                             count; near ties listed for km_refine
+//             km_refine       fp64 decision of the near ties; fixes labels and counts
 //             km_scan         exclusive scan -> stable positions; a head whose labels
 //                             did not change is final (its later passes would repeat)
 //             km_scatter      perm[position] = token (stable within a cluster)
