@@ -281,21 +281,25 @@ def run_ours(args, w):
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
 
     # end to end through the public API from pinned host buffers
+    # Two calls in flight: a step's copies overlap the previous step's
+    # computation; each step reads its own result back into its own host
+    # buffer.
     e2e = vc.HostAttention(shape, params, dev)
-    o_host = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
-    for _ in range(max(1, args.warmup // 2)):
-        e2e(host["q"], host["k"], host["v"], o_host)
+    o_host = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    for i in range(max(2, args.warmup // 2)):
+        e2e(host["q"], host["k"], host["v"], o_host[i % 2])
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e_steps = max(2, min(args.steps, 6))
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e(host["q"], host["k"], host["v"], o_host)
+    pending = [e2e(host["q"], host["k"], host["v"], o_host[i % 2]) for i in range(e2e_steps)]
+    for p in pending:  # the timed region ends when every step's output is back
+        p.wait()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
-    vc.check(e2e.ws)
+    e2e.check()
 
     if rank == 0:
         peaks = load_peaks()

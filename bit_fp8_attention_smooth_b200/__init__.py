@@ -65,6 +65,7 @@ def lib():
             "vc_smooth_prepare": (ctypes.c_int, [P, P, PS, PP, PR, P, S, P]),
             "vc_attn_fwd": (ctypes.c_int, [P, PR, PS, PP, P, P, S, P]),
             "vc_attention": (ctypes.c_int, [P, P, P, PS, PP, PR, P, P, S, P]),
+            "vc_attention_host": (ctypes.c_int, [P, P, P, P, PS, PP, ctypes.c_int, P, P, P, P, PR, P, S, P, P, P]),
             "vc_check": (ctypes.c_int, [P, P]),
             "vc_attn_fwd_noalloc": (ctypes.c_int, [P, PR, PS, PP, P, P]),
             "vc_e4m3_encode": (ctypes.c_int, [P, P, i64, P]),
@@ -246,25 +247,76 @@ def expcast_bytes(A: torch.Tensor, s: torch.Tensor, cb: torch.Tensor, stream=Non
     return out
 
 
-class HostAttention:
-    """End-to-end call from pinned host buffers: H2D copies, the CUDA path, D2H
-    copy of O, all on one stream (device buffers are allocated once)."""
+class _HostSet:
+    """One set of device buffers and streams for vc_attention_host."""
 
-    def __init__(self, shape, params: Params, device="cuda"):
-        self.shape, self.params = tuple(shape), params
+    def __init__(self, shape, params: Params, device):
         self.q = torch.empty(shape, dtype=torch.bfloat16, device=device)
         self.k = torch.empty_like(self.q)
         self.v = torch.empty_like(self.q)
         self.o = torch.empty_like(self.q)
-        self.prep = alloc_prep(self.shape, params, device)
-        self.ws = alloc_workspace(self.shape, params, device)
-        self.h2d_bytes = 3 * self.q.numel() * 2
-        self.d2h_bytes = self.o.numel() * 2
+        self.prep = alloc_prep(shape, params, device)
+        self.ws = alloc_workspace(shape, params, device)
+        self.streams = [torch.cuda.Stream(device=self.q.device) for _ in range(3)]  # h2d, compute, d2h
+
+
+class HostAttention:
+    """End-to-end call from pinned host buffers (vc_attention_host): the B*H
+    problems run in `groups` runs, each one's H2D copy, prep + attention and
+    D2H copy on three streams, so the transfers of one run overlap the
+    computation of its neighbours.  With `sets` = 2 the calls alternate
+    between two independent sets of device buffers, workspaces and streams,
+    so the copies of one call also overlap the computation of the previous
+    one.  Device memory is allocated once, in the constructor."""
+
+    def __init__(self, shape, params: Params, device="cuda", groups: int = 4, sets: int = 2):
+        self.shape, self.params, self.groups = tuple(shape), params, groups
+        self.sets = [_HostSet(self.shape, params, device) for _ in range(max(1, sets))]
+        self.calls = 0
+        n = 1
+        for x in self.shape:
+            n *= x
+        self.h2d_bytes = 3 * n * 2
+        self.d2h_bytes = n * 2
+
+    @property
+    def ws(self):  # workspace of the set the last call used (for vc_check)
+        return self.sets[(self.calls - 1) % len(self.sets)].ws
+
+    def check(self):
+        """Synchronise every set and raise VcError on a recorded device error."""
+        for st in self.sets:
+            _ok(lib().vc_check(st.ws.data_ptr(), ctypes.c_void_p(st.streams[2].cuda_stream)), "vc_check")
 
     def __call__(self, q_host, k_host, v_host, o_host, stream=None):
-        self.q.copy_(q_host, non_blocking=True)
-        self.k.copy_(k_host, non_blocking=True)
-        self.v.copy_(v_host, non_blocking=True)
-        attention(self.q, self.k, self.v, self.params, out=self.o, prep=self.prep, workspace=self.ws, stream=stream)
-        o_host.copy_(self.o, non_blocking=True)
-        return o_host
+        for t, n in ((q_host, "q_host"), (k_host, "k_host"), (v_host, "v_host"), (o_host, "o_host")):
+            if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or tuple(t.shape) != self.shape:
+                raise ValueError(f"{n} must be a contiguous bf16 host tensor of shape {self.shape}")
+        st = self.sets[self.calls % len(self.sets)]
+        self.calls += 1
+        cur = torch.cuda.current_stream(st.q.device) if stream is None else stream
+        for s in st.streams:
+            s.wait_stream(cur)
+        s_in, s_c, s_out = st.streams
+        rc = lib().vc_attention_host(
+            q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), o_host.data_ptr(), ctypes.byref(_Shape(*self.shape)),
+            ctypes.byref(self.params.c()), self.groups, st.q.data_ptr(), st.k.data_ptr(), st.v.data_ptr(),
+            st.o.data_ptr(), ctypes.byref(_prep_struct(st.prep)), st.ws.data_ptr(), st.ws.numel(),
+            ctypes.c_void_p(s_in.cuda_stream), ctypes.c_void_p(s_c.cuda_stream), ctypes.c_void_p(s_out.cuda_stream))
+        _ok(rc, "vc_attention_host")
+        # The caller's stream moves on once O is back; the next call (other
+        # set) does not wait for this one.
+        return _HostDone(cur, s_out, s_c)
+
+
+class _HostDone:
+    """Returned by HostAttention: `wait()` makes the caller's stream wait for
+    the call's output copy (the call itself leaves the caller's stream free,
+    so consecutive calls overlap)."""
+
+    def __init__(self, cur, s_out, s_c):
+        self._cur, self._s_out, self._s_c = cur, s_out, s_c
+
+    def wait(self):
+        self._cur.wait_stream(self._s_out)
+        self._cur.wait_stream(self._s_c)

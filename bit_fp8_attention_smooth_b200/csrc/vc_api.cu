@@ -307,6 +307,85 @@ vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_sha
     return attn_impl(Q, *scratch, *shape, *params, O, ws, L, s);
 }
 
+vc_status vc_attention_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, const vc_shape* shape,
+                            const vc_params* params, int groups, void* Qd, void* Kd, void* Vd, void* Od,
+                            const vc_prep* scratch, void* workspace, size_t workspace_bytes, void* h2d_stream,
+                            void* compute_stream, void* d2h_stream) {
+    vc_status st = check_shape_params(shape, params);
+    if (st != VC_OK) return st;
+    if (!Qh || !Kh || !Vh || !Oh) return VC_ERR_INVALID_ARG;
+    if (!aligned16(Qd) || !aligned16(Kd) || !aligned16(Vd) || !aligned16(Od) || !aligned16(workspace))
+        return VC_ERR_INVALID_ARG;
+    if ((st = check_prep_ptrs(scratch, false)) != VC_OK) return st;
+    const WsLayout L = ws_layout(*shape, *params);
+    if (workspace_bytes < L.total) return VC_ERR_WORKSPACE;
+    if ((st = check_device()) != VC_OK) return st;
+    const int64_t BH = (int64_t)shape->B * shape->H;
+    const int G = groups < 1 ? 1 : (groups > BH ? (int)BH : groups);
+    const int N = shape->N, D = shape->d, BK = params->block;
+    const int T = (N + BK - 1) / BK;
+    const size_t row = (size_t)N * D * 2;  // bytes of one (b, h) slice of Q, K, V or O
+    cudaStream_t sin = static_cast<cudaStream_t>(h2d_stream);
+    cudaStream_t sc = static_cast<cudaStream_t>(compute_stream);
+    cudaStream_t sout = static_cast<cudaStream_t>(d2h_stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    {   // Work of an earlier call on these streams comes first: its computation
+        // before this call's copies into Qd/Kd/Vd, its copies out of Od before
+        // this call writes Od.
+        cudaEvent_t c_prev = nullptr, o_prev = nullptr;
+        if (cudaEventCreateWithFlags(&c_prev, cudaEventDisableTiming) != cudaSuccess) return VC_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&o_prev, cudaEventDisableTiming) != cudaSuccess) {
+            cudaEventDestroy(c_prev);
+            return VC_ERR_CUDA;
+        }
+        const bool fine = cudaEventRecord(c_prev, sc) == cudaSuccess && cudaEventRecord(o_prev, sout) == cudaSuccess &&
+                          cudaStreamWaitEvent(sin, c_prev, 0) == cudaSuccess &&
+                          cudaStreamWaitEvent(sc, o_prev, 0) == cudaSuccess;
+        cudaEventDestroy(c_prev);
+        cudaEventDestroy(o_prev);
+        if (!fine) return VC_ERR_CUDA;
+    }
+    auto at = [](const void* p, size_t off) { return static_cast<const uint8_t*>(p) + off; };
+    auto atw = [](void* p, size_t off) { return static_cast<uint8_t*>(p) + off; };
+    for (int g = 0; g < G; ++g) {
+        const int64_t h0 = BH * g / G, h1 = BH * (g + 1) / G;
+        const int hg = (int)(h1 - h0);
+        if (hg == 0) continue;
+        const vc_shape gs{1, hg, N, D};
+        const size_t off = (size_t)h0 * row, bytes = (size_t)hg * row;
+        vc_prep gp = *scratch;  // the group's slices of the prep buffers
+        gp.perm = scratch->perm + (size_t)h0 * N;
+        gp.labels = scratch->labels ? scratch->labels + (size_t)h0 * N : nullptr;
+        gp.k_fp8 = scratch->k_fp8 + (size_t)h0 * T * BK * D;
+        gp.k_scale = scratch->k_scale + (size_t)h0 * T;
+        gp.vt_fp8 = scratch->vt_fp8 + (size_t)h0 * D * T * BK;
+        gp.v_mean = scratch->v_mean + (size_t)h0 * T * D;
+        gp.v_scale = scratch->v_scale + (size_t)h0 * D;
+        cudaEvent_t in_done = nullptr, out_ready = nullptr;
+        if (cudaEventCreateWithFlags(&in_done, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&out_ready, cudaEventDisableTiming) != cudaSuccess) {
+            if (in_done) cudaEventDestroy(in_done);
+            return VC_ERR_CUDA;
+        }
+        bool fine = cudaMemcpyAsync(atw(Qd, off), at(Qh, off), bytes, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
+                    cudaMemcpyAsync(atw(Kd, off), at(Kh, off), bytes, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
+                    cudaMemcpyAsync(atw(Vd, off), at(Vh, off), bytes, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
+                    cudaEventRecord(in_done, sin) == cudaSuccess && cudaStreamWaitEvent(sc, in_done, 0) == cudaSuccess;
+        if (fine) {
+            const WsLayout GL = ws_layout(gs, *params);  // a group's layout fits in the full one
+            st = prepare_impl(at(Kd, off), at(Vd, off), gs, *params, gp, ws, GL, sc);
+            if (st == VC_OK) st = attn_impl(at(Qd, off), gp, gs, *params, atw(Od, off), ws, GL, sc);
+            fine = st == VC_OK && cudaEventRecord(out_ready, sc) == cudaSuccess &&
+                   cudaStreamWaitEvent(sout, out_ready, 0) == cudaSuccess &&
+                   cudaMemcpyAsync(atw(Oh, off), at(Od, off), bytes, cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+        }
+        cudaEventDestroy(in_done);  // released once complete
+        cudaEventDestroy(out_ready);
+        if (!fine) return st != VC_OK ? st : VC_ERR_CUDA;
+    }
+    return VC_OK;
+}
+
 vc_status vc_attn_fwd_noalloc(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params,
                               void* O, void* stream) {
     vc_status st = check_shape_params(shape, params);

@@ -150,6 +150,33 @@ vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_sha
                        const vc_prep* scratch, void* O, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * vc_attention from host memory, with the transfers overlapped with the
+ * computation.  The pages describe no such entry point; it serves callers
+ * whose tensors live in host memory (a per-call H2D of Q, K, V and a D2H of
+ * O).  The B*H independent (b, h) problems are split into `groups`
+ * consecutive runs.  Group g's Q, K, V are copied on `h2d_stream`, its V-Smooth
+ * prep and attention run on `compute_stream` once they have landed, and its
+ * O is copied back on `d2h_stream`.  So the copies of group g+1 and g-1
+ * overlap the computation of group g.
+ *   Qh, Kh, Vh   bf16 [B,H,N,d] host input; page-locked (pinned) memory, or
+ *                the copies do not overlap
+ *   Oh           bf16 [B,H,N,d] host output, written asynchronously
+ *   Qd, Kd, Vd, Od, scratch, workspace   device buffers as for vc_attention
+ *                (full shape); workspace >= vc_workspace_bytes(shape)
+ *   groups       1 .. B*H (clamped); 1 = no overlap
+ * Results equal those of vc_attention on the same inputs.  The call only
+ * enqueues: Oh is complete when d2h_stream has reached the end of the call;
+ * vc_check(workspace, d2h_stream) synchronises and reports device errors.
+ * The dependencies between the three streams use CUDA events that the call
+ * creates and releases (released events stay valid until they complete); it
+ * allocates no memory.
+ */
+vc_status vc_attention_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, const vc_shape* shape,
+                            const vc_params* params, int groups, void* Qd, void* Kd, void* Vd, void* Od,
+                            const vc_prep* scratch, void* workspace, size_t workspace_bytes, void* h2d_stream,
+                            void* compute_stream, void* d2h_stream);
+
+/*
  * Allocation-free variant of vc_attn_fwd, for callers that cannot allocate
  * device memory at call time: a host runtime that hands the op only its
  * input and output buffers and owns every other byte, or a real-time loop that
