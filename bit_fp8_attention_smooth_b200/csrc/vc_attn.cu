@@ -217,8 +217,10 @@ __global__ void __launch_bounds__(576, 1)
         };
         auto issue_pv = [&](int t) -> bool {
             const int st = t % STAGES, pb = t & 1;
-            if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
+            // V(t) first (it lands long before the softmax finishes), so PV(t)
+            // is issued as soon as p_full(t) completes
             if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
+            if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint32_t ap = tmem + Cfg::P_COL0 + pb * (BK / 4);
             const uint64_t dv = smem_desc(base + Cfg::OFF_V + st * Cfg::VX_BYTES, BK);
@@ -331,8 +333,11 @@ __global__ void __launch_bounds__(576, 1)
                 const float2 t23 = expcast_t2(A, s[4 * q + 2], s[4 * q + 3], cbm);
                 pw[q] = pack4_low_bytes(t01.x, t01.y, t23.x, t23.y);
             }
-            // P slot sb was last read by the PV MMA of tile t-2.
-            if (t >= 2 && !warp_wait(bar(Cfg::B_PVDONE + sb), ((t - 2) >> 1) & 1, ctl, abort_flag)) break;
+            // P slot sb was last read by the PV MMA of tile t-2.  That MMA has
+            // completed: one elected thread issues every MMA and commit, a
+            // commit tracks all of that thread's earlier MMAs, and QK(t) --
+            // whose commit s_full(t) this warp waited for -- was issued after
+            // PV(t-2).
             tc_fence_after();
             const uint32_t pcol = lane_tmem + Cfg::P_COL0 + sb * (BK / 4) + hf * (HB / 4);
             if constexpr (HB / 4 == 16)
