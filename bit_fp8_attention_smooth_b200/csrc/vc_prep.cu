@@ -458,10 +458,16 @@ __global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties,
 }
 
 // Exclusive scan of hist[bh] in (cluster, block) order -> offs; cluster ranges.
+// The histogram goes through shared memory in chunks of KM_SCAN_CHUNK entries:
+// loaded and stored coalesced, scanned as 1024 contiguous runs of 16 plus a
+// block scan of the run totals, with a carry between chunks.
+constexpr int KM_SCAN_CHUNK = 16 * 1024;
+
 __global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist, int32_t* __restrict__ offs,
                                                 int32_t* __restrict__ cstart, int32_t* __restrict__ ccount,
                                                 KmState* __restrict__ state, int N, int C, int nblk, int it,
                                                 const int* __restrict__ status) {
+    extern __shared__ int h_s[];  // [KM_SCAN_CHUNK]
     __shared__ int s_part[1024];
     __shared__ int s_skip;
     if (ctl_failed(status)) return;
@@ -478,24 +484,35 @@ __global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist
     __syncthreads();
     if (s_skip) return;
     const int64_t L = (int64_t)C * nblk;
-    const int64_t per = (L + 1023) / 1024;
-    const int64_t a = imin64(L, per * tid), b = imin64(L, a + per);
     const int32_t* hh = hist + (size_t)bh * L;
     int32_t* oo = offs + (size_t)bh * L;
-    int s = 0;
-    for (int64_t i = a; i < b; ++i) s += hh[i];
-    s_part[tid] = s;
-    __syncthreads();
-    for (int d = 1; d < 1024; d <<= 1) {
-        const int v = tid >= d ? s_part[tid - d] : 0;
+    int carry = 0;
+    for (int64_t c0 = 0; c0 < L; c0 += KM_SCAN_CHUNK) {
+        const int n = (int)(L - c0 < KM_SCAN_CHUNK ? L - c0 : KM_SCAN_CHUNK);
+        for (int i = tid; i < n; i += 1024) h_s[i] = hh[c0 + i];
         __syncthreads();
-        s_part[tid] += v;
+        const int a = min(n, 16 * tid), b = min(n, a + 16);
+        int sum = 0;
+        for (int i = a; i < b; ++i) sum += h_s[i];
+        s_part[tid] = sum;
         __syncthreads();
-    }
-    int run = s_part[tid] - s;  // exclusive prefix of this segment
-    for (int64_t i = a; i < b; ++i) {
-        oo[i] = run;
-        run += hh[i];
+        for (int d = 1; d < 1024; d <<= 1) {
+            const int v = tid >= d ? s_part[tid - d] : 0;
+            __syncthreads();
+            s_part[tid] += v;
+            __syncthreads();
+        }
+        int run = carry + s_part[tid] - sum;  // exclusive prefix of this run
+        for (int i = a; i < b; ++i) {
+            const int x = h_s[i];
+            h_s[i] = run;
+            run += x;
+        }
+        const int total = s_part[1023];
+        __syncthreads();
+        for (int i = tid; i < n; i += 1024) oo[c0 + i] = h_s[i];
+        carry += total;
+        __syncthreads();
     }
     __syncthreads();
     for (int k = tid; k < C; k += 1024) {
@@ -506,20 +523,28 @@ __global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist
     }
 }
 
+// perm[position] = token, stable within a cluster: a token's position is its
+// cluster's offset for this tile plus the number of earlier tokens of the
+// tile with the same cluster (within its warp by __match_any_sync, plus the
+// counts of the earlier warps).
 __global__ void __launch_bounds__(KM_TOK) km_scatter(const int32_t* __restrict__ labels,
                                                      const int32_t* __restrict__ offs, int32_t* __restrict__ perm,
                                                      const KmState* __restrict__ state, int N, int C,
                                                      const int* __restrict__ status) {
-    __shared__ int lab_s[KM_TOK];
+    __shared__ int cnt_s[KM_TOK / 32][256];
     const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x, r = threadIdx.x;
     if (ctl_failed(status) || state[bh].done) return;
+    const int warp = r >> 5, lane = r & 31;
+    for (int i = r; i < (KM_TOK / 32) * 256; i += KM_TOK) (&cnt_s[0][0])[i] = 0;
     const int j = blk * KM_TOK + r;
     const int L = j < N ? labels[(size_t)bh * N + j] : -1;
-    lab_s[r] = L;
+    const uint32_t same = __match_any_sync(0xffffffffu, L);
     __syncthreads();
-    if (j >= N) return;
-    int rank = 0;
-    for (int q = 0; q < r; ++q) rank += (lab_s[q] == L);
+    if (L >= 0 && lane == __ffs(same) - 1) cnt_s[warp][L] = __popc(same);
+    __syncthreads();
+    if (L < 0) return;
+    int rank = __popc(same & ((1u << lane) - 1));
+    for (int w = 0; w < warp; ++w) rank += cnt_s[w][L];
     perm[(size_t)bh * N + offs[((size_t)bh * C + L) * nblk + blk] + rank] = j;
 }
 
@@ -539,6 +564,7 @@ __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict
     constexpr int TPR = D / 8;    // threads per row
     constexpr int R = 128 / TPR;  // rows per pass
     __shared__ double red[R][D];
+    __shared__ int pp_s[KM_UPD_ROWS];
     __shared__ int seg_s;
     const int bh = blockIdx.y;
     if (ctl_failed(status) || state[bh].done) return;
@@ -554,8 +580,10 @@ __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict
         seg_s = lo;
     }
     __syncthreads();
-    const int32_t* pp = perm + (size_t)bh * N;
     const uint4* vb = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D) + cg;
+    for (int i = tid; i < r1 - r0; i += 128) pp_s[i] = perm[(size_t)bh * N + r0 + i];
+    __syncthreads();
+    const int* pp = pp_s - r0;  // indexed by position
     for (int k = seg_s; k < C; ++k) {
         const int a = max(r0, cs[k]);
         const int b = min(r1, k + 1 < C ? cs[k + 1] : N);
@@ -570,14 +598,12 @@ __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict
             for (int e = 0; e < 8; ++e) acc[e] = __dadd_rn(acc[e], (double)bf2f(h[e]));
         };
         int i = a + rr;
-        for (; i + 3 * R < b; i += 4 * R) {
-            const int t0 = pp[i], t1 = pp[i + R], t2 = pp[i + 2 * R], t3 = pp[i + 3 * R];
-            const uint4 x0 = __ldg(vb + (size_t)t0 * TPR), x1 = __ldg(vb + (size_t)t1 * TPR);
-            const uint4 x2 = __ldg(vb + (size_t)t2 * TPR), x3 = __ldg(vb + (size_t)t3 * TPR);
-            add(x0);
-            add(x1);
-            add(x2);
-            add(x3);
+        for (; i + 7 * R < b; i += 8 * R) {
+            uint4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = __ldg(vb + (size_t)pp[i + u * R] * TPR);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) add(x[u]);
         }
         for (; i < b; i += R) add(__ldg(vb + (size_t)pp[i] * TPR));
 #pragma unroll
@@ -858,6 +884,8 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(km_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, KM_SCAN_CHUNK * sizeof(int));
+        if (e != cudaSuccess) return e;
         configured = true;
     }
     CUtensorMap tv, th, tl;
@@ -873,7 +901,7 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
                                                             it, tpc, p.ctl);
         km_refine<D><<<148 * 8, 256, 0, s>>>(p.ties, p.tie_count, p.V, p.cent64, p.labels, p.hist, p.state, p.N,
                                               p.C, Cp, it, p.ctl.status);
-        km_scan<<<p.BH, 1024, 0, s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it,
+        km_scan<<<p.BH, 1024, KM_SCAN_CHUNK * sizeof(int), s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it,
                                       p.ctl.status);
         km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C,
                                                        p.ctl.status);
