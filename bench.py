@@ -215,7 +215,12 @@ def config_of(w):
 
 
 def launches_per_step(p) -> int:
-    prep = (1 + 3 * p.iters + 2 * (p.iters - 1) + 2) if p.smooth else 4
+    """Kernels of the library one step launches (the launch list in profiles/
+    shows the same sequence): km_init; per k-means pass km_assign, km_refine,
+    km_scan, km_scatter; between passes km_update, km_finalize; then
+    prep_kv_block, prep_v_quant, quant_q and the attention kernel.  V-Smooth
+    off: identity_order, prep_kv_block, prep_v_quant (plus a memset)."""
+    prep = (1 + 4 * p.iters + 2 * (p.iters - 1) + 2) if p.smooth else 3
     return prep + 2
 
 
