@@ -15,21 +15,20 @@
 //                   (E4M3 A operands: 4 values a column).  O's column D
 //                   accumulates the running row sum l: the PV B operand is the
 //                   V^T tile followed by 16 rows of E4M3 ones.
-//   warp 0       TMA producer: K tile, V^T tile and block mean per key tile
-//                through a STAGES-deep ring.
-//   warp 1       TMEM owner and MMA issuer (one thread), kind::f8f6f4:
-//                  S[t%2] = Q K_t^T     (A = Q in TMEM)
-//                  [O|l] += P_t [V_t|1] (A = P_t in TMEM; N = D + 16)
-//   warps 2..9   softmax, two warps per query row (each half of the tile's
-//                scores): they first write the row's E4M3 Q into TMEM; per
-//                tile: row max of S, integer row reference M (raised online;
-//                a rise by k rescales O by 2^-k, exactly), ExpCast bytes
-//                stored to TMEM as the A operand of the PV MMA.
-//   warps 10..17 correction, two warps per row (each half of the channels):
-//                the tile's row sum l_t = l(t) - 2^-k l(t-1) from O's column D,
-//                acc += l_t * mu_t (the block-mean restore), rescaled with O;
-//                epilogue O = (v_scale * O + acc) / l in bf16, original token
-//                order.
+//   warp 0      TMA producer: K tile, V^T tile and block mean per key tile
+//               through a STAGES-deep ring.
+//   warp 1      TMEM owner and MMA issuer (one elected lane), kind::f8f6f4:
+//                 S[t%2] = Q K_t^T     (A = Q in TMEM)
+//                 [O|l] += P_t [V_t|1] (A = P_t in TMEM; N = D + 16)
+//   warps 2..5  softmax, one warp per TMEM lane quadrant, a thread per query
+//               row: it first writes the row's E4M3 Q into TMEM; per tile: row
+//               max of S, integer row reference M (raised online; a rise by k
+//               rescales O and l by 2^-k, exactly), ExpCast bytes stored to
+//               TMEM as the A operand of the PV MMA.
+//   warps 6..9  correction, one warp per quadrant: the tile's row sum
+//               l_t = l(t) - 2^-k l(t-1) from O's column D, acc += l_t * mu_t
+//               (the block-mean restore), rescaled with O; epilogue
+//               O = (v_scale * O + acc) / l in bf16, original token order.
 // Every wait is bounded (DevCtl); on a timeout the CTA drains its copies and
 // MMAs, frees TMEM and exits with the status word set.  A CTA does nothing
 // when the status word already holds an error.
@@ -41,7 +40,7 @@ template <int D, int BK>
 struct AttnCfg {
     static constexpr int BM = 128;
     static constexpr int STAGES = 4;
-    static constexpr int THREADS = 576;  // 18 warps
+    static constexpr int THREADS = 320;  // 10 warps
     static constexpr int K_BYTES = BK * D;
     static constexpr int V_BYTES = D * BK;            // the TMA-loaded V^T tile
     static constexpr int VX_BYTES = (D + 16) * BK;    // + 16 rows of ones (the l column)
@@ -50,9 +49,7 @@ struct AttnCfg {
     static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
     static constexpr int OFF_MU = OFF_V + STAGES * VX_BYTES;
     static constexpr int OFF_KINC = OFF_MU + STAGES * MU_BYTES;
-    static constexpr int OFF_MXEX = OFF_KINC + 4 * BM * 4;
-    static constexpr int OFF_PAIRCNT = OFF_MXEX + 2 * 2 * BM * 4;  // pair-barrier arrivals per softmax warp
-    static constexpr int OFF_BAR = OFF_PAIRCNT + 8 * 4;
+    static constexpr int OFF_BAR = OFF_KINC + 4 * BM * 4;
     // barrier slots
     static constexpr int B_QREADY = 0;
     static constexpr int B_KFULL = 1;
@@ -105,7 +102,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, const 
 }
 
 template <int D, int BK>
-__global__ void __launch_bounds__(576, 1)
+__global__ void __launch_bounds__(320, 1)
     vc_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const AttnArgs args) {
     using Cfg = AttnCfg<D, BK>;
@@ -131,20 +128,20 @@ __global__ void __launch_bounds__(576, 1)
 
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
-        mbar_init(bar(Cfg::B_QREADY), 8);
+        mbar_init(bar(Cfg::B_QREADY), 4);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar(Cfg::B_KFULL + s), 1);
             mbar_init(bar(Cfg::B_KEMPTY + s), 1);
             mbar_init(bar(Cfg::B_VFULL + s), 1);
-            mbar_init(bar(Cfg::B_VEMPTY + s), 1 + 8);
+            mbar_init(bar(Cfg::B_VEMPTY + s), 1 + 4);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(Cfg::B_SFULL + i), 1);
-            mbar_init(bar(Cfg::B_PFULL + i), 8);
+            mbar_init(bar(Cfg::B_PFULL + i), 4);
             mbar_init(bar(Cfg::B_PVDONE + i), 1);
-            mbar_init(bar(Cfg::B_LREAD + i), 8);
+            mbar_init(bar(Cfg::B_LREAD + i), 4);
         }
-        for (int i = 0; i < 4; ++i) mbar_init(bar(Cfg::B_KINC + i), 8);
+        for (int i = 0; i < 4; ++i) mbar_init(bar(Cfg::B_KINC + i), 4);
         mbar_init(bar(Cfg::B_MMADONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -165,7 +162,6 @@ __global__ void __launch_bounds__(576, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const DevCtl ctl = args.ctl;
-    int pair_arrivals = 0;  // softmax warps: arrivals on the pair's named barrier
 
     if (warp == 0) {
         // -------------------------------------------------------- producer
@@ -238,33 +234,27 @@ __global__ void __launch_bounds__(576, 1)
         }
         mma_commit_warp(bar(Cfg::B_MMADONE));
         drain_wait(bar(Cfg::B_MMADONE), 0, ctl);
-    } else if (warp < 10) {
+    } else if (warp < 6) {
         // -------------------------------------------------------- softmax
-        // Two warps per TMEM lane quadrant: warp (qd, hf) handles rows
-        // 32qd..32qd+31, score columns [hf*BK/2, (hf+1)*BK/2).  The pair
-        // exchanges half-row maxima through shared memory.
-        constexpr int HB = BK / 2;
-        constexpr int HD = D / 2;
+        // One warp per TMEM lane quadrant: warp w handles rows
+        // 32qd..32qd+31 (qd = w % 4), a thread the whole row of BK scores.
         const int qd = warp & 3;
-        const int hf = (warp - 2) >> 2;
         const int row = qd * 32 + lane;
         const uint32_t lane_tmem = tmem + ((uint32_t)(qd * 32) << 16);
         const int qrow = q0 + row;
-        {   // this warp's half of the row's E4M3 Q into TMEM (zeros past N)
-            uint32_t qw[HD / 4];
-            const uint4* src = reinterpret_cast<const uint4*>(args.q_fp8 + ((size_t)bh * N + qrow) * D + hf * HD);
+        {   // the row's E4M3 Q into TMEM (zeros past N)
+            uint32_t qw[D / 4];
+            const uint4* src = reinterpret_cast<const uint4*>(args.q_fp8 + ((size_t)bh * N + qrow) * D);
 #pragma unroll
-            for (int i = 0; i < HD / 16; ++i) {
+            for (int i = 0; i < D / 16; ++i) {
                 const uint4 v = qrow < N ? src[i] : make_uint4(0u, 0u, 0u, 0u);
                 qw[4 * i + 0] = v.x;
                 qw[4 * i + 1] = v.y;
                 qw[4 * i + 2] = v.z;
                 qw[4 * i + 3] = v.w;
             }
-            if constexpr (HD / 4 == 16)
-                tmem_st16(lane_tmem + Cfg::Q_COL + hf * (HD / 4), qw);
-            else
-                tmem_st8(lane_tmem + Cfg::Q_COL + hf * (HD / 4), qw);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tmem_st16(lane_tmem + Cfg::Q_COL + 16 * c, qw + 16 * c);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -273,129 +263,101 @@ __global__ void __launch_bounds__(576, 1)
         const float sqv = qrow < N ? args.sq[(size_t)bh * N + qrow] : 0.0f;
         const float aq = __fmul_rn(args.kappa, sqv);
         const float c0 = 56.0f + (float)args.beta;
-        float* mx_ex = reinterpret_cast<float*>(smem + Cfg::OFF_MXEX);  // [tile parity][half][row]
         float M = 0.0f;
         float sk_next = args.k_scale[(size_t)bh * T];
-        bool done = true;
         for (int t = 0; t < T; ++t) {
-            done = false;
             const int sb = t & 1;
             const float sk = sk_next;
             if (t + 1 < T) sk_next = args.k_scale[(size_t)bh * T + t + 1];
             if (!warp_wait(bar(Cfg::B_SFULL + sb), (t >> 1) & 1, ctl, abort_flag)) break;
             tc_fence_after();
-            float s[HB];
+            float s[BK];
 #pragma unroll
-            for (int c = 0; c < HB / 32; ++c)
-                tmem_ld32(lane_tmem + Cfg::S_COL0 + sb * BK + hf * HB + 32 * c, s + 32 * c);
-            // read after this warp's last pair barrier, in the shadow of the
-            // TMEM load: enough to stop before the next one (below)
-            const int abort_seen = *abort_flag;
+            for (int c = 0; c < BK / 32; ++c) tmem_ld32(lane_tmem + Cfg::S_COL0 + sb * BK + 32 * c, s + 32 * c);
             tmem_wait_ld();
 
-            const int valid = N - t * BK - hf * HB;
-            if (valid < HB) {
+            const int valid = N - t * BK;
+            if (valid < BK) {
 #pragma unroll
-                for (int j = 0; j < HB; ++j)
+                for (int j = 0; j < BK; ++j)
                     if (j >= valid) s[j] = -INFINITY;
             }
-            // half-row max: 8 independent 3-input max chains, then a short tree
+            // row max: 8 independent 3-input max chains, then a short tree
             float m8[8];
 #pragma unroll
             for (int a = 0; a < 8; ++a) m8[a] = fmaxf(s[2 * a], s[2 * a + 1]);
 #pragma unroll
-            for (int j = 16; j < HB; j += 16)
+            for (int j = 16; j < BK; j += 16)
 #pragma unroll
                 for (int a = 0; a < 8; ++a) m8[a] = fmax3(m8[a], s[j + 2 * a], s[j + 2 * a + 1]);
-            const float mh =
+            const float mx =
                 fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-            mx_ex[((t & 1) * 2 + hf) * Cfg::BM + row] = mh;
-            // The pair meets on named barrier 1 + qd.  A warp never enters it
-            // once it has seen the CTA abort (its partner may have left); a
-            // warp that leaves early arrives once more instead, which frees a
-            // partner already waiting there (see the teardown for the balance).
-            // An abort that frees a waiting partner is visible to it through
-            // the barrier, so the partner stops before its next meeting.
-            if (__any_sync(0xffffffffu, abort_seen != 0)) break;
-            named_barrier_sync(1 + qd, 64);
-            ++pair_arrivals;
-            const float mx = fmaxf(mh, mx_ex[((t & 1) * 2 + (1 - hf)) * Cfg::BM + row]);
             const float A = __fmul_rn(aq, sk);
             const float Mc = ceilf(__fmul_rn(__fmul_rn(A, mx), 0.125f));
             const float Mnew = t == 0 ? Mc : fmaxf(M, Mc);
             const int kinc = t == 0 ? 0 : (int)(Mnew - M);
             M = Mnew;
             const float cbm = (c0 - 8.0f * M) + kMagic;
-            uint32_t pw[HB / 4];
-#pragma unroll
-            for (int q = 0; q < HB / 4; ++q) {
-                const float2 t01 = expcast_t2(A, s[4 * q], s[4 * q + 1], cbm);
-                const float2 t23 = expcast_t2(A, s[4 * q + 2], s[4 * q + 3], cbm);
-                pw[q] = pack4_low_bytes(t01.x, t01.y, t23.x, t23.y);
-            }
             // P slot sb was last read by the PV MMA of tile t-2.  That MMA has
             // completed: one elected thread issues every MMA and commit, a
             // commit tracks all of that thread's earlier MMAs, and QK(t) --
             // whose commit s_full(t) this warp waited for -- was issued after
             // PV(t-2).
-            tc_fence_after();
-            const uint32_t pcol = lane_tmem + Cfg::P_COL0 + sb * (BK / 4) + hf * (HB / 4);
-            if constexpr (HB / 4 == 16)
-                tmem_st16(pcol, pw);
-            else
-                tmem_st8(pcol, pw);
+            const uint32_t pcol = lane_tmem + Cfg::P_COL0 + sb * (BK / 4);
+#pragma unroll
+            for (int c = 0; c < BK / 64; ++c) {  // 64 scores -> 16 words of bytes
+                uint32_t pw[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float* sp = s + 64 * c + 4 * q;
+                    const float2 t01 = expcast_t2(A, sp[0], sp[1], cbm);
+                    const float2 t23 = expcast_t2(A, sp[2], sp[3], cbm);
+                    pw[q] = pack4_low_bytes(t01.x, t01.y, t23.x, t23.y);
+                }
+                tmem_st16(pcol + 16 * c, pw);
+            }
             if (t > 0 && __any_sync(0xffffffffu, kinc > 0)) {
-                // O holds PV of tiles < t: wait for it, then scale this warp's
-                // half of the O columns by 2^-kinc (before this tile's PV,
-                // which waits on p_full below).
+                // O holds PV of tiles < t: wait for it, then scale O and l by
+                // 2^-kinc (before this tile's PV, which waits on p_full below).
                 if (!warp_wait(bar(Cfg::B_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) break;
-                // ... and for the correction warps to have read l after PV(t-1)
+                // ... and for the correction warp to have read l after PV(t-1)
                 if (!warp_wait(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) break;
                 tc_fence_after();
                 const float f = exp2_neg_int(kinc);
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     float o[32];
-                    tmem_ld32(lane_tmem + Cfg::O_COL + hf * HD + 32 * c, o);
+                    tmem_ld32(lane_tmem + Cfg::O_COL + 32 * c, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= f;
-                    tmem_st32(lane_tmem + Cfg::O_COL + hf * HD + 32 * c, o);
+                    tmem_st32(lane_tmem + Cfg::O_COL + 32 * c, o);
                 }
-                if (hf == 1) {  // the running row sum l, column D
-                    float lv = tmem_ld1(lane_tmem + Cfg::L_COL);
-                    tmem_wait_ld();
-                    lv *= f;
-                    tmem_st1(lane_tmem + Cfg::L_COL, lv);
-                }
+                float lv = tmem_ld1(lane_tmem + Cfg::L_COL);
+                tmem_wait_ld();
+                lv *= f;
+                tmem_st1(lane_tmem + Cfg::L_COL, lv);
             }
             tmem_wait_st();
-            if (hf == 0) kinc_ring[(t & 3) * Cfg::BM + row] = kinc;
+            kinc_ring[(t & 3) * Cfg::BM + row] = kinc;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(Cfg::B_PFULL + sb));
                 mbar_arrive(bar(Cfg::B_KINC + (t & 3)));
             }
-            done = true;
-        }
-        if (!done) {
-            named_barrier_arrive(1 + qd, 64);
-            ++pair_arrivals;
         }
     } else {
         // -------------------------------------------------------- correction + epilogue
-        // Two warps per lane quadrant: warp (qd, hf) owns output channels
-        // [hf*D/2, (hf+1)*D/2) of rows 32qd..32qd+31.
-        constexpr int HD = D / 2;
+        // One warp per lane quadrant: warp w owns every output channel of
+        // rows 32qd..32qd+31 (qd = w % 4).
         const int qd = warp & 3;
-        const int hf = (warp - 10) >> 2;
         const int row = qd * 32 + lane;
         const uint32_t lane_tmem = tmem + ((uint32_t)(qd * 32) << 16);
         const int qrow = q0 + row;
-        float acc[HD];
+        float acc[D];
 #pragma unroll
-        for (int c = 0; c < HD; ++c) acc[c] = 0.0f;
+        for (int c = 0; c < D; ++c) acc[c] = 0.0f;
         float l = 0.0f;  // running row sum after the last tile seen
         bool ok = true;
         for (int t = 0; t < T; ++t) {
@@ -414,16 +376,15 @@ __global__ void __launch_bounds__(576, 1)
             if (kinc > 0) {
                 const float f = exp2_neg_int(kinc);
 #pragma unroll
-                for (int c = 0; c < HD; ++c) acc[c] *= f;
+                for (int c = 0; c < D; ++c) acc[c] *= f;
                 lb = lt - l * f;
             } else {
                 lb = lt - l;
             }
             l = lt;
-            const float4* mu =
-                reinterpret_cast<const float4*>(smem + Cfg::OFF_MU + st * Cfg::MU_BYTES) + hf * (HD / 4);
+            const float4* mu = reinterpret_cast<const float4*>(smem + Cfg::OFF_MU + st * Cfg::MU_BYTES);
 #pragma unroll
-            for (int c4 = 0; c4 < HD / 4; ++c4) {
+            for (int c4 = 0; c4 < D / 4; ++c4) {
                 const float4 m = mu[c4];
                 const float2 a01 = ffma2(make_float2(lb, lb), make_float2(m.x, m.y),
                                          make_float2(acc[4 * c4 + 0], acc[4 * c4 + 1]));
@@ -441,12 +402,12 @@ __global__ void __launch_bounds__(576, 1)
             // The last PV (tile T-1) has completed, so O is final.
             tc_fence_after();
             const float inv_l = 1.0f / l;
-            const float* vsc = args.v_scale + (size_t)bh * D + hf * HD;
-            __nv_bfloat16* orow = args.out + ((size_t)bh * N + qrow) * D + hf * HD;
+            const float* vsc = args.v_scale + (size_t)bh * D;
+            __nv_bfloat16* orow = args.out + ((size_t)bh * N + qrow) * D;
 #pragma unroll
-            for (int c = 0; c < HD / 16; ++c) {
+            for (int c = 0; c < D / 16; ++c) {
                 float o[16];
-                tmem_ld16(lane_tmem + Cfg::O_COL + hf * HD + 16 * c, o);
+                tmem_ld16(lane_tmem + Cfg::O_COL + 16 * c, o);
                 tmem_wait_ld();
                 uint32_t packed[8];
 #pragma unroll
@@ -467,17 +428,9 @@ __global__ void __launch_bounds__(576, 1)
     }
 
     // ------------------------------------------------------------ teardown
-    int* pair_cnt = reinterpret_cast<int*>(smem + Cfg::OFF_PAIRCNT);
-    if (warp >= 2 && warp < 10) {
-        tmem_wait_st();  // an aborted softmax warp may hold a pending store
-        if (lane == 0) pair_cnt[warp - 2] = pair_arrivals;
-    }
+    if (warp >= 2 && warp < 6) tmem_wait_st();  // an aborted softmax warp may hold a pending store
     tc_fence_before();
     __syncthreads();
-    // After an abort one generation of a pair barrier may hold a single
-    // warp's arrival: complete it, so no barrier is left half-way.
-    if (warp >= 2 && warp < 6 && ((pair_cnt[warp - 2] + pair_cnt[warp + 2]) & 1))
-        named_barrier_arrive(1 + (warp & 3), 64);
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
