@@ -216,6 +216,11 @@ __global__ void __launch_bounds__(320, 1)
             // V(t) first (it lands long before the softmax finishes), so PV(t)
             // is issued as soon as p_full(t) completes
             if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
+            // PV(t) adds into O's l column: the correction warps must have read
+            // l(t-1) first (they do so as soon as PV(t-1) lands, long before
+            // the softmax posts P(t))
+            if (t > 0 && !warp_wait(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag))
+                return false;
             if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint32_t ap = tmem + Cfg::P_COL0 + pb * (BK / 4);
@@ -298,6 +303,11 @@ __global__ void __launch_bounds__(320, 1)
             const int kinc = t == 0 ? 0 : (int)(Mnew - M);
             M = Mnew;
             const float cbm = (c0 - 8.0f * M) + kMagic;
+            // k goes out at once: the correction warps scale l by 2^-k when
+            // they read it after PV(t-1)
+            kinc_ring[(t & 3) * Cfg::BM + row] = kinc;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(Cfg::B_KINC + (t & 3)));
             // P slot sb was last read by the PV MMA of tile t-2.  That MMA has
             // completed: one elected thread issues every MMA and commit, a
             // commit tracks all of that thread's earlier MMAs, and QK(t) --
@@ -310,42 +320,30 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const float* sp = s + 64 * c + 4 * q;
-                    const float2 t01 = expcast_t2(A, sp[0], sp[1], cbm);
-                    const float2 t23 = expcast_t2(A, sp[2], sp[3], cbm);
-                    pw[q] = pack4_low_bytes(t01.x, t01.y, t23.x, t23.y);
+                    pw[q] = expcast4(A, sp[0], sp[1], sp[2], sp[3], cbm);
                 }
                 tmem_st16(pcol + 16 * c, pw);
             }
             if (t > 0 && __any_sync(0xffffffffu, kinc > 0)) {
-                // O holds PV of tiles < t: wait for it, then scale O and l by
-                // 2^-kinc (before this tile's PV, which waits on p_full below).
+                // O holds PV of tiles < t: wait for it, then scale O by 2^-kinc
+                // (before this tile's PV, which waits on p_full below; l is
+                // scaled by the correction warps).  All of O in one round trip.
                 if (!warp_wait(bar(Cfg::B_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) break;
-                // ... and for the correction warp to have read l after PV(t-1)
-                if (!warp_wait(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) break;
                 tc_fence_after();
                 const float f = exp2_neg_int(kinc);
+                float o[D];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    float o[32];
-                    tmem_ld32(lane_tmem + Cfg::O_COL + 32 * c, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] *= f;
-                    tmem_st32(lane_tmem + Cfg::O_COL + 32 * c, o);
-                }
-                float lv = tmem_ld1(lane_tmem + Cfg::L_COL);
+                for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_tmem + Cfg::O_COL + 32 * c, o + 32 * c);
                 tmem_wait_ld();
-                lv *= f;
-                tmem_st1(lane_tmem + Cfg::L_COL, lv);
+#pragma unroll
+                for (int i = 0; i < D; ++i) o[i] *= f;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) tmem_st32(lane_tmem + Cfg::O_COL + 32 * c, o + 32 * c);
             }
             tmem_wait_st();
-            kinc_ring[(t & 3) * Cfg::BM + row] = kinc;
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(Cfg::B_PFULL + sb));
-                mbar_arrive(bar(Cfg::B_KINC + (t & 3)));
-            }
+            if (lane == 0) mbar_arrive(bar(Cfg::B_PFULL + sb));
         }
     } else {
         // -------------------------------------------------------- correction + epilogue
@@ -359,22 +357,35 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int c = 0; c < D; ++c) acc[c] = 0.0f;
         float l = 0.0f;  // running row sum after the last tile seen
-        bool ok = true;
-        for (int t = 0; t < T; ++t) {
+        // k of tile 0 (always 0); each later tile's k is read one iteration
+        // early, to scale l before that tile's PV.
+        bool ok = T == 0 || warp_wait(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag);
+        int kinc = 0;
+        for (int t = 0; ok && t < T; ++t) {
             const int st = t % STAGES;
-            if (!(ok = warp_wait(bar(Cfg::B_KINC + (t & 3)), (t >> 2) & 1, ctl, abort_flag))) break;
-            const int kinc = kinc_ring[(t & 3) * Cfg::BM + row];
             if (!(ok = warp_wait(bar(Cfg::B_PVDONE + (t & 1)), (t >> 1) & 1, ctl, abort_flag))) break;
             tc_fence_after();
             const float lt = tmem_ld1(lane_tmem + Cfg::L_COL);
             tmem_wait_ld();
+            const int kt = kinc;  // this tile's k
+            if (t + 1 < T) {
+                // l(t) * 2^-k(t+1) into O's l column (exact), before PV(t+1),
+                // which waits for l_read(t); the softmax scales the rest of O
+                const int tn = t + 1;
+                if (!(ok = warp_wait(bar(Cfg::B_KINC + (tn & 3)), (tn >> 2) & 1, ctl, abort_flag))) break;
+                kinc = kinc_ring[(tn & 3) * Cfg::BM + row];
+                if (__any_sync(0xffffffffu, kinc > 0)) {
+                    tmem_st1(lane_tmem + Cfg::L_COL, lt * exp2_neg_int(kinc));
+                    tmem_wait_st();
+                }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(Cfg::B_LREAD + (t & 1)));
             if (!(ok = warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag))) break;
             float lb;
-            if (kinc > 0) {
-                const float f = exp2_neg_int(kinc);
+            if (kt > 0) {
+                const float f = exp2_neg_int(kt);
 #pragma unroll
                 for (int c = 0; c < D; ++c) acc[c] *= f;
                 lb = lt - l * f;
@@ -469,8 +480,7 @@ cudaError_t launch_attn(int D, int BK, const CUtensorMap& tk, const CUtensorMap&
 __global__ void vc_expcast_kernel(const float* A, const float* s, const float* cb, uint8_t* out, int64_t n) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const float cbm = cb[i] + kMagic;
-        const float2 t = expcast_t2(A[i], s[i], s[i], cbm);
-        out[i] = (uint8_t)(__float_as_uint(t.x) & 0xFFu);
+        out[i] = (uint8_t)(expcast4(A[i], s[i], s[i], s[i], s[i], cbm) & 0xFFu);
     }
 }
 

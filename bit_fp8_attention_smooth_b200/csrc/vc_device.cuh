@@ -254,6 +254,13 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// 8 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
 // 16 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
     uint32_t* r = reinterpret_cast<uint32_t*>(v);
@@ -333,23 +340,29 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// One FMA per score: t = A*s + cbm with cbm = cb + 1.5*2^23 (cb an integer,
-// |cb| < 2^22) rounds A*s + cb to the integer n in t's low mantissa bits.  The
-// clamp n -> max(n, 0) stays on the FMA pipe and is exact:
-// sat(t * 2^-23 - 1.5) = max(n, 0) * 2^-23 (saturation also sends -inf and
-// NaN to 0), and w * 2^23 + 1.5*2^23 puts max(n, 0) back into the low bits.
-// The byte is the low 8 bits.  Scores go in pairs through the packed FMA.
-__device__ __forceinline__ float2 expcast_t2(float A, float s0, float s1, float cbm) {
-    const float2 t = ffma2(make_float2(A, A), make_float2(s0, s1), make_float2(cbm, cbm));
-    float w0, w1;
-    asm("fma.rn.sat.f32 %0, %1, 0f34000000, 0fBFC00000;" : "=f"(w0) : "f"(t.x));
-    asm("fma.rn.sat.f32 %0, %1, 0f34000000, 0fBFC00000;" : "=f"(w1) : "f"(t.y));
-    return ffma2(make_float2(w0, w1), make_float2(8388608.0f, 8388608.0f), make_float2(kMagic, kMagic));
+// Four ExpCast bytes in one word (byte j from s_j), exactly
+// clamp(round_half_even(A*s + cb), 0, 255) for an integer cb, |cb| < 2^22:
+//  1. t = A*s + cbm, cbm = cb + 1.5*2^23: the packed FMA rounds A*s + cb, once,
+//     to the integer n held in t's low mantissa bits (the one FMA per score).
+//  2. w = t * 2^-149 - 1.5*2^-126 = n * 2^-149, exactly: a subnormal whose bit
+//     pattern, read as int32, is n (n < 0, -inf included, gives a negative int).
+//  3. cvt.pack.sat.u8.s32 clamps two such ints to [0, 255] and packs them.
+// Six instructions for four scores, all exact.
+__device__ __forceinline__ uint32_t pack2_sat_u8(int32_t hi, int32_t lo, uint32_t upper) {
+    // [sat(lo), sat(hi), upper.b0, upper.b1] from byte 0 up
+    uint32_t d;
+    asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(hi), "r"(lo), "r"(upper));
+    return d;
 }
-__device__ __forceinline__ uint32_t pack4_low_bytes(float a, float b, float c, float d) {
-    const uint32_t lo = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
-    const uint32_t hi = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
-    return __byte_perm(lo, hi, 0x5410);
+__device__ __forceinline__ uint32_t expcast4(float A, float s0, float s1, float s2, float s3, float cbm) {
+    const float2 t01 = ffma2(make_float2(A, A), make_float2(s0, s1), make_float2(cbm, cbm));
+    const float2 t23 = ffma2(make_float2(A, A), make_float2(s2, s3), make_float2(cbm, cbm));
+    const float k = __uint_as_float(1u);             // 2^-149
+    const float mk = __uint_as_float(0x80C00000u);   // -1.5 * 2^-126 = -(1.5*2^23) * 2^-149
+    const float2 w01 = ffma2(t01, make_float2(k, k), make_float2(mk, mk));
+    const float2 w23 = ffma2(t23, make_float2(k, k), make_float2(mk, mk));
+    const uint32_t hi = pack2_sat_u8(__float_as_int(w23.y), __float_as_int(w23.x), 0u);
+    return pack2_sat_u8(__float_as_int(w01.y), __float_as_int(w01.x), hi);
 }
 
 }  // namespace vc
