@@ -54,7 +54,13 @@ def lib():
             "vo_quant_q": (None, [P, i32, i32, P, P]),
             "vo_quant_k": (None, [P, i32, i32, i32, P, P, P]),
             "vo_smooth_v": (None, [P, i32, i32, i32, P, i32, P, P, P]),
-            "vo_attn_emul": (None, [P, P, i32, P, P, P, P, P, i32, i32, i32, f64, i32, i32, P, P, P]),
+            "vo_e2m1_value": (f64, [ctypes.c_uint8]),
+            "vo_e2m1_encode": (ctypes.c_uint8, [f32]),
+            "vo_e2m1_value_array": (None, [P, i64, P]),
+            "vo_e2m1_encode_array": (None, [P, i64, P]),
+            "vo_nvfp4_block_array": (None, [P, i64, i32, P, P]),
+            "vo_smooth_v_nvfp4": (None, [P, i32, i32, i32, P, i32, P, P, P, P]),
+            "vo_attn_emul": (None, [P, P, i32, P, P, P, P, P, i32, i32, i32, f64, i32, i32, i32, P, P, P]),
             "vo_attn_exact": (None, [P, P, P, P, i32, i32, i32, P]),
         }
         for name, (res, args) in sig.items():
@@ -87,6 +93,32 @@ def e4m3_encode(x) -> np.ndarray:
     out = np.empty(x.shape, np.uint8)
     lib().vo_e4m3_encode_array(_p(x), x.size, _p(out))
     return out
+
+
+def e2m1_value(codes) -> np.ndarray:
+    c = _c(codes, np.uint8)
+    out = np.empty(c.shape, np.float64)
+    lib().vo_e2m1_value_array(_p(c), c.size, _p(out))
+    return out
+
+
+def e2m1_encode(x) -> np.ndarray:
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().vo_e2m1_encode_array(_p(x), x.size, _p(out))
+    return out
+
+
+def nvfp4_blocks(x) -> tuple[np.ndarray, np.ndarray]:
+    """NVFP4 coding of the blocks along the last axis of x (length <= 16):
+    returns (E2M1 codes shaped like x, UE4M3 scales shaped x.shape[:-1])."""
+    x = _c(x, np.float32)
+    n = x.shape[-1]
+    assert 1 <= n <= 16
+    codes = np.empty(x.shape, np.uint8)
+    scales = np.empty(x.shape[:-1], np.uint8)
+    lib().vo_nvfp4_block_array(_p(x), x.size // n, n, _p(codes), _p(scales))
+    return codes, scales
 
 
 def expcast_bytes(A, s, cb) -> np.ndarray:
@@ -149,8 +181,31 @@ def smooth_v(v_bits: np.ndarray, perm: np.ndarray, bk: int, smooth: bool = True)
     return vhat, vmu, vsc
 
 
-def prep_head(k_bits, v_bits, *, C: int, iters: int, bk: int, smooth: bool = True):
-    """The whole V-Smooth prep of one head, step by step."""
+def smooth_v_nvfp4(v_bits: np.ndarray, perm: np.ndarray, bk: int, smooth: bool = True):
+    """4-bit residual: E2M1 codes vq [T*bk, d], UE4M3 block scales vgs
+    [T, bk/16, d], block means vmu [T, d], channel scales vsc [d]."""
+    v = _c(v_bits, np.uint16)
+    n, d = v.shape
+    T = -(-n // bk)
+    vq = np.empty((T * bk, d), np.uint8)
+    vgs = np.empty((T, bk // 16, d), np.uint8)
+    vmu = np.empty((T, d), np.float32)
+    vsc = np.empty(d, np.float32)
+    lib().vo_smooth_v_nvfp4(_p(v), n, d, bk, _p(_c(perm, np.int32)), int(smooth), _p(vq), _p(vgs), _p(vmu),
+                            _p(vsc))
+    return vq, vgs, vmu, vsc
+
+
+def nvfp4_v_values(vq: np.ndarray, vgs: np.ndarray) -> np.ndarray:
+    """Residual values in channel-scale units: value(block scale) * value(code)."""
+    T, G, d = vgs.shape
+    sv = np.repeat(e4m3_value(vgs), 16, axis=1).reshape(T * G * 16, d)
+    return sv * e2m1_value(vq)
+
+
+def prep_head(k_bits, v_bits, *, C: int, iters: int, bk: int, smooth: bool = True, resid_fmt: int = 0):
+    """The whole V-Smooth prep of one head, step by step (resid_fmt 1: the
+    4-bit residual, whose outputs add vq and vgs in place of vhat)."""
     n = v_bits.shape[0]
     if smooth:
         labels, cent = kmeans(v_bits, C, iters)
@@ -159,6 +214,10 @@ def prep_head(k_bits, v_bits, *, C: int, iters: int, bk: int, smooth: bool = Tru
         labels, cent = np.zeros(n, np.int32), None
         perm = np.arange(n, dtype=np.int32)
     khat, ksc = quant_k(k_bits, perm, bk)
+    if resid_fmt == 1:
+        vq, vgs, vmu, vsc = smooth_v_nvfp4(v_bits, perm, bk, smooth)
+        return dict(labels=labels, centroids=cent, perm=perm, khat=khat, ksc=ksc, vq=vq, vgs=vgs, vmu=vmu,
+                    vsc=vsc)
     vhat, vmu, vsc = smooth_v(v_bits, perm, bk, smooth)
     return dict(labels=labels, centroids=cent, perm=perm, khat=khat, ksc=ksc, vhat=vhat, vmu=vmu, vsc=vsc)
 
@@ -170,8 +229,9 @@ def _chunks(nrows: int, parts: int):
 
 
 def attn_emul(qv, sq, kv, ksc, rv, vmu, vsc, *, n: int, bk: int, beta: int, exact: bool = False,
-              kappa_value: float | None = None, threads: int | None = None):
-    """Replay of the attention forward over the given query rows (values)."""
+              pfmt: int = 0, kappa_value: float | None = None, threads: int | None = None):
+    """Replay of the attention forward over the given query rows (values);
+    pfmt 1 re-codes each 16-key block of P to NVFP4 (the 4-bit path)."""
     qv, sq = _c(qv, np.float64), _c(sq, np.float32)
     kv, ksc, rv = _c(kv, np.float64), _c(ksc, np.float32), _c(rv, np.float64)
     vmu, vsc = _c(vmu, np.float32), _c(vsc, np.float32)
@@ -188,7 +248,7 @@ def attn_emul(qv, sq, kv, ksc, rv, vmu, vsc, *, n: int, bk: int, beta: int, exac
         if b <= a:
             return
         L.vo_attn_emul(_p(qv[a:b]), _p(sq[a:b]), b - a, _p(kv), _p(ksc), _p(rv), _p(vmu), _p(vsc), n, d, bk,
-                       kap, int(beta), int(exact), _p(out[a:b]), _p(M[a:b]), _p(l[a:b]))
+                       kap, int(beta), int(exact), int(pfmt), _p(out[a:b]), _p(M[a:b]), _p(l[a:b]))
 
     threads = threads or os.cpu_count() or 1
     with ThreadPoolExecutor(threads) as ex:
@@ -214,16 +274,17 @@ def attn_exact(q_bits, k_bits, v_bits, rows, threads: int | None = None) -> np.n
 
 
 def forward_head(q_bits, k_bits, v_bits, rows, *, C: int, iters: int, bk: int, beta: int,
-                 smooth: bool = True, prep=None, threads: int | None = None):
-    """V-Smooth prep plus the quantised attention replay for selected rows of one head."""
+                 smooth: bool = True, resid_fmt: int = 0, prep=None, threads: int | None = None):
+    """V-Smooth prep plus the quantised attention replay for selected rows of
+    one head (resid_fmt 1: 4-bit residual and NVFP4 P in the PV product)."""
     n, d = k_bits.shape
     if prep is None:
-        prep = prep_head(k_bits, v_bits, C=C, iters=iters, bk=bk, smooth=smooth)
+        prep = prep_head(k_bits, v_bits, C=C, iters=iters, bk=bk, smooth=smooth, resid_fmt=resid_fmt)
     rows = np.asarray(rows, dtype=np.int64)
     qhat, sq = quant_q(np.asarray(q_bits)[rows])
-    out, M, l = attn_emul(e4m3_value(qhat), sq, e4m3_value(prep["khat"]), prep["ksc"],
-                          e4m3_value(prep["vhat"]), prep["vmu"], prep["vsc"], n=n, bk=bk, beta=beta,
-                          threads=threads)
+    rv = nvfp4_v_values(prep["vq"], prep["vgs"]) if resid_fmt == 1 else e4m3_value(prep["vhat"])
+    out, M, l = attn_emul(e4m3_value(qhat), sq, e4m3_value(prep["khat"]), prep["ksc"], rv, prep["vmu"],
+                          prep["vsc"], n=n, bk=bk, beta=beta, pfmt=resid_fmt, threads=threads)
     return dict(prep=prep, qhat=qhat, sq=sq, out=out, M=M, l=l)
 
 

@@ -39,6 +39,16 @@
  *     beta an integer, a single rounding of the exact value.
  *   - Mean restore: O += l_b * mu_b per tile with l_b = sum of the decoded
  *     bytes of the tile, all terms rescaled by 2^-k when M rises by k.
+ *   - NVFP4 (the 4-bit residual [MarkTechPost]: "per-channel E4M3/NVFP4
+ *     residuals"): E2M1 values (OCP MX FP4: sign, 2 exponent bits with bias 1,
+ *     1 mantissa bit; max 6) in blocks of 16 along the reduction axis, each
+ *     block with a UE4M3 scale s = E4M3(amax/6); a value x is coded
+ *     E2M1(x * (1/s)), with 1/s and the product rounded to fp32, E2M1 rounding
+ *     to nearest (ties to the even code) and saturating at 6; a zero scale
+ *     codes zeros.  The V residual keeps one fp32 scale per channel,
+ *     s_c = amax_c/(6*448), before its 16-token blocks.  The PV product of the
+ *     4-bit path takes P in the same 16-key blocks, re-coded from the ExpCast
+ *     byte's E4M3 value.
  */
 #include <math.h>
 #include <stdint.h>
@@ -110,6 +120,69 @@ VO_API void vo_e4m3_encode_array(const float* x, int64_t n, uint8_t* out) {
 
 VO_API void vo_e4m3_value_array(const uint8_t* c, int64_t n, double* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = vo_e4m3_value(c[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 codec (OCP MX FP4), from the format definition: sign bit 3, exponent  */
+/* bits 2..1 (bias 1), mantissa bit 0; exponent field 0 is subnormal (m/2).   */
+/* No infinities or NaN; the largest magnitude is 6.                          */
+/* ------------------------------------------------------------------------ */
+VO_API double vo_e2m1_value(uint8_t code) {
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double v = e == 0 ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, e - 1);
+    return sign ? -v : v;
+}
+
+/* Nearest E2M1 value, ties to the even code, saturating to +-6. */
+VO_API uint8_t vo_e2m1_encode(float x) {
+    uint8_t sign = signbit(x) ? 0x8 : 0x0;
+    double a = fabs((double)x);
+    if (a >= 6.0) return sign | 0x7;
+    int lo = 0; /* value(lo) <= a < value(lo + 1) */
+    while (lo < 7 && vo_e2m1_value((uint8_t)(lo + 1)) <= a) ++lo;
+    double dlo = a - vo_e2m1_value((uint8_t)lo);
+    double dhi = vo_e2m1_value((uint8_t)(lo + 1)) - a;
+    int code;
+    if (dlo < dhi)
+        code = lo;
+    else if (dhi < dlo)
+        code = lo + 1;
+    else
+        code = (lo & 1) ? lo + 1 : lo;
+    return sign | (uint8_t)code;
+}
+
+VO_API void vo_e2m1_value_array(const uint8_t* c, int64_t n, double* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = vo_e2m1_value(c[i]);
+}
+
+VO_API void vo_e2m1_encode_array(const float* x, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = vo_e2m1_encode(x[i]);
+}
+
+/* One NVFP4 block of n <= 16 values: the UE4M3 scale s = E4M3(amax/6) (the
+ * quotient in fp32), then each code E2M1(x * r) with r = 1/value(s) in fp32.
+ * A zero scale gives zero codes. */
+VO_API void vo_nvfp4_block(const float* x, int n, uint8_t* codes, uint8_t* scale) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+    uint8_t s = vo_e4m3_encode(amax / 6.0f);
+    float sv = (float)vo_e4m3_value(s);
+    *scale = s;
+    if (sv == 0.0f) {
+        for (int i = 0; i < n; ++i) codes[i] = 0;
+        return;
+    }
+    float r = 1.0f / sv;
+    for (int i = 0; i < n; ++i) codes[i] = vo_e2m1_encode(x[i] * r);
+}
+
+/* nblocks consecutive blocks of len values each */
+VO_API void vo_nvfp4_block_array(const float* x, int64_t nblocks, int len, uint8_t* codes, uint8_t* scales) {
+    for (int64_t b = 0; b < nblocks; ++b) vo_nvfp4_block(x + b * len, len, codes + b * len, scales + b);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -297,6 +370,61 @@ VO_API void vo_smooth_v(const uint16_t* v, int n, int d, int bk, const int32_t* 
     free(inv);
 }
 
+/* The 4-bit residual [MarkTechPost] ("per-channel E4M3/NVFP4 residuals"): the
+ * same block means and residuals as vo_smooth_v; per channel one fp32 scale
+ * s_c = amax_c/(6*448), y = r * (6*448/amax_c); then NVFP4 blocks of 16
+ * consecutive tokens of a channel inside each hardware block (bk a multiple of
+ * 16; padding tokens count as 0).
+ * vq [T*bk*d] E2M1 codes token-major (padding rows zero), vgs [T*(bk/16)*d]
+ * UE4M3 block scales ([T][bk/16][d]), vmu [T*d], vsc [d]. */
+VO_API void vo_smooth_v_nvfp4(const uint16_t* v, int n, int d, int bk, const int32_t* perm, int smooth, uint8_t* vq,
+                              uint8_t* vgs, float* vmu, float* vsc) {
+    int T = (n + bk - 1) / bk;
+    int G = bk / 16;
+    float* amax = (float*)calloc((size_t)d, sizeof(float));
+    float* inv = (float*)calloc((size_t)d, sizeof(float));
+    float* y = (float*)malloc(sizeof(float) * (size_t)bk * d);
+    float x[16];
+    uint8_t codes[16];
+    memset(vq, 0, (size_t)T * bk * d);
+    for (int b = 0; b < T; ++b) {
+        int valid = (n - b * bk) < bk ? (n - b * bk) : bk;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            if (smooth)
+                for (int r = 0; r < valid; ++r) s += (double)bf16_to_float(v[(size_t)perm[b * bk + r] * d + c]);
+            vmu[(size_t)b * d + c] = smooth ? (float)(s / (double)valid) : 0.0f;
+        }
+        for (int r = 0; r < valid; ++r)
+            for (int c = 0; c < d; ++c) {
+                float res = bf16_to_float(v[(size_t)perm[b * bk + r] * d + c]) - vmu[(size_t)b * d + c];
+                if (fabsf(res) > amax[c]) amax[c] = fabsf(res);
+            }
+    }
+    for (int c = 0; c < d; ++c) {
+        vsc[c] = amax[c] > 0.0f ? amax[c] / 2688.0f : 1.0f;
+        inv[c] = amax[c] > 0.0f ? 2688.0f / amax[c] : 0.0f;
+    }
+    for (int b = 0; b < T; ++b) {
+        int valid = (n - b * bk) < bk ? (n - b * bk) : bk;
+        for (int r = 0; r < bk; ++r)
+            for (int c = 0; c < d; ++c) {
+                float res = r < valid ? bf16_to_float(v[(size_t)perm[b * bk + r] * d + c]) - vmu[(size_t)b * d + c]
+                                      : 0.0f;
+                y[(size_t)r * d + c] = res * inv[c];
+            }
+        for (int g = 0; g < G; ++g)
+            for (int c = 0; c < d; ++c) {
+                for (int i = 0; i < 16; ++i) x[i] = y[(size_t)(16 * g + i) * d + c];
+                vo_nvfp4_block(x, 16, codes, &vgs[((size_t)b * G + g) * d + c]);
+                for (int i = 0; i < 16; ++i) vq[((size_t)b * bk + 16 * g + i) * d + c] = codes[i];
+            }
+    }
+    free(amax);
+    free(inv);
+    free(y);
+}
+
 /* ------------------------------------------------------------------------ */
 /* The quantised attention forward, replayed row by row in tile order.       */
 /*                                                                            */
@@ -310,12 +438,15 @@ VO_API void vo_smooth_v(const uint16_t* v, int n, int d, int bk, const int32_t* 
 /* exact == 0: the method -- fp32 scores, fp32 A = (kappa*sq)*sk, ExpCast     */
 /*             bytes, p = E4M3 value of the byte.                             */
 /* exact == 1: fp64 scores and A, p = 2^((t - 56)/8) with t unrounded.        */
+/* pfmt == 1 (4-bit path, exact == 0): each 16-key block of a tile's P is     */
+/*             re-coded to NVFP4 (vo_nvfp4_block on the E4M3 values; keys past */
+/*             n count as 0) and p is the coded value.                         */
 /* Output: out [nrows*d] in fp64 (before the final bf16 rounding), and, when   */
 /* non-NULL, the final integer reference Mout and normaliser lout per row.    */
 /* ------------------------------------------------------------------------ */
 VO_API void vo_attn_emul(const double* qv, const float* sq, int nrows, const double* kv, const float* ksc,
                          const double* rv, const float* vmu, const float* vsc, int n, int d, int bk, double kappa,
-                         int beta, int exact, double* out, double* Mout, double* lout) {
+                         int beta, int exact, int pfmt, double* out, double* Mout, double* lout) {
     int T = (n + bk - 1) / bk;
     double* sc = (double*)malloc(sizeof(double) * (size_t)bk);
     double* p = (double*)malloc(sizeof(double) * (size_t)bk);
@@ -367,8 +498,18 @@ VO_API void vo_attn_emul(const double* qv, const float* sq, int nrows, const dou
                 } else {
                     p[j] = vo_e4m3_value(vo_expcast_byte((float)A, (float)sc[j], (float)cb));
                 }
-                lb += p[j];
             }
+            if (!exact && pfmt == 1) {
+                float x[16];
+                uint8_t codes[16], sc16;
+                for (int g = 0; g < bk / 16; ++g) {
+                    for (int i = 0; i < 16; ++i) x[i] = 16 * g + i < valid ? (float)p[16 * g + i] : 0.0f;
+                    vo_nvfp4_block(x, 16, codes, &sc16);
+                    for (int i = 0; i < 16 && 16 * g + i < valid; ++i)
+                        p[16 * g + i] = vo_e4m3_value(sc16) * vo_e2m1_value(codes[i]);
+                }
+            }
+            for (int j = 0; j < valid; ++j) lb += p[j];
             /* residual part through the quantised V, mean part as l_b * mu_b */
             for (int j = 0; j < valid; ++j) {
                 const double* rr = rv + ((size_t)b * bk + j) * d;

@@ -1,0 +1,177 @@
+"""Pins of the oracle's 4-bit (NVFP4) path.
+
+Independent references:
+- ml_dtypes' float4_e2m1fn, for the E2M1 codec;
+- brute force over the eight E2M1 magnitudes, for the block coder;
+- numpy recomputation of the residual and its scales, for the V residual;
+- a small online replay in Python on top of the pinned primitives, for the
+  P re-coding inside the attention replay.
+
+The 4-bit residual is the one the pages name as "per-channel E4M3/NVFP4
+residuals" (zerohour.day summary, key facts).
+"""
+import ml_dtypes
+import numpy as np
+import pytest
+
+import oracle
+from bit_fp8_attention_smooth_b200 import synth
+from conftest import bf16_values
+
+F4 = ml_dtypes.float4_e2m1fn
+MAGS = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def test_e2m1_decode_exhaustive_vs_ml_dtypes():
+    codes = np.arange(16, dtype=np.uint8)
+    ref = codes.view(F4).astype(np.float64)
+    np.testing.assert_array_equal(oracle.e2m1_value(codes), ref)
+
+
+def test_e2m1_encode_vs_ml_dtypes():
+    rng = np.random.default_rng(0)
+    mids = (MAGS[1:] + MAGS[:-1]) / 2  # every tie
+    x = np.concatenate([rng.standard_normal(20000) * 3, rng.uniform(-8, 8, 20000), mids, -mids, MAGS, -MAGS,
+                        [7.0, 100.0, -100.0, 1e-30, -1e-30, 0.0, -0.0]]).astype(np.float32)
+    ref = x.astype(F4).view(np.uint8)
+    np.testing.assert_array_equal(oracle.e2m1_encode(x), ref)
+
+
+def test_e2m1_ties_to_even_and_saturation():
+    x = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 1e9], np.float32)
+    # ties go to the code whose mantissa bit is 0
+    np.testing.assert_array_equal(oracle.e2m1_value(oracle.e2m1_encode(x)), [0, 1, 1, 2, 2, 4, 4, 6, 6])
+
+
+def _brute_block(x):
+    """NVFP4 block by brute force: scale E4M3(amax/6), then for each value the
+    E2M1 code nearest to x*(1/s), ties to the even code."""
+    x = np.asarray(x, np.float32)
+    amax = np.float32(np.abs(x).max())
+    s = oracle.e4m3_encode(np.float32(amax / np.float32(6.0)))[()]
+    sv = np.float32(oracle.e4m3_value(np.uint8(s)))
+    if sv == 0:
+        return np.zeros(x.shape, np.uint8), s
+    r = np.float32(np.float32(1.0) / sv)
+    y = (x * r).astype(np.float32).astype(np.float64)
+    codes = []
+    for v in y:
+        a = min(abs(v), 6.0)
+        dist = np.abs(MAGS - a)
+        best = np.flatnonzero(dist == dist.min())
+        c = best[0] if len(best) == 1 else best[best % 2 == 0][0]
+        codes.append(int(c) | (8 if np.signbit(v) else 0))
+    return np.array(codes, np.uint8), s
+
+
+def test_nvfp4_block_vs_brute_force():
+    rng = np.random.default_rng(1)
+    blocks = [rng.standard_normal(16) * 10 ** rng.uniform(-4, 2) for _ in range(300)]
+    blocks += [rng.uniform(0, 448, 16), np.full(16, 6.0), np.zeros(16), np.r_[np.zeros(15), 1e-6],
+               np.r_[448.0, np.zeros(15)], rng.standard_normal(7) * 3]
+    for b in blocks:
+        x = np.asarray(b, np.float32)
+        codes, scale = oracle.nvfp4_blocks(x[None])
+        ref_codes, ref_scale = _brute_block(x)
+        assert scale[0] == ref_scale
+        np.testing.assert_array_equal(codes[0], ref_codes)
+
+
+def test_nvfp4_block_worked_example():
+    # amax 6 -> scale E4M3(1.0) = 0x38, codes are plain E2M1 of x
+    x = np.array([6, -3, 1.5, 0.25, 0.75, -0.5, 4, 2.5, 0, 1, -6, 5, 3.5, -1.25, 0.1, 2], np.float32)
+    codes, scale = oracle.nvfp4_blocks(x[None])
+    assert scale[0] == 0x38
+    np.testing.assert_array_equal(codes[0], x.astype(F4).view(np.uint8))
+    # all-zero block: zero scale, zero codes
+    codes, scale = oracle.nvfp4_blocks(np.zeros((1, 16), np.float32))
+    assert scale[0] == 0 and not codes.any()
+
+
+@pytest.mark.parametrize("smooth", [True, False])
+def test_smooth_v_nvfp4_matches_its_definition(smooth):
+    w = synth.WORKLOADS["tiny_1k_d64"]
+    k, v = synth.head_bits(w, "k", 0, 0), synth.head_bits(w, "v", 0, 0)
+    n, d = v.shape
+    bk = 64
+    if smooth:
+        labels, _ = oracle.kmeans(v, w.C, w.iters)
+        perm = oracle.stable_perm(labels, w.C)
+    else:
+        perm = np.arange(n, dtype=np.int32)
+    vq, vgs, vmu, vsc = oracle.smooth_v_nvfp4(v, perm, bk, smooth)
+    vhat, vmu8, vsc8 = oracle.smooth_v(v, perm, bk, smooth)
+    np.testing.assert_array_equal(vmu, vmu8)  # same block means as the E4M3 residual
+    vals = bf16_values(v)[perm].astype(np.float32)
+    T = n // bk
+    res = (vals - np.repeat(vmu, bk, axis=0)).astype(np.float32)
+    amax = np.abs(res).max(axis=0)
+    np.testing.assert_array_equal(vsc, np.where(amax > 0, amax / np.float32(2688), 1).astype(np.float32))
+    inv = np.where(amax > 0, np.float32(2688) / amax, 0).astype(np.float32)
+    y = (res * inv).astype(np.float32)
+    # blocks of 16 tokens along the token axis, per channel
+    yb = y.reshape(T, bk // 16, 16, d).transpose(0, 1, 3, 2)
+    codes, scales = oracle.nvfp4_blocks(yb)
+    np.testing.assert_array_equal(vgs, scales)
+    np.testing.assert_array_equal(vq, codes.transpose(0, 1, 3, 2).reshape(n, d))
+    # coded values stay within half an E2M1 step (at most 1) times the block scale
+    deq = oracle.nvfp4_v_values(vq, vgs)
+    bound = np.repeat(oracle.e4m3_value(vgs), 16, axis=1).reshape(n, d) * 1.0 + 1e-30
+    assert np.all(np.abs(deq - y) <= bound * 1.0000001 + np.abs(y) * 0.07)
+
+
+def _replay_nvfp4_rows(qv, sq, kv, ksc, rv, vmu, vsc, n, bk, beta):
+    """Online replay in Python for a few rows, P re-coded per 16 keys."""
+    d = qv.shape[1]
+    T = -(-n // bk)
+    kap = np.float32(oracle.kappa(d))
+    outs = []
+    for i in range(qv.shape[0]):
+        M, l, first = 0.0, 0.0, True
+        ores = np.zeros(d)
+        omean = np.zeros(d)
+        for b in range(T):
+            valid = min(bk, n - b * bk)
+            A = np.float32(kap * np.float32(sq[i])) * np.float32(ksc[b])
+            s = (kv[b * bk:b * bk + valid] @ qv[i]).astype(np.float32)
+            Mc = np.ceil(float(np.float32(A * s.max())) / 8.0)
+            Mnew = Mc if first else max(M, Mc)
+            if not first and Mnew > M:
+                f = 2.0 ** -(Mnew - M)
+                ores *= f
+                omean *= f
+                l *= f
+            M, first = Mnew, False
+            cb = np.float32(56 + beta - 8 * M)
+            p8 = oracle.e4m3_value(oracle.expcast_bytes(np.full(valid, A, np.float32), s, np.full(valid, cb)))
+            x = np.zeros(bk, np.float32)
+            x[:valid] = p8
+            codes, sc = oracle.nvfp4_blocks(x.reshape(bk // 16, 16))
+            p = (oracle.e4m3_value(sc)[:, None] * oracle.e2m1_value(codes)).reshape(bk)[:valid]
+            ores += p @ rv[b * bk:b * bk + valid]
+            omean += p.sum() * vmu[b].astype(np.float64)
+            l += p.sum()
+        outs.append((vsc * ores + omean) / l)
+    return np.array(outs)
+
+
+def test_attn_replay_nvfp4_p_vs_python_replay():
+    w = synth.custom("nvfp4_pin", 1, 1, 200, 64, 5, pool=6, C=6, iters=3, block=64)
+    q, k, v = (synth.head_bits(w, t, 0, 0) for t in "qkv")
+    n, d = k.shape
+    prep = oracle.prep_head(k, v, C=w.C, iters=w.iters, bk=64, resid_fmt=1)
+    rows = np.arange(0, n, 23)
+    qhat, sq = oracle.quant_q(q[rows])
+    qv = oracle.e4m3_value(qhat)
+    kv = oracle.e4m3_value(prep["khat"])
+    rv = oracle.nvfp4_v_values(prep["vq"], prep["vgs"])
+    out, M, l = oracle.attn_emul(qv, sq, kv, prep["ksc"], rv, prep["vmu"], prep["vsc"], n=n, bk=64, beta=64,
+                                 pfmt=1)
+    ref = _replay_nvfp4_rows(qv, sq, kv, prep["ksc"], rv, prep["vmu"], prep["vsc"], n, 64, 64)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    # and the 4-bit path stays near the 8-bit one and near exact attention
+    r8 = oracle.forward_head(q, k, v, rows, C=w.C, iters=w.iters, bk=64, beta=64)["out"]
+    exact = oracle.attn_exact(q, k, v, rows)
+    ref_norm = np.linalg.norm(exact)
+    assert np.linalg.norm(out - exact) / ref_norm < 0.2
+    assert np.linalg.norm(out - r8) / ref_norm < 0.2
