@@ -40,10 +40,11 @@ class _Params(ctypes.Structure):
 
 
 class _Prep(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("perm", "labels", "k_fp8", "k_scale", "vt_fp8", "v_mean", "v_scale")]
+    _fields_ = [(n, ctypes.c_void_p)
+                for n in ("perm", "labels", "k_fp8", "k_scale", "vt_fp8", "v_mean", "v_scale", "v_bscale")]
 
 
-PREP_FIELDS = ("perm", "labels", "k_fp8", "k_scale", "vt_fp8", "v_mean", "v_scale")
+PREP_FIELDS = ("perm", "labels", "k_fp8", "k_scale", "vt_fp8", "v_mean", "v_scale", "v_bscale")
 
 _lib = None
 
@@ -129,7 +130,7 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def prep_sizes(shape, params: Params):
     sh = _Shape(*shape) if not isinstance(shape, _Shape) else shape
-    out = (ctypes.c_size_t * 7)()
+    out = (ctypes.c_size_t * 8)()
     _ok(lib().vc_prep_buffer_bytes(ctypes.byref(sh), ctypes.byref(params.c()), out), "vc_prep_buffer_bytes")
     return list(out)
 
@@ -147,19 +148,25 @@ def alloc_workspace(shape, params: Params, device="cuda") -> torch.Tensor:
 
 
 def alloc_prep(shape, params: Params, device="cuda") -> Dict[str, torch.Tensor]:
-    """Caller-owned prep buffers with their logical shapes and dtypes."""
+    """Caller-owned prep buffers with their logical shapes and dtypes (the
+    4-bit residual, resid_fmt 1: vt_fp8 holds two E2M1 codes a byte and
+    v_bscale the UE4M3 block scales)."""
     B, H, N, d = shape
     T = -(-N // params.block)
     Tp = T * params.block
-    return {
+    fp4 = params.resid_fmt == 1
+    prep = {
         "perm": torch.empty((B, H, N), dtype=torch.int32, device=device),
         "labels": torch.empty((B, H, N), dtype=torch.int32, device=device),
         "k_fp8": torch.empty((B, H, Tp, d), dtype=torch.uint8, device=device),
         "k_scale": torch.empty((B, H, T), dtype=torch.float32, device=device),
-        "vt_fp8": torch.empty((B, H, d, Tp), dtype=torch.uint8, device=device),
+        "vt_fp8": torch.empty((B, H, d, Tp // 2 if fp4 else Tp), dtype=torch.uint8, device=device),
         "v_mean": torch.empty((B, H, T, d), dtype=torch.float32, device=device),
         "v_scale": torch.empty((B, H, d), dtype=torch.float32, device=device),
     }
+    if fp4:
+        prep["v_bscale"] = torch.empty((B, H, T, d, params.block // 16), dtype=torch.uint8, device=device)
+    return prep
 
 
 def _prep_struct(prep: Dict[str, torch.Tensor]) -> _Prep:

@@ -65,7 +65,8 @@ vc_status check_shape_params(const vc_shape* s, const vc_params* p) {
         return VC_ERR_INVALID_ARG;
     if (s->d != 64 && s->d != 128) return VC_ERR_UNSUPPORTED;
     if (p->block != 64 && p->block != 128) return VC_ERR_UNSUPPORTED;
-    if (p->resid_fmt != 0) return VC_ERR_UNSUPPORTED;
+    if (p->resid_fmt != 0 && p->resid_fmt != 1) return VC_ERR_INVALID_ARG;
+    if (p->resid_fmt == 1 && p->block != 128) return VC_ERR_UNSUPPORTED;  // the 4-bit path: block 128
     if (p->smooth != 0 && p->smooth != 1) return VC_ERR_INVALID_ARG;
     if (p->beta < 0 || p->beta > 70) return VC_ERR_INVALID_ARG;
     if (p->wait_limit_ns < 0) return VC_ERR_INVALID_ARG;
@@ -76,8 +77,9 @@ vc_status check_shape_params(const vc_shape* s, const vc_params* p) {
     return VC_OK;
 }
 
-vc_status check_prep_ptrs(const vc_prep* pr, bool need_labels) {
+vc_status check_prep_ptrs(const vc_prep* pr, const vc_params* p, bool need_labels) {
     if (!pr) return VC_ERR_INVALID_ARG;
+    if (p->resid_fmt == 1 && !aligned16(pr->v_bscale)) return VC_ERR_INVALID_ARG;
     if (!aligned16(pr->perm) || !aligned16(pr->k_fp8) || !aligned16(pr->k_scale) || !aligned16(pr->vt_fp8) ||
         !aligned16(pr->v_mean) || !aligned16(pr->v_scale))
         return VC_ERR_INVALID_ARG;
@@ -127,12 +129,14 @@ vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc
     pl.iters = p.iters;
     pl.BK = p.block;
     pl.smooth = p.smooth;
+    pl.resid_fmt = p.resid_fmt;
     pl.perm = out.perm;
     pl.k_fp8 = out.k_fp8;
     pl.k_scale = out.k_scale;
     pl.vt_fp8 = out.vt_fp8;
     pl.v_mean = out.v_mean;
     pl.v_scale = out.v_scale;
+    pl.v_bscale = out.v_bscale;
     pl.labels = out.labels ? out.labels : reinterpret_cast<int32_t*>(ws + L.labels);
     pl.c_hi = reinterpret_cast<__nv_bfloat16*>(ws + L.c_hi);
     pl.c_lo = reinterpret_cast<__nv_bfloat16*>(ws + L.c_lo);
@@ -163,8 +167,11 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
     if (vc::launch_quant_q(static_cast<const __nv_bfloat16*>(Q), qfp8, sq, (int64_t)BH * N, D, stream) != cudaSuccess)
         return VC_ERR_CUDA;
     CUtensorMap tk, tv;
+    // V^T tiles: BK codes a channel row, bytes (E4M3) or two codes a byte (E2M1)
+    const uint64_t vrow = p.resid_fmt == 1 ? Tp / 2 : Tp;
+    const uint32_t vbox = p.resid_fmt == 1 ? BK / 2 : BK;
     if (!vc::make_tmap_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.k_fp8, D, Tp, BH, D, BK) ||
-        !vc::make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.vt_fp8, Tp, D, BH, BK, D))
+        !vc::make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pr.vt_fp8, vrow, D, BH, vbox, D))
         return VC_ERR_CUDA;
     vc::AttnArgs a{};
     a.q_fp8 = qfp8;
@@ -172,6 +179,7 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
     a.k_scale = pr.k_scale;
     a.v_mean = pr.v_mean;
     a.v_scale = pr.v_scale;
+    a.v_bscale = pr.v_bscale;
     a.out = static_cast<__nv_bfloat16*>(O);
     a.N = N;
     a.T = T;
@@ -179,7 +187,9 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
     a.beta = p.beta;
     a.ctl.status = reinterpret_cast<int*>(ws + L.status);
     a.ctl.limit_ns = p.wait_limit_ns > 0 ? p.wait_limit_ns : kDefaultWaitNs;
-    return vc::launch_attn(D, BK, tk, tv, a, BH, stream) == cudaSuccess ? VC_OK : VC_ERR_CUDA;
+    const cudaError_t e = p.resid_fmt == 1 ? vc::launch_attn4(D, tk, tv, a, BH, stream)
+                                           : vc::launch_attn(D, BK, tk, tv, a, BH, stream);
+    return e == cudaSuccess ? VC_OK : VC_ERR_CUDA;
 }
 
 }  // namespace
@@ -251,9 +261,11 @@ vc_status vc_prep_buffer_bytes(const vc_shape* shape, const vc_params* params, s
     bytes[1] = 4 * BH * N;   // labels
     bytes[2] = BH * Tp * D;  // k_fp8
     bytes[3] = 4 * BH * T;   // k_scale
-    bytes[4] = BH * D * Tp;  // vt_fp8
+    const bool fp4 = params->resid_fmt == 1;
+    bytes[4] = fp4 ? BH * D * Tp / 2 : BH * D * Tp;  // vt_fp8 (E2M1: two codes a byte)
     bytes[5] = 4 * BH * T * D;  // v_mean
     bytes[6] = 4 * BH * D;   // v_scale
+    bytes[7] = fp4 ? BH * T * D * (params->block / 16) : 0;  // v_bscale
     return VC_OK;
 }
 
@@ -270,7 +282,7 @@ vc_status vc_smooth_prepare(const void* K, const void* V, const vc_shape* shape,
     vc_status st = check_shape_params(shape, params);
     if (st != VC_OK) return st;
     if (!aligned16(K) || !aligned16(V) || !aligned16(workspace)) return VC_ERR_INVALID_ARG;
-    if ((st = check_prep_ptrs(out, false)) != VC_OK) return st;
+    if ((st = check_prep_ptrs(out, params, false)) != VC_OK) return st;
     const WsLayout L = ws_layout(*shape, *params);
     if (workspace_bytes < L.total) return VC_ERR_WORKSPACE;
     if ((st = check_device()) != VC_OK) return st;
@@ -283,7 +295,7 @@ vc_status vc_attn_fwd(const void* Q, const vc_prep* prep, const vc_shape* shape,
     vc_status st = check_shape_params(shape, params);
     if (st != VC_OK) return st;
     if (!aligned16(Q) || !aligned16(O) || !aligned16(workspace)) return VC_ERR_INVALID_ARG;
-    if ((st = check_prep_ptrs(prep, false)) != VC_OK) return st;
+    if ((st = check_prep_ptrs(prep, params, false)) != VC_OK) return st;
     const WsLayout L = ws_layout(*shape, *params);
     if (workspace_bytes < L.total) return VC_ERR_WORKSPACE;
     if ((st = check_device()) != VC_OK) return st;
@@ -297,7 +309,7 @@ vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_sha
     if (st != VC_OK) return st;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
         return VC_ERR_INVALID_ARG;
-    if ((st = check_prep_ptrs(scratch, false)) != VC_OK) return st;
+    if ((st = check_prep_ptrs(scratch, params, false)) != VC_OK) return st;
     const WsLayout L = ws_layout(*shape, *params);
     if (workspace_bytes < L.total) return VC_ERR_WORKSPACE;
     if ((st = check_device()) != VC_OK) return st;
@@ -316,7 +328,7 @@ vc_status vc_attention_host(const void* Qh, const void* Kh, const void* Vh, void
     if (!Qh || !Kh || !Vh || !Oh) return VC_ERR_INVALID_ARG;
     if (!aligned16(Qd) || !aligned16(Kd) || !aligned16(Vd) || !aligned16(Od) || !aligned16(workspace))
         return VC_ERR_INVALID_ARG;
-    if ((st = check_prep_ptrs(scratch, false)) != VC_OK) return st;
+    if ((st = check_prep_ptrs(scratch, params, false)) != VC_OK) return st;
     const WsLayout L = ws_layout(*shape, *params);
     if (workspace_bytes < L.total) return VC_ERR_WORKSPACE;
     if ((st = check_device()) != VC_OK) return st;
@@ -358,9 +370,10 @@ vc_status vc_attention_host(const void* Qh, const void* Kh, const void* Vh, void
         gp.labels = scratch->labels ? scratch->labels + (size_t)h0 * N : nullptr;
         gp.k_fp8 = scratch->k_fp8 + (size_t)h0 * T * BK * D;
         gp.k_scale = scratch->k_scale + (size_t)h0 * T;
-        gp.vt_fp8 = scratch->vt_fp8 + (size_t)h0 * D * T * BK;
+        gp.vt_fp8 = scratch->vt_fp8 + (size_t)h0 * D * T * BK / (params->resid_fmt == 1 ? 2 : 1);
         gp.v_mean = scratch->v_mean + (size_t)h0 * T * D;
         gp.v_scale = scratch->v_scale + (size_t)h0 * D;
+        gp.v_bscale = params->resid_fmt == 1 ? scratch->v_bscale + (size_t)h0 * T * D * (BK / 16) : nullptr;
         cudaEvent_t in_done = nullptr, out_ready = nullptr;
         if (cudaEventCreateWithFlags(&in_done, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&out_ready, cudaEventDisableTiming) != cudaSuccess) {
@@ -391,7 +404,7 @@ vc_status vc_attn_fwd_noalloc(const void* Q, const vc_prep* prep, const vc_shape
     vc_status st = check_shape_params(shape, params);
     if (st != VC_OK) return st;
     if (!aligned16(Q) || !aligned16(O)) return VC_ERR_INVALID_ARG;
-    if ((st = check_prep_ptrs(prep, false)) != VC_OK) return st;
+    if ((st = check_prep_ptrs(prep, params, false)) != VC_OK) return st;
     const WsLayout L = ws_layout(*shape, *params);  // the attention region only: status, Q fp8, Q scales
     if (L.attn_end > VC_NOALLOC_SCRATCH_BYTES) return VC_ERR_WORKSPACE;
     if ((st = check_device()) != VC_OK) return st;

@@ -290,6 +290,31 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n) {
            | (uint32_t(128 >> 4) << 24);      // M / 16
 }
 
+// Instruction descriptor of kind::mxf4nvf4 with block16 scaling: D fp32, A and
+// B E2M1 (two codes a byte), both K-major, UE4M3 scale factors, M = 128,
+// N = n, K = 64 an instruction; the scale-factor byte offsets (sf ids) are 0.
+__host__ __device__ constexpr uint32_t idesc_nvf4_f32(int n) {
+    return (1u << 7) | (1u << 10)           // A, B format: E2M1
+           | (uint32_t(n >> 3) << 17)       // N / 8
+           | (0u << 23)                     // scale format: UE4M3
+           | (uint32_t(128 >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= (sfa . A[smem]) (sfb . B[smem])^T, kind::mxf4nvf4, one elected
+// lane of the warp.  Scale factors live in tensor memory: for row r of A (B)
+// and 16-element block j of this instruction's K = 64, the byte j of column
+// sf + r/32, in lane r%32 of every 32-lane quadrant.
+__device__ __forceinline__ void mma_nvf4_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred pe, pa;\n\t"
+        "elect.sync _|pe, 0xffffffff;\n\t"
+        "setp.ne.b32 pa, %4, 0;\n\t"
+        "@pe tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], pa;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored as rows of
 // `row_bytes` (64 or 128) with the matching swizzle, 8-row groups packed
 // (stride 8 * row_bytes).  The tile base must be 1024-byte aligned.
@@ -311,6 +336,28 @@ __device__ __forceinline__ uint32_t swz_offset(int row, int chunk, int row_bytes
 // ---------------------------------------------------------------- E4M3
 // Two fp32 values -> two E4M3 bytes (round to nearest even, saturate to
 // +-448); lo ends up in the low byte.
+// A non-negative E4M3 byte -> its fp32 value, exactly: a 20-bit shift puts
+// the byte's exponent and mantissa fields on fp32's (a subnormal byte on a
+// subnormal float), and the bias difference (127 - 7) is a factor 2^120.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    return __fmul_rn(__uint_as_float(code << 20), 0x1p120f);
+}
+
+// Eight fp32 values -> E2M1 codes (nearest, ties to even, saturating at 6),
+// four bits each, x[0] in the lowest nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const float* x) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
+    return out;
+}
+
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));

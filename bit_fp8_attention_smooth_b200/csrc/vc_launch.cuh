@@ -12,6 +12,7 @@ struct AttnArgs {
     const float* k_scale;  // [BH, T]
     const float* v_mean;   // [BH, T, D]
     const float* v_scale;  // [BH, D]
+    const uint8_t* v_bscale;  // 4-bit path: [BH, T, D, BK/16] UE4M3 block scales of the V residual
     __nv_bfloat16* out;    // [BH, N, D]
     int N, T;
     float kappa;  // fp32(8 * log2(e) / sqrt(D))
@@ -37,13 +38,15 @@ struct PrepLaunch {
     const __nv_bfloat16* K;
     const __nv_bfloat16* V;
     int BH, N, D, C, iters, BK, smooth;
+    int resid_fmt;  // 0: E4M3 residual; 1: 4-bit (NVFP4) residual
     // outputs
     int32_t* perm;
     uint8_t* k_fp8;
     float* k_scale;
-    uint8_t* vt_fp8;
+    uint8_t* vt_fp8;    // E4M3 residual, or E2M1 codes two a byte
     float* v_mean;
     float* v_scale;
+    uint8_t* v_bscale;  // 4-bit path: [BH, T, D, BK/16] UE4M3 block scales
     // workspace
     int32_t* labels;
     __nv_bfloat16* c_hi;  // [BH, Cp, D] centroid high bf16 part
@@ -51,9 +54,9 @@ struct PrepLaunch {
     float* cnorm;         // [BH, Cp] squared centroid norms
     double* cent64;       // [BH, C, D] fp64 centroids (the exact near-tie decision)
     double* sums;         // [BH, C, D] fp64 member sums of the Lloyd update
-    float* vnorm2;
+    float* vnorm2;        // [BH, N] |v|^2 of every token (bounds the tensor-core distance error)
     KmTie* ties;          // [BH * N] near-tie list of the current pass
-    int* tie_count;       // [2] list lengths, by pass parity        // [BH, N] |v|^2 of every token (bounds the tensor-core distance error)
+    int* tie_count;       // [2] list lengths, by pass parity
     int32_t* cstart;
     int32_t* ccount;
     int32_t* hist;
@@ -70,6 +73,9 @@ bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dtype, int elem_bytes, con
 
 cudaError_t launch_attn(int D, int BK, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int BH,
                         cudaStream_t stream);
+// The 4-bit path (block 128): NVFP4 P and V residual in the PV product.
+cudaError_t launch_attn4(int D, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int BH,
+                         cudaStream_t stream);
 cudaError_t launch_prep(const PrepLaunch& p, cudaStream_t s);
 cudaError_t launch_quant_q(const __nv_bfloat16* Q, uint8_t* q_fp8, float* sq, int64_t tokens, int D,
                            cudaStream_t s);

@@ -20,6 +20,7 @@
 //   prep_kv_block             per block: K amax scale + E4M3 K, V block mean (fp64 sum),
 //                             residual channel amax
 //   prep_v_quant              per-channel residual scale, E4M3 residual, transposed
+//   prep_v_quant_nvfp4        the same with the 4-bit (NVFP4) residual and its block scales
 //   quant_q                   per-token E4M3 Q (used by the attention call)
 #include <math.h>
 
@@ -814,6 +815,89 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_v_quant(const __nv_bfloat16
     }
 }
 
+// The 4-bit residual: the same block means and residual channel maxima as the
+// E4M3 path, then per channel one fp32 scale s_c = amax_c/(6*448) and, for
+// every 16 consecutive tokens of a channel inside the block, an NVFP4 block:
+// y = r * (6*448/amax_c), UE4M3 scale E4M3(amax_16/6), codes E2M1(y * (1/s))
+// (a zero scale codes zeros).  Codes leave transposed and packed two a byte
+// (token 2i in the low nibble): vt[bh][c][token/2]; the block scales leave as
+// v_bscale[bh][b][c][BK/16], the bytes one PV tile needs, contiguous.
+template <int D, int BK>
+__global__ void __launch_bounds__(PREP_THREADS) prep_v_quant_nvfp4(const __nv_bfloat16* __restrict__ V,
+                                                                   const int32_t* __restrict__ perm,
+                                                                   const float* __restrict__ v_mean,
+                                                                   const uint32_t* __restrict__ vamax,
+                                                                   uint8_t* __restrict__ vt_fp4,
+                                                                   uint8_t* __restrict__ v_bscale,
+                                                                   float* __restrict__ v_scale, int N, int T,
+                                                                   const int* __restrict__ status) {
+    constexpr int NT = PREP_THREADS;
+    constexpr int RG = NT / D;
+    constexpr int CH = D / 8;
+    constexpr int G = BK / 16;       // NVFP4 blocks per channel and tile
+    constexpr int WSTR = BK / 8 + 1; // words per channel row of codes (+1: conflict-free)
+    extern __shared__ uint4 v_s[];   // [BK][CH]
+    __shared__ int tok_s[BK];
+    __shared__ uint32_t cw[D * WSTR];
+    __shared__ __align__(16) uint8_t sc_s[D * G];  // read back as words
+    if (ctl_failed(status)) return;  // perm is undefined
+    const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const int valid = min(BK, N - b * BK);
+    const int64_t Tp = (int64_t)T * BK;
+    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    __syncthreads();
+    const uint4* vg = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D);
+#pragma unroll
+    for (int u = 0; u < BK * CH / NT; ++u) {
+        const int i = tid + u * NT;
+        const int r = i / CH;
+        if (r < valid) v_s[i] = __ldg(vg + (size_t)tok_s[r] * CH + i % CH);
+    }
+    const int c = tid % D, rg = tid / D;
+    const float amax = __uint_as_float(vamax[(size_t)bh * D + c]);
+    const float inv = amax > 0.0f ? __fdiv_rn(2688.0f, amax) : 0.0f;
+    if (b == 0 && rg == 0) v_scale[(size_t)bh * D + c] = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    const float mu = v_mean[((size_t)bh * T + b) * D + c];
+    __syncthreads();
+    const __nv_bfloat16* vsh = reinterpret_cast<const __nv_bfloat16*>(v_s);
+    for (int g = rg; g < G; g += RG) {
+        float y[16];
+        float ga = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int r = 16 * g + e;
+            y[e] = r < valid ? __fmul_rn(__fsub_rn(bf2f(vsh[r * D + c]), mu), inv) : 0.0f;
+            ga = fmaxf(ga, fabsf(y[e]));
+        }
+        const uint8_t sc = (uint8_t)(e4m3x2(__fdiv_rn(ga, 6.0f), 0.0f) & 0xFF);
+        const float sv = e4m3_to_f32(sc);
+        uint32_t w0 = 0, w1 = 0;
+        if (sv > 0.0f) {
+            const float rs = __frcp_rn(sv);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(y[e], rs);
+            w0 = e2m1x8(y);
+            w1 = e2m1x8(y + 8);
+        }
+        cw[c * WSTR + 2 * g] = w0;
+        cw[c * WSTR + 2 * g + 1] = w1;
+        sc_s[c * G + g] = sc;
+    }
+    __syncthreads();
+    // codes: BK/2 bytes a channel row, as 16-byte pieces
+    constexpr int PIECES = BK / 32;
+    for (int i = tid; i < D * PIECES; i += NT) {
+        const int cc = i / PIECES, pc = i % PIECES;
+        const uint32_t* src = cw + cc * WSTR + 4 * pc;
+        *reinterpret_cast<uint4*>(vt_fp4 + ((size_t)bh * D + cc) * (Tp / 2) + (size_t)b * (BK / 2) + 16 * pc) =
+            make_uint4(src[0], src[1], src[2], src[3]);
+    }
+    // block scales: D * G bytes, contiguous for the tile
+    for (int i = tid; i < D * G / 4; i += NT)
+        reinterpret_cast<uint32_t*>(v_bscale + ((size_t)bh * T + b) * D * G)[i] =
+            reinterpret_cast<const uint32_t*>(sc_s)[i];
+}
+
 // Per-token Q: amax over d, inv = 448/amax, code = E4M3(q * inv), sq = amax/448.
 template <int D>
 __global__ void __launch_bounds__(256) quant_q(const __nv_bfloat16* __restrict__ Q, uint8_t* __restrict__ q_fp8,
@@ -933,12 +1017,22 @@ static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
         e = cudaFuncSetAttribute(prep_v_quant<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  v_quant_smem<D, BK>());
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(prep_v_quant_nvfp4<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 v_quant_smem<D, BK>());
+        if (e != cudaSuccess) return e;
         configured = true;
     }
     prep_kv_block<D, BK><<<dim3(T, p.BH), PREP_THREADS, kv_block_smem<D, BK>(), s>>>(
         p.K, p.V, p.perm, p.smooth, p.k_fp8, p.k_scale, p.v_mean, p.vamax, p.N, T, p.ctl.status);
-    prep_v_quant<D, BK><<<dim3(T, p.BH), PREP_THREADS, v_quant_smem<D, BK>(), s>>>(
-        p.V, p.perm, p.smooth, p.v_mean, p.vamax, p.vt_fp8, p.v_scale, p.N, T, p.ctl.status);
+    if (p.resid_fmt == 1) {
+        if constexpr (BK % 32 == 0) {
+            prep_v_quant_nvfp4<D, BK><<<dim3(T, p.BH), PREP_THREADS, v_quant_smem<D, BK>(), s>>>(
+                p.V, p.perm, p.v_mean, p.vamax, p.vt_fp8, p.v_bscale, p.v_scale, p.N, T, p.ctl.status);
+        }
+    } else {
+        prep_v_quant<D, BK><<<dim3(T, p.BH), PREP_THREADS, v_quant_smem<D, BK>(), s>>>(
+            p.V, p.perm, p.smooth, p.v_mean, p.vamax, p.vt_fp8, p.v_scale, p.N, T, p.ctl.status);
+    }
     return cudaGetLastError();
 }
 

@@ -48,12 +48,12 @@
 extern "C" {
 #endif
 
-#define VC_ABI_VERSION 1
+#define VC_ABI_VERSION 2
 
 typedef enum {
     VC_OK = 0,
     VC_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad size or parameter */
-    VC_ERR_UNSUPPORTED = 2,    /* d or block outside {64,128}, NVFP4 residual, not sm_100 */
+    VC_ERR_UNSUPPORTED = 2,    /* d or block outside {64,128}, 4-bit residual with block != 128, not sm_100 */
     VC_ERR_CUDA = 3,           /* a CUDA runtime or driver call failed */
     VC_ERR_DEVICE_TIMEOUT = 4, /* a device-side wait ran out (see wait_limit_ns) */
     VC_ERR_WORKSPACE = 5       /* workspace smaller than vc_workspace_bytes() */
@@ -70,7 +70,7 @@ typedef struct {
     int32_t block;         /* hardware block = KV tile: 64 or 128 tokens */
     int32_t beta;          /* ExpCast shift: byte = round(8z + 56 + beta); integer in [0, 70] */
     int32_t smooth;        /* 1 = V-Smooth; 0 = plain per-channel FP8 V (identity order, zero means) */
-    int32_t resid_fmt;     /* 0 = E4M3 residual (the only format built) */
+    int32_t resid_fmt;     /* 0 = E4M3 residual; 1 = 4-bit NVFP4 residual (block 128 only) */
     int64_t wait_limit_ns; /* bound on any single device-side wait; 0 = 2 s */
 } vc_params;
 
@@ -82,10 +82,18 @@ typedef struct {
  *   k_fp8    uint8 [B,H,Tp,d]     E4M3 K rows in regrouped order; rows >= N are 0
  *   k_scale  fp32  [B,H,T]        per-block K scale: K ~= k_scale[b] * E4M3(k_fp8)
  *   vt_fp8   uint8 [B,H,d,Tp]     E4M3 V residual, channel-major (transposed);
- *                                 columns >= N are 0
+ *                                 columns >= N are 0.  With resid_fmt 1:
+ *                                 [B,H,d,Tp/2], E2M1 codes two a byte (token
+ *                                 2i in the low nibble)
  *   v_mean   fp32  [B,H,T,d]      block means of V (kept in fp32)
  *   v_scale  fp32  [B,H,d]        per-channel residual scale:
  *                                 V[perm[i]] ~= v_mean[i / block] + v_scale * E4M3(vt_fp8[:, i])
+ *   v_bscale uint8 [B,H,T,d,block/16]  resid_fmt 1 only (NULL otherwise): the
+ *                                 UE4M3 scale of each 16-token run of a channel:
+ *                                 V[perm[i]][c] ~= v_mean[i / block][c] + v_scale[c] *
+ *                                   E4M3(v_bscale[i / block][c][(i % block) / 16]) * E2M1(code)
+ *   (4-bit residual: the zerohour.day summary's "per-channel E4M3/NVFP4
+ *   residuals"; E2M1 and UE4M3 as in the OCP MX formats.)
  */
 typedef struct {
     int32_t* perm;
@@ -95,6 +103,7 @@ typedef struct {
     uint8_t* vt_fp8;
     float* v_mean;
     float* v_scale;
+    uint8_t* v_bscale;
 } vc_prep;
 
 /* ABI version of the loaded library (VC_ABI_VERSION). */
@@ -103,8 +112,9 @@ int vc_abi_version(void);
 /* Static, human-readable name of a vc_status value. */
 const char* vc_status_string(int status);
 
-/* Byte sizes of the seven vc_prep buffers, in struct order, for this shape and
- * block size.  bytes must point to 7 size_t.  Host only; no CUDA call. */
+/* Byte sizes of the eight vc_prep buffers, in struct order, for this shape and
+ * params (v_bscale is 0 bytes unless resid_fmt is 1).  bytes must point to 8
+ * size_t.  Host only; no CUDA call. */
 vc_status vc_prep_buffer_bytes(const vc_shape* shape, const vc_params* params, size_t* bytes);
 
 /* Workspace size needed by vc_smooth_prepare, vc_attn_fwd and vc_attention
@@ -123,7 +133,10 @@ vc_status vc_workspace_bytes(const vc_shape* shape, const vc_params* params, siz
  * c_k = V[floor(k N / C)], `iters` assignment passes, squared Euclidean
  * distance, ties to the lowest cluster, empty clusters keep their centroid);
  * stable regroup by cluster id; per block: K amax scale and E4M3 K, V mean,
- * V residual; per channel: residual amax scale and E4M3 residual.
+ * V residual; per channel: residual amax scale and E4M3 residual.  With
+ * resid_fmt 1 the residual is 4-bit: per channel s_c = amax_c / (6 * 448), and
+ * each 16-token run of a channel an NVFP4 block (UE4M3 scale E4M3(amax/6),
+ * E2M1 codes of y * (1/scale) with y = r / s_c).
  */
 vc_status vc_smooth_prepare(const void* K, const void* V, const vc_shape* shape, const vc_params* params,
                             const vc_prep* out, void* workspace, size_t workspace_bytes, void* stream);
@@ -139,7 +152,10 @@ vc_status vc_smooth_prepare(const void* K, const void* V, const vc_shape* shape,
  * per tile an integer row reference M (raised online); each score maps to the
  * E4M3 probability byte max(0, round(A*s + 56 + beta - 8M)) with one FMA;
  * FP8 PV; row sums of the tile restore the block means; O = (v_scale * O_res +
- * sum_b l_b mu_b) / l.  Non-causal; keys >= N are masked.
+ * sum_b l_b mu_b) / l.  Non-causal; keys >= N are masked.  With resid_fmt 1
+ * the PV product is 4-bit (tcgen05 kind::mxf4nvf4): each 16-key run of a row's
+ * P is re-coded from the ExpCast byte's E4M3 value to NVFP4 (UE4M3 scale
+ * E4M3(max/6), E2M1 codes of p * (1/scale)), against the 4-bit residual.
  */
 vc_status vc_attn_fwd(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params, void* O,
                       void* workspace, size_t workspace_bytes, void* stream);

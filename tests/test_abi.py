@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(libpath):
 
 def test_library_loads_and_answers_host_queries(libpath):
     L = ctypes.CDLL(libpath)
-    assert L.vc_abi_version() == 1
+    assert L.vc_abi_version() == 2
     L.vc_status_string.restype = ctypes.c_char_p
     assert L.vc_status_string(0) == b"ok"
     import bit_fp8_attention_smooth_b200 as vc
@@ -51,7 +51,17 @@ def test_library_loads_and_answers_host_queries(libpath):
     shape = (1, 40, 32768, 128)
     params = vc.Params(C=64, iters=10, block=128)
     sizes = vc.prep_sizes(shape, params)
-    assert sizes[2] == 40 * 32768 * 128 and sizes[4] == 40 * 128 * 32768
+    assert sizes[2] == 40 * 32768 * 128 and sizes[4] == 40 * 128 * 32768 and sizes[7] == 0
+    # the 4-bit residual: two codes a byte, one UE4M3 scale per 16 tokens of a channel
+    p4 = vc.Params(C=64, iters=10, block=128, resid_fmt=1)
+    s4 = vc.prep_sizes(shape, p4)
+    assert s4[4] == 40 * 128 * 32768 // 2 and s4[7] == 40 * 256 * 128 * 8
+    with pytest.raises(vc.VcError) as e:  # block 64 has no 4-bit path
+        vc.prep_sizes(shape, vc.Params(C=64, iters=10, block=64, resid_fmt=1))
+    assert e.value.status == vc.VC_ERR_UNSUPPORTED
+    with pytest.raises(vc.VcError) as e:
+        vc.prep_sizes(shape, vc.Params(C=64, iters=10, block=128, resid_fmt=2))
+    assert e.value.status == vc.VC_ERR_INVALID_ARG
     assert vc.workspace_bytes(shape, params) >= 40 * 32768 * 128
     with pytest.raises(vc.VcError) as e:
         vc.workspace_bytes((1, 1, 100, 96), params)
