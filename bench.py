@@ -164,9 +164,11 @@ def oracle_sample(w, rows: int, threads: int):
     q, k, v = (synth.head_bits(w, t, 0, 0) for t in "qkv")
     sel = np.linspace(0, w.N - 1, rows).astype(np.int64)
     t0 = time.perf_counter()
-    prep = oracle.prep_head(k, v, C=w.C, iters=w.iters, bk=w.block)
+    rf = resid_fmt_of(w)
+    prep = oracle.prep_head(k, v, C=w.C, iters=w.iters, bk=w.block, resid_fmt=rf)
     t1 = time.perf_counter()
-    oracle.forward_head(q, k, v, sel, C=w.C, iters=w.iters, bk=w.block, beta=BETA, prep=prep, threads=threads)
+    oracle.forward_head(q, k, v, sel, C=w.C, iters=w.iters, bk=w.block, beta=BETA, resid_fmt=rf, prep=prep,
+                        threads=threads)
     t2 = time.perf_counter()
     head_s = (t1 - t0) + (t2 - t1) * (w.N / rows)
     head_flops = 4.0 * float(w.N) ** 2 * w.d
@@ -208,9 +210,15 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def resid_fmt_of(w) -> int:
+    """1 for the 4-bit (NVFP4) residual workload, else 0 (E4M3)."""
+    return 1 if w.resid_fmt == "nvfp4" else 0
+
+
 def config_of(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "C": w.C, "kmeans_iters": w.iters,
             "block": w.block, "beta": BETA, "v_smooth": True,
+            "residual": "nvfp4 (E2M1 + UE4M3 per 16)" if resid_fmt_of(w) else "e4m3",
             "l2": f"inputs {3 * w.B * w.H * w.N * w.d * 2 / 1e9:.2f} GB per step > 126 MB L2 (no flush needed)"}
 
 
@@ -309,17 +317,28 @@ def run_ours(args, w):
     if rank == 0:
         peaks = load_peaks()
         fp8_peak = peaks["bf16_sustained"] * FP8_PER_BF16
+        four_bit = resid_fmt_of(w) == 1
+        if four_bit:
+            # QK^T (half the flops) at the FP8 rate, PV (the other half) at the
+            # FP4 rate, twice FP8: the time at peak is 3/4 of the all-FP8 time
+            peak, kernel = fp8_peak * 4.0 / 3.0, "vc_attn_fwd (Q quantise + vc_attn4_kernel)"
+            peak_src = (f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16) for QK^T, "
+                        f"x 4 (fp4:bf16) for PV; harmonic over the two halves")
+        else:
+            peak, kernel = fp8_peak, "vc_attn_fwd (Q quantise + vc_attn_kernel)"
+            peak_src = f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16)"
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic", "config": config_of(w),
+            "vs_baseline": None, "dtype": "e4m3+e2m1" if four_bit else "e4m3", "data": "synthetic",
+            "config": config_of(w),
             "attn_ms": attn_ms, "prep_ms": prep_ms, "attn_tflops": attn_tflops,
             "frac_of_nominal_fp8_4500": value / 4500.0, "attn_frac_of_nominal_fp8_4500": attn_tflops / 4500.0,
             "roofline": {
-                "bound": "tensor", "kernel": "vc_attn_fwd (Q quantise + vc_attn_kernel)",
-                "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
-                "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16)",
-                "traffic": attn_traffic_bytes(w.B * w.H),
+                "bound": "tensor", "kernel": kernel,
+                "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                "peak_source": peak_src,
+                "traffic": None if four_bit else attn_traffic_bytes(w.B * w.H),
                 "traffic_unit": "bytes per launch (ncu capture on 8 heads, scaled by heads)",
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,

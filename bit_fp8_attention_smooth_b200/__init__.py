@@ -108,6 +108,9 @@ class Params:
 
     @classmethod
     def for_workload(cls, w, **kw) -> "Params":
+        """The workload's k-means, block and residual format (the 4-bit
+        residual for a workload that names nvfp4), overridable by keyword."""
+        kw.setdefault("resid_fmt", 1 if getattr(w, "resid_fmt", "e4m3") == "nvfp4" else 0)
         return cls(C=w.C, iters=w.iters, block=w.block, **kw)
 
 

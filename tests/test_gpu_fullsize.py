@@ -31,12 +31,17 @@ def _sample_rows(N):
     return rows
 
 
-def _check_workload(vc, w, smooth=True):
+def _unpack_codes(vt):
+    codes = np.stack([vt & 0xF, vt >> 4], axis=-1).reshape(vt.shape[0], -1)
+    return np.ascontiguousarray(codes.T)
+
+
+def _check_workload(vc, w, smooth=True, resid_fmt=0):
     shape = (w.B, w.H, w.N, w.d)
     q = synth.tensor_bf16(w, "q").cuda()
     k = synth.tensor_bf16(w, "k").cuda()
     v = synth.tensor_bf16(w, "v").cuda()
-    params = vc.Params.for_workload(w, beta=BETA, smooth=smooth)
+    params = vc.Params.for_workload(w, beta=BETA, smooth=smooth, resid_fmt=resid_fmt)
     ws = vc.alloc_workspace(shape, params)
     prep = vc.smooth_prepare(k, v, params, workspace=ws)
     out = vc.attn_fwd(q, prep, params, workspace=ws)
@@ -46,13 +51,17 @@ def _check_workload(vc, w, smooth=True):
     gout = {h: out[0, h, rows].float().cpu().numpy() for h in heads}
     gprep = {h: gpu_prep_head({kk: t[:, h:h + 1].cpu() for kk, t in prep.items()}, 0, 0, w.N, w.block)
              for h in heads}
+    if resid_fmt == 1:  # the 4-bit residual: unpacked codes and block scales
+        for h in heads:
+            gprep[h]["vq"] = _unpack_codes(gprep[h].pop("vhat").T)  # back to [d, Tp/2] bytes
+            gprep[h]["vgs"] = prep["v_bscale"][0, h].cpu().numpy().transpose(0, 2, 1)
     del q, k, v, out, prep, ws
     torch.cuda.empty_cache()
 
     def run(h):
         qb, kb, vb = (synth.head_bits(w, t, 0, h) for t in "qkv")
         r = oracle.forward_head(qb, kb, vb, rows, C=w.C, iters=w.iters, bk=w.block, beta=BETA, smooth=smooth,
-                                threads=8)
+                                resid_fmt=resid_fmt, threads=8)
         r["exact"] = oracle.attn_exact(qb, kb, vb, rows, threads=8)
         return r
 
@@ -64,11 +73,11 @@ def _check_workload(vc, w, smooth=True):
         agree = (got["labels"] == ref["prep"]["labels"]).mean()
         assert agree >= 0.999, (h, agree)
         if np.array_equal(got["perm"], ref["prep"]["perm"]):
-            for key in ("khat", "ksc", "vmu", "vsc", "vhat"):
+            for key in ("khat", "ksc", "vmu", "vsc") + (("vq", "vgs") if resid_fmt == 1 else ("vhat",)):
                 assert np.array_equal(got[key], ref["prep"][key]), (h, key)
         rel, cos, _ = metrics(gout[h], ref["out"])
         rel_x, _, psnr_x = metrics(gout[h], ref["exact"])
-        print(f"{w.name} smooth={smooth} head {h}: labels agree {agree:.5f}, "
+        print(f"{w.name} smooth={smooth} resid_fmt={resid_fmt} head {h}: labels agree {agree:.5f}, "
               f"vs emulation rel={rel:.2e} cos={cos:.6f}; vs exact rel={rel_x:.3e} psnr={psnr_x:.1f} dB")
         assert rel <= REL_L2_TOL and cos >= COS_TOL, (h, rel, cos)
 
@@ -82,8 +91,13 @@ def test_grid720p_ragged(vc, smooth):
     _check_workload(vc, synth.WORKLOADS["grid720p_75600_d128"], smooth)
 
 
+def test_nvfp4_32k(vc):
+    """The 4-bit workload as specified: NVFP4 residual, mxf4nvf4 PV."""
+    _check_workload(vc, synth.WORKLOADS["nvfp4_32k_d128"], resid_fmt=1)
+
+
 def test_nvfp4_shape_with_e4m3_residual(vc):
-    _check_workload(vc, synth.WORKLOADS["nvfp4_32k_d128"])
+    _check_workload(vc, synth.WORKLOADS["nvfp4_32k_d128"], resid_fmt=0)
 
 
 def test_longclip(vc):
