@@ -60,7 +60,8 @@ struct Attn4Cfg {
     static constexpr int OFF_MU = OFF_SFB + STAGES * SFB_BYTES;
     static constexpr int OFF_SFA = OFF_MU + STAGES * MU_BYTES;  // [parity][2][BM] words
     static constexpr int OFF_KINC = OFF_SFA + 2 * 2 * BM * 4;
-    static constexpr int OFF_BAR = OFF_KINC + 4 * BM * 4;
+    static constexpr int OFF_PLUT = OFF_KINC + 4 * BM * 4;  // 128 P block-scale entries
+    static constexpr int OFF_BAR = OFF_PLUT + 128 * 8;
     static constexpr int B_QREADY = 0;
     static constexpr int B_KFULL = 1;
     static constexpr int B_KEMPTY = B_KFULL + STAGES;
@@ -126,35 +127,65 @@ __device__ __forceinline__ bool softmax_sync_and(bool v) {
     return r != 0;
 }
 
-// One 16-key NVFP4 block of P from the ExpCast codes n[0..15] (E4M3 bytes of
-// the probabilities, each >= 0): the UE4M3 scale E4M3(max/6) and the E2M1 codes
-// of p * (1/scale) (p the E4M3 value; the product rounded once in fp32, as
-// (p 2^-60)(r 2^60) with both factors exact).  A zero scale codes zeros.
-__device__ __forceinline__ void p_block_nvfp4(const uint32_t* n, uint32_t& w0, uint32_t& w1, uint32_t& scale) {
-    uint32_t m = n[0];
-#pragma unroll
-    for (int e = 1; e < 16; ++e) m = max(m, n[e]);
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// The NVFP4 block scale of P depends only on the block's largest ExpCast code
+// m (E4M3 codes increase with their values): its UE4M3 code E4M3(value(m)/6)
+// and the reciprocal of its value, rounded to fp32, times 2^60 (0 for a zero
+// scale).  One entry per code, built once per CTA with the same divide and
+// reciprocal the block coder would use.
+struct PScaleEntry {
+    uint32_t sc;
+    float r60;
+};
+
+__device__ __forceinline__ PScaleEntry p_scale_entry(uint32_t m) {
     const uint32_t sc = (uint32_t)(e4m3x2(__fdiv_rn(e4m3_to_f32(m), 6.0f), 0.0f) & 0xFF);
     const float sv = e4m3_to_f32(sc);
-    const float r60 = sv > 0.0f ? __fmul_rn(__frcp_rn(sv), 0x1p60f) : 0.0f;
+    return PScaleEntry{sc, sv > 0.0f ? __fmul_rn(__frcp_rn(sv), 0x1p60f) : 0.0f};
+}
+
+// One 16-key NVFP4 block of P from the ExpCast codes, given as the floats
+// w[e] = code * 2^-149 (whose bit patterns are the codes, ordered as the
+// codes): the UE4M3 scale E4M3(max/6) and the E2M1 codes of p * (1/scale),
+// p the E4M3 value, the product rounded once in fp32 as (p 2^-60)(r 2^60),
+// both factors exact.  A zero scale codes zeros.
+__device__ __forceinline__ void p_block_nvfp4(const float* w, const PScaleEntry* lut, uint32_t& w0, uint32_t& w1,
+                                              uint32_t& scale) {
+    const float m5[5] = {fmax3(w[0], w[1], w[2]), fmax3(w[3], w[4], w[5]), fmax3(w[6], w[7], w[8]),
+                         fmax3(w[9], w[10], w[11]), fmax3(w[12], w[13], w[14])};
+    const float mx = fmaxf(fmax3(m5[0], m5[1], m5[2]), fmax3(m5[3], m5[4], w[15]));
+    const PScaleEntry ent = lut[__float_as_uint(mx) & 127u];
+    const float2 k60 = make_float2(0x1p60f, 0x1p60f), r = make_float2(ent.r60, ent.r60);
     float x[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) x[e] = __fmul_rn(__fmul_rn(__uint_as_float(n[e] << 20), 0x1p60f), r60);
+    for (int e = 0; e < 16; e += 2) {
+        const float2 p = make_float2(__uint_as_float(__float_as_uint(w[e]) << 20),
+                                     __uint_as_float(__float_as_uint(w[e + 1]) << 20));
+        const float2 y = fmul2(fmul2(p, k60), r);
+        x[e] = y.x;
+        x[e + 1] = y.y;
+    }
     w0 = e2m1x8(x);
     w1 = e2m1x8(x + 8);
-    scale = sc;
+    scale = ent.sc;
 }
 
 // ExpCast codes of two scores, clamped at 0: t = A*s + cbm rounds A*s + cb to
 // the integer n once (cbm = cb + 1.5*2^23), and sat(t*2^-149 - 1.5*2^-126) is
 // max(n, 0)*2^-149 exactly, whose bit pattern is max(n, 0).
-__device__ __forceinline__ void expcast_codes2(float A, float s0, float s1, float cbm, uint32_t& n0, uint32_t& n1) {
+__device__ __forceinline__ void expcast_codes2(float A, float s0, float s1, float cbm, float& w0, float& w1) {
     const float2 t = ffma2(make_float2(A, A), make_float2(s0, s1), make_float2(cbm, cbm));
-    float w0, w1;
     asm("fma.rn.sat.f32 %0, %1, 0f00000001, 0f80C00000;" : "=f"(w0) : "f"(t.x));
     asm("fma.rn.sat.f32 %0, %1, 0f00000001, 0f80C00000;" : "=f"(w1) : "f"(t.y));
-    n0 = __float_as_uint(w0);
-    n1 = __float_as_uint(w1);
 }
 
 template <int D>
@@ -321,9 +352,12 @@ __global__ void __launch_bounds__(320, 1)
         const float aq = __fmul_rn(args.kappa, sqv);
         const float c0 = 56.0f + (float)args.beta;
         uint32_t* sfa_x = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_SFA);  // [parity][MMA][row]
+        PScaleEntry* plut = reinterpret_cast<PScaleEntry*>(smem + Cfg::OFF_PLUT);
+        plut[row] = p_scale_entry((uint32_t)row);  // the 128 softmax threads, one code each
+        bool run = softmax_sync_and(true);
         float M = 0.0f;
         float sk_next = args.k_scale[(size_t)bh * T];
-        for (int t = 0; t < T; ++t) {
+        for (int t = 0; run && t < T; ++t) {
             const int sb = t & 1;
             const float sk = sk_next;
             if (t + 1 < T) sk_next = args.k_scale[(size_t)bh * T + t + 1];
@@ -370,12 +404,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int g = 2 * ch + h;
-                        uint32_t n[16];
+                        float wc[16];
 #pragma unroll
                         for (int e = 0; e < 16; e += 2)
-                            expcast_codes2(A, s[16 * g + e], s[16 * g + e + 1], cbm, n[e], n[e + 1]);
+                            expcast_codes2(A, s[16 * g + e], s[16 * g + e + 1], cbm, wc[e], wc[e + 1]);
                         uint32_t sc;
-                        p_block_nvfp4(n, pw[2 * h], pw[2 * h + 1], sc);
+                        p_block_nvfp4(wc, plut, pw[2 * h], pw[2 * h + 1], sc);
                         sfw[g / 4] |= sc << (8 * (g % 4));
                     }
                     *reinterpret_cast<uint4*>(ptile + swz_offset(row, ch, Cfg::VROW)) =
