@@ -99,7 +99,7 @@ class Params:
     iters: int = 10
     block: int = 128
     beta: int = 64
-    smooth: bool = True
+    smooth: int = 1  # 1 V-Smooth, 0 plain FP8 V, 2 V-Smooth reusing the prep's regroup
     resid_fmt: int = 0
     wait_limit_ns: int = 0
 
@@ -112,6 +112,39 @@ class Params:
         residual for a workload that names nvfp4), overridable by keyword."""
         kw.setdefault("resid_fmt", 1 if getattr(w, "resid_fmt", "e4m3") == "nvfp4" else 0)
         return cls(C=w.C, iters=w.iters, block=w.block, **kw)
+
+
+@dataclasses.dataclass(frozen=True)
+class VSmoothSchedule:
+    """Which prep each step of a denoising loop runs.
+
+    The pages run V-Smooth only in the first quarter of the denoising steps on
+    B200 and call its cost a scheduling trade-off (chooseai.io news 7051,
+    意义与局限).  Step i (0-based) of `total_steps` runs V-Smooth when
+    i < on_fraction * total_steps, and plain per-channel FP8 V after that.
+    Within the V-Smooth steps, k-means runs on every `recluster_every`-th step
+    (always on step 0); the steps in between reuse the latest regroup
+    (Params.smooth = 2), which leaves only the block quantisation to run.
+    """
+
+    total_steps: int
+    on_fraction: float = 0.25
+    recluster_every: int = 1
+
+    def __post_init__(self):
+        if self.total_steps < 1 or not 0.0 <= self.on_fraction <= 1.0 or self.recluster_every < 1:
+            raise ValueError(f"bad schedule {self}")
+
+    def mode(self, step: int) -> int:
+        """Params.smooth for this step: 1 cluster, 2 reuse the regroup, 0 off."""
+        if not 0 <= step < self.total_steps:
+            raise ValueError(f"step {step} outside 0..{self.total_steps - 1}")
+        if step >= self.on_fraction * self.total_steps:
+            return 0
+        return 1 if step % self.recluster_every == 0 else 2
+
+    def params(self, base: Params, step: int) -> Params:
+        return dataclasses.replace(base, smooth=self.mode(step))
 
 
 def _shape(t: torch.Tensor) -> _Shape:

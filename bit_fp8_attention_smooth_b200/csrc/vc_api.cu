@@ -67,10 +67,10 @@ vc_status check_shape_params(const vc_shape* s, const vc_params* p) {
     if (p->block != 64 && p->block != 128) return VC_ERR_UNSUPPORTED;
     if (p->resid_fmt != 0 && p->resid_fmt != 1) return VC_ERR_INVALID_ARG;
     if (p->resid_fmt == 1 && p->block != 128) return VC_ERR_UNSUPPORTED;  // the 4-bit path: block 128
-    if (p->smooth != 0 && p->smooth != 1) return VC_ERR_INVALID_ARG;
+    if (p->smooth < 0 || p->smooth > 2) return VC_ERR_INVALID_ARG;
     if (p->beta < 0 || p->beta > 70) return VC_ERR_INVALID_ARG;
     if (p->wait_limit_ns < 0) return VC_ERR_INVALID_ARG;
-    if (p->smooth) {
+    if (p->smooth == 1) {
         if (p->C < 1 || p->C > 256 || p->C > s->N) return VC_ERR_INVALID_ARG;
         if (p->iters < 1 || p->iters > 64) return VC_ERR_INVALID_ARG;
     }
@@ -125,7 +125,7 @@ vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc
     pl.BH = s.B * s.H;
     pl.N = s.N;
     pl.D = s.d;
-    pl.C = p.smooth ? p.C : 1;
+    pl.C = p.smooth == 1 ? p.C : 1;
     pl.iters = p.iters;
     pl.BK = p.block;
     pl.smooth = p.smooth;

@@ -651,6 +651,10 @@ __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __r
 // vamax with an integer max on the fp32 bits (all >= 0).
 constexpr int PREP_THREADS = 256;
 
+// A regrouped position's token, forced into [0, N): a permutation passed in by
+// the caller (the reuse mode) can then never index outside the head.
+__device__ __forceinline__ int clamp_tok(int32_t t, int N) { return (uint32_t)t < (uint32_t)N ? t : 0; }
+
 template <int D, int BK>
 constexpr int kv_block_smem() {
     return 2 * BK * D * 2;
@@ -674,7 +678,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat1
     if (ctl_failed(status)) return;  // perm is undefined
     const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int valid = min(BK, N - b * BK);
-    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? clamp_tok(perm[(size_t)bh * N + b * BK + r], N) : 0;
     __syncthreads();
     uint4* ks = kv_s;
     uint4* vs = kv_s + BK * CH;
@@ -779,7 +783,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_v_quant(const __nv_bfloat16
     const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int valid = min(BK, N - b * BK);
     const int Tp = T * BK;
-    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? clamp_tok(perm[(size_t)bh * N + b * BK + r], N) : 0;
     __syncthreads();
     const uint4* vg = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D);
 #pragma unroll
@@ -844,7 +848,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_v_quant_nvfp4(const __nv_bf
     const int b = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int valid = min(BK, N - b * BK);
     const int64_t Tp = (int64_t)T * BK;
-    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? perm[(size_t)bh * N + b * BK + r] : 0;
+    for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? clamp_tok(perm[(size_t)bh * N + b * BK + r], N) : 0;
     __syncthreads();
     const uint4* vg = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D);
 #pragma unroll
@@ -1002,10 +1006,12 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
 template <int D, int BK>
 static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
     const int T = (p.N + BK - 1) / BK;
-    if (!p.smooth) {  // plain per-channel FP8 V: identity order, zeroed channel maxima
-        const int64_t total = (int64_t)p.BH * p.N;
-        identity_order<<<(unsigned)imin64((total + 255) / 256, 148 * 32), 256, 0, s>>>(p.perm, p.labels,
-                                                                                             total, p.N);
+    if (p.smooth != 1) {  // no k-means this call: the channel maxima start from zero here
+        if (p.smooth == 0) {  // plain per-channel FP8 V: identity order
+            const int64_t total = (int64_t)p.BH * p.N;
+            identity_order<<<(unsigned)imin64((total + 255) / 256, 148 * 32), 256, 0, s>>>(p.perm, p.labels,
+                                                                                                 total, p.N);
+        }  // smooth == 2: the regroup already in perm is kept
         cudaError_t e = cudaMemsetAsync(p.vamax, 0, sizeof(uint32_t) * (size_t)p.BH * D, s);
         if (e != cudaSuccess) return e;
     }
@@ -1038,7 +1044,7 @@ static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
 
 cudaError_t launch_prep(const PrepLaunch& p, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
-    if (p.smooth) {
+    if (p.smooth == 1) {
         e = p.D == 128 ? kmeans_t<128>(p, s) : kmeans_t<64>(p, s);
         if (e != cudaSuccess) return e;
     }

@@ -69,7 +69,9 @@ typedef struct {
     int32_t iters;         /* k-means assignment passes, 1 <= iters <= 64 */
     int32_t block;         /* hardware block = KV tile: 64 or 128 tokens */
     int32_t beta;          /* ExpCast shift: byte = round(8z + 56 + beta); integer in [0, 70] */
-    int32_t smooth;        /* 1 = V-Smooth; 0 = plain per-channel FP8 V (identity order, zero means) */
+    int32_t smooth;        /* 1 = V-Smooth; 0 = plain per-channel FP8 V (identity order, zero means);
+                              2 = V-Smooth reusing the regroup already in the prep's perm (from an
+                              earlier call on the same shape): no k-means, K/V quantised in that order */
     int32_t resid_fmt;     /* 0 = E4M3 residual; 1 = 4-bit NVFP4 residual (block 128 only) */
     int64_t wait_limit_ns; /* bound on any single device-side wait; 0 = 2 s */
 } vc_params;
@@ -133,7 +135,12 @@ vc_status vc_workspace_bytes(const vc_shape* shape, const vc_params* params, siz
  * c_k = V[floor(k N / C)], `iters` assignment passes, squared Euclidean
  * distance, ties to the lowest cluster, empty clusters keep their centroid);
  * stable regroup by cluster id; per block: K amax scale and E4M3 K, V mean,
- * V residual; per channel: residual amax scale and E4M3 residual.  With
+ * V residual; per channel: residual amax scale and E4M3 residual.  smooth 2
+ * skips the k-means and the regroup and keeps out->perm (and out->labels) as
+ * they are: a later denoising step reuses an earlier step's clustering (the
+ * pages run V-Smooth only in the first quarter of the steps on B200 and call
+ * its cost a scheduling trade-off: chooseai.io news 7051, 意义与局限).  perm
+ * entries outside [0, N) are read as token 0.  With
  * resid_fmt 1 the residual is 4-bit: per channel s_c = amax_c / (6 * 448), and
  * each 16-token run of a channel an NVFP4 block (UE4M3 scale E4M3(amax/6),
  * E2M1 codes of y * (1/scale) with y = r / s_c).
