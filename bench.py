@@ -245,6 +245,12 @@ def run_ours(args, w):
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
     vc.lib()
+    full = w
+    if args.split_heads:  # strong scaling: this rank takes its share of the heads
+        if world > w.H:
+            raise SystemExit(f"--split-heads needs at most {w.H} ranks")
+        h0, h1 = vc.head_range(rank, world, w.H)
+        w = dataclasses.replace(w, H=h1 - h0)
     params = vc.Params.for_workload(w, beta=BETA)
     shape = (w.B, w.H, w.N, w.d)
 
@@ -289,8 +295,9 @@ def run_ours(args, w):
     attn_ms = max_over_ranks(attn_ms, dev)
     prep_ms = max_over_ranks(prep_ms, dev)
     ms_per_step = total_ms / args.steps
-    flops = w.attn_flops
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    flops = w.attn_flops  # this rank's
+    job_flops = full.attn_flops if args.split_heads else world * flops
+    value = job_flops / (ms_per_step * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
 
     # the prep of a later denoising step that keeps this step's regroup
@@ -342,9 +349,10 @@ def run_ours(args, w):
             peak_src = f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16)"
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if args.split_heads else "weak",
             "vs_baseline": None, "dtype": "e4m3+e2m1" if four_bit else "e4m3", "data": "synthetic",
-            "config": config_of(w),
+            "config": dict(config_of(full), **({"heads_per_rank": w.H} if args.split_heads else {})),
             "attn_ms": attn_ms, "prep_ms": prep_ms, "prep_reuse_ms": prep_reuse_ms, "attn_tflops": attn_tflops,
             "frac_of_nominal_fp8_4500": value / 4500.0, "attn_frac_of_nominal_fp8_4500": attn_tflops / 4500.0,
             "roofline": {
@@ -354,7 +362,7 @@ def run_ours(args, w):
                 "traffic": None if four_bit else attn_traffic_bytes(w.B * w.H),
                 "traffic_unit": "bytes per launch (ncu capture on 8 heads, scaled by heads)",
             },
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+            "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": e2e.h2d_bytes, "d2h_bytes_per_step": e2e.d2h_bytes},
             "gpu_launches": launches_per_step(params) * args.steps,
             "clocks": clocks.summary(),
@@ -383,6 +391,9 @@ def main():
     ap.add_argument("--workload", default="mid_32k_d128", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split-heads", action="store_true",
+                    help="strong scaling: the ranks split the workload's heads (default: weak scaling, every rank "
+                         "runs the whole workload)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads of the workload (profiling captures on a smaller case)")
     args = ap.parse_args()

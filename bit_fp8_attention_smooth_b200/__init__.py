@@ -147,6 +147,40 @@ class VSmoothSchedule:
         return dataclasses.replace(base, smooth=self.mode(step))
 
 
+def head_range(rank: int, world: int, H: int):
+    """Heads [h0, h1) of rank `rank` when H heads are split over `world`
+    ranks: contiguous, sizes differing by at most one.  Every (b, h) problem of
+    the path is independent, k-means included, so a head split needs no
+    exchange on the data path."""
+    if world < 1 or not 0 <= rank < world or H < 0:
+        raise ValueError(f"bad split: rank {rank} of {world}, {H} heads")
+    return H * rank // world, H * (rank + 1) // world
+
+
+def gather_heads(o_local: torch.Tensor, H: int, group=None) -> torch.Tensor:
+    """All-gather per-rank output heads [B, h1 - h0, N, d] (this rank's
+    head_range) into the full [B, H, N, d] on every rank, over
+    torch.distributed (NCCL for CUDA tensors).  Only for callers that need
+    every head on every rank: the attention itself needs no collective."""
+    import torch.distributed as dist
+
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    B, h_loc, N, d = o_local.shape
+    h0, h1 = head_range(rank, world, H)
+    if h1 - h0 != h_loc:
+        raise ValueError(f"rank {rank} holds {h_loc} heads, its range is {h1 - h0}")
+    width = -(-H // world)  # uneven splits travel padded to the widest rank
+    send = torch.zeros((B, width, N, d), dtype=o_local.dtype, device=o_local.device)
+    send[:, :h_loc] = o_local
+    parts = [torch.empty_like(send) for _ in range(world)]
+    dist.all_gather(parts, send, group=group)
+    out = torch.empty((B, H, N, d), dtype=o_local.dtype, device=o_local.device)
+    for r, part in enumerate(parts):
+        a, b = head_range(r, world, H)
+        out[:, a:b] = part[:, :b - a]
+    return out
+
+
 def _shape(t: torch.Tensor) -> _Shape:
     if t.dim() != 4:
         raise ValueError("expected a [B, H, N, d] tensor")
