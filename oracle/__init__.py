@@ -60,7 +60,7 @@ def lib():
             "vo_e2m1_encode_array": (None, [P, i64, P]),
             "vo_nvfp4_block_array": (None, [P, i64, i32, P, P]),
             "vo_smooth_v_nvfp4": (None, [P, i32, i32, i32, P, i32, P, P, P, P]),
-            "vo_attn_emul": (None, [P, P, i32, P, P, P, P, P, i32, i32, i32, f64, i32, i32, i32, P, P, P]),
+            "vo_attn_emul": (None, [P, P, i32, P, P, P, P, P, i32, i32, i32, f64, i32, i32, i32, P, P, P, P]),
             "vo_attn_exact": (None, [P, P, P, P, i32, i32, i32, P]),
         }
         for name, (res, args) in sig.items():
@@ -229,9 +229,11 @@ def _chunks(nrows: int, parts: int):
 
 
 def attn_emul(qv, sq, kv, ksc, rv, vmu, vsc, *, n: int, bk: int, beta: int, exact: bool = False,
-              pfmt: int = 0, kappa_value: float | None = None, threads: int | None = None):
+              pfmt: int = 0, rowmask=None, kappa_value: float | None = None, threads: int | None = None):
     """Replay of the attention forward over the given query rows (values);
-    pfmt 1 re-codes each 16-key block of P to NVFP4 (the 4-bit path)."""
+    pfmt 1 re-codes each 16-key block of P to NVFP4 (the 4-bit path);
+    rowmask [nrows, T] (0 = drop the key tile for that row) is a block-sparse
+    mask."""
     qv, sq = _c(qv, np.float64), _c(sq, np.float32)
     kv, ksc, rv = _c(kv, np.float64), _c(ksc, np.float32), _c(rv, np.float64)
     vmu, vsc = _c(vmu, np.float32), _c(vsc, np.float32)
@@ -242,13 +244,18 @@ def attn_emul(qv, sq, kv, ksc, rv, vmu, vsc, *, n: int, bk: int, beta: int, exac
     out = np.empty((nrows, d), np.float64)
     M = np.empty(nrows, np.float64)
     l = np.empty(nrows, np.float64)
+    T = -(-n // bk)
+    if rowmask is not None:
+        rowmask = _c(rowmask, np.uint8)
+        assert rowmask.shape == (nrows, T)
     L = lib()
 
     def run(a, b):
         if b <= a:
             return
+        rm = None if rowmask is None else _p(rowmask[a:b])
         L.vo_attn_emul(_p(qv[a:b]), _p(sq[a:b]), b - a, _p(kv), _p(ksc), _p(rv), _p(vmu), _p(vsc), n, d, bk,
-                       kap, int(beta), int(exact), int(pfmt), _p(out[a:b]), _p(M[a:b]), _p(l[a:b]))
+                       kap, int(beta), int(exact), int(pfmt), rm, _p(out[a:b]), _p(M[a:b]), _p(l[a:b]))
 
     threads = threads or os.cpu_count() or 1
     with ThreadPoolExecutor(threads) as ex:
@@ -274,7 +281,8 @@ def attn_exact(q_bits, k_bits, v_bits, rows, threads: int | None = None) -> np.n
 
 
 def forward_head(q_bits, k_bits, v_bits, rows, *, C: int, iters: int, bk: int, beta: int,
-                 smooth: bool = True, resid_fmt: int = 0, prep=None, threads: int | None = None):
+                 smooth: bool = True, resid_fmt: int = 0, prep=None, tile_mask=None, bm: int = 128,
+                 threads: int | None = None):
     """V-Smooth prep plus the quantised attention replay for selected rows of
     one head (resid_fmt 1: 4-bit residual and NVFP4 P in the PV product)."""
     n, d = k_bits.shape
@@ -283,8 +291,10 @@ def forward_head(q_bits, k_bits, v_bits, rows, *, C: int, iters: int, bk: int, b
     rows = np.asarray(rows, dtype=np.int64)
     qhat, sq = quant_q(np.asarray(q_bits)[rows])
     rv = nvfp4_v_values(prep["vq"], prep["vgs"]) if resid_fmt == 1 else e4m3_value(prep["vhat"])
+    # a block-sparse mask [Tq, T] over (query tile of bm rows, key tile), per row
+    rowmask = None if tile_mask is None else np.asarray(tile_mask, np.uint8)[rows // bm]
     out, M, l = attn_emul(e4m3_value(qhat), sq, e4m3_value(prep["khat"]), prep["ksc"], rv, prep["vmu"],
-                          prep["vsc"], n=n, bk=bk, beta=beta, pfmt=resid_fmt, threads=threads)
+                          prep["vsc"], n=n, bk=bk, beta=beta, pfmt=resid_fmt, rowmask=rowmask, threads=threads)
     return dict(prep=prep, qhat=qhat, sq=sq, out=out, M=M, l=l)
 
 

@@ -438,6 +438,9 @@ VO_API void vo_smooth_v_nvfp4(const uint16_t* v, int n, int d, int bk, const int
 /* exact == 0: the method -- fp32 scores, fp32 A = (kappa*sq)*sk, ExpCast     */
 /*             bytes, p = E4M3 value of the byte.                             */
 /* exact == 1: fp64 scores and A, p = 2^((t - 56)/8) with t unrounded.        */
+/* rowmask (may be NULL): [nrows][T]; 0 drops key tile b for row i, as a     */
+/*             block-sparse mask would (the tile takes no part in the row's    */
+/*             max, weights or sums); a row with no tile left outputs 0.       */
 /* pfmt == 1 (4-bit path, exact == 0): each 16-key block of a tile's P is     */
 /*             re-coded to NVFP4 (vo_nvfp4_block on the E4M3 values; keys past */
 /*             n count as 0) and p is the coded value.                         */
@@ -446,7 +449,8 @@ VO_API void vo_smooth_v_nvfp4(const uint16_t* v, int n, int d, int bk, const int
 /* ------------------------------------------------------------------------ */
 VO_API void vo_attn_emul(const double* qv, const float* sq, int nrows, const double* kv, const float* ksc,
                          const double* rv, const float* vmu, const float* vsc, int n, int d, int bk, double kappa,
-                         int beta, int exact, int pfmt, double* out, double* Mout, double* lout) {
+                         int beta, int exact, int pfmt, const uint8_t* rowmask, double* out, double* Mout,
+                         double* lout) {
     int T = (n + bk - 1) / bk;
     double* sc = (double*)malloc(sizeof(double) * (size_t)bk);
     double* p = (double*)malloc(sizeof(double) * (size_t)bk);
@@ -460,6 +464,7 @@ VO_API void vo_attn_emul(const double* qv, const float* sq, int nrows, const dou
         for (int c = 0; c < d; ++c) ores[c] = omean[c] = 0.0;
         float aq32 = kappa32 * sq[i];
         for (int b = 0; b < T; ++b) {
+            if (rowmask && !rowmask[(size_t)i * T + b]) continue;
             int valid = (n - b * bk) < bk ? (n - b * bk) : bk;
             double A;
             if (exact)
@@ -518,7 +523,7 @@ VO_API void vo_attn_emul(const double* qv, const float* sq, int nrows, const dou
             for (int c = 0; c < d; ++c) omean[c] += lb * (double)vmu[(size_t)b * d + c];
             l += lb;
         }
-        for (int c = 0; c < d; ++c) out[(size_t)i * d + c] = ((double)vsc[c] * ores[c] + omean[c]) / l;
+        for (int c = 0; c < d; ++c) out[(size_t)i * d + c] = first ? 0.0 : ((double)vsc[c] * ores[c] + omean[c]) / l;
         if (Mout) Mout[i] = M;
         if (lout) lout[i] = l;
     }
