@@ -261,6 +261,13 @@ def run_ours(args, w):
     prep = vc.alloc_prep(shape, params, dev)
     ws = vc.alloc_workspace(shape, params, dev)
     stream = torch.cuda.current_stream(dev)
+    # block-sparse: each query tile keeps a seeded random share of the key tiles
+    tile_mask, density = None, 1.0
+    if args.tile_density < 1.0:
+        g = torch.Generator().manual_seed(7)
+        tm = torch.rand((w.B, w.H, -(-w.N // 128), -(-w.N // w.block)), generator=g) < args.tile_density
+        tile_mask = tm.to(torch.uint8).to(dev)
+        density = float(tm.float().mean())
 
     def step(evs=None):
         if evs is not None:
@@ -268,7 +275,7 @@ def run_ours(args, w):
         vc.smooth_prepare(kd, vd, params, prep=prep, workspace=ws)
         if evs is not None:
             evs[1].record(stream)
-        vc.attn_fwd(qd, prep, params, out=out, workspace=ws)
+        vc.attn_fwd(qd, prep, params, out=out, workspace=ws, tile_mask=tile_mask)
         if evs is not None:
             evs[2].record(stream)
 
@@ -295,8 +302,10 @@ def run_ours(args, w):
     attn_ms = max_over_ranks(attn_ms, dev)
     prep_ms = max_over_ranks(prep_ms, dev)
     ms_per_step = total_ms / args.steps
-    flops = w.attn_flops  # this rank's
-    job_flops = full.attn_flops if args.split_heads else world * flops
+    flops = w.attn_flops * density  # this rank's (the kept key tiles only)
+    job_flops = full.attn_flops * density if args.split_heads else world * flops
+    # the host-buffer leg runs the dense call (vc_attention_host takes no mask)
+    dense_job_flops = full.attn_flops if args.split_heads else world * w.attn_flops
     value = job_flops / (ms_per_step * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
 
@@ -352,17 +361,18 @@ def run_ours(args, w):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if args.split_heads else "weak",
             "vs_baseline": None, "dtype": "e4m3+e2m1" if four_bit else "e4m3", "data": "synthetic",
-            "config": dict(config_of(full), **({"heads_per_rank": w.H} if args.split_heads else {})),
+            "config": dict(config_of(full), **({"heads_per_rank": w.H} if args.split_heads else {}),
+                           **({"tile_density": density} if tile_mask is not None else {})),
             "attn_ms": attn_ms, "prep_ms": prep_ms, "prep_reuse_ms": prep_reuse_ms, "attn_tflops": attn_tflops,
             "frac_of_nominal_fp8_4500": value / 4500.0, "attn_frac_of_nominal_fp8_4500": attn_tflops / 4500.0,
             "roofline": {
                 "bound": "tensor", "kernel": kernel,
                 "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
                 "peak_source": peak_src,
-                "traffic": None if four_bit else attn_traffic_bytes(w.B * w.H),
+                "traffic": None if four_bit or tile_mask is not None else attn_traffic_bytes(w.B * w.H),
                 "traffic_unit": "bytes per launch (ncu capture on 8 heads, scaled by heads)",
             },
-            "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+            "e2e": {"value": dense_job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": e2e.h2d_bytes, "d2h_bytes_per_step": e2e.d2h_bytes},
             "gpu_launches": launches_per_step(params) * args.steps,
             "clocks": clocks.summary(),
@@ -391,6 +401,9 @@ def main():
     ap.add_argument("--workload", default="mid_32k_d128", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tile-density", type=float, default=1.0,
+                    help="block-sparse attention: the share of key tiles each query tile keeps (seeded random mask; "
+                         "flops count the kept tiles only)")
     ap.add_argument("--split-heads", action="store_true",
                     help="strong scaling: the ranks split the workload's heads (default: weak scaling, every rank "
                          "runs the whole workload)")

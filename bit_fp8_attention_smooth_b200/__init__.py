@@ -65,6 +65,7 @@ def lib():
             "vc_workspace_bytes": (ctypes.c_int, [PS, PP, ctypes.POINTER(S)]),
             "vc_smooth_prepare": (ctypes.c_int, [P, P, PS, PP, PR, P, S, P]),
             "vc_attn_fwd": (ctypes.c_int, [P, PR, PS, PP, P, P, S, P]),
+            "vc_attn_fwd_masked": (ctypes.c_int, [P, PR, PS, PP, P, P, P, S, P]),
             "vc_attention": (ctypes.c_int, [P, P, P, PS, PP, PR, P, P, S, P]),
             "vc_attention_host": (ctypes.c_int, [P, P, P, P, PS, PP, ctypes.c_int, P, P, P, P, PR, P, S, P, P, P]),
             "vc_check": (ctypes.c_int, [P, P]),
@@ -260,15 +261,29 @@ def smooth_prepare(K: torch.Tensor, V: torch.Tensor, params: Params, prep=None, 
     return prep
 
 
-def attn_fwd(Q: torch.Tensor, prep, params: Params, out=None, workspace=None, stream=None) -> torch.Tensor:
-    """ExpCast-FP8 attention over prepped K/V; returns O (bf16, Q's layout)."""
+def attn_fwd(Q: torch.Tensor, prep, params: Params, out=None, workspace=None, stream=None,
+             tile_mask: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """ExpCast-FP8 attention over prepped K/V; returns O (bf16, Q's layout).
+    tile_mask (uint8 [B, H, ceil(N/128), ceil(N/block)] on the device) makes it
+    block-sparse: nonzero keeps a key tile for a query tile."""
     _check_input(Q, "Q")
     shape = tuple(Q.shape)
     out = torch.empty_like(Q) if out is None else out
     ws = alloc_workspace(shape, params, Q.device) if workspace is None else workspace
-    st = lib().vc_attn_fwd(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
-                           ctypes.byref(params.c()), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
-    _ok(st, "vc_attn_fwd")
+    if tile_mask is None:
+        st = lib().vc_attn_fwd(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
+                               ctypes.byref(params.c()), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+        _ok(st, "vc_attn_fwd")
+        return out
+    B, H, N, _ = shape
+    want = (B, H, -(-N // 128), -(-N // params.block))
+    if tile_mask.dtype != torch.uint8 or tuple(tile_mask.shape) != want or not tile_mask.is_contiguous() \
+            or tile_mask.device != Q.device:
+        raise ValueError(f"tile_mask must be a contiguous uint8 {want} tensor on {Q.device}")
+    st = lib().vc_attn_fwd_masked(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
+                                  ctypes.byref(params.c()), tile_mask.data_ptr(), out.data_ptr(), ws.data_ptr(),
+                                  ws.numel(), _stream(stream))
+    _ok(st, "vc_attn_fwd_masked")
     return out
 
 

@@ -158,7 +158,9 @@ vc_status prepare_impl(const void* K, const void* V, const vc_shape& s, const vc
 }
 
 vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const vc_params& p, void* O, uint8_t* ws,
-                    const WsLayout& L, cudaStream_t stream) {
+                    const WsLayout& L, cudaStream_t stream, const uint8_t* tile_mask = nullptr);
+vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const vc_params& p, void* O, uint8_t* ws,
+                    const WsLayout& L, cudaStream_t stream, const uint8_t* tile_mask) {
     const int BH = s.B * s.H, N = s.N, D = s.d, BK = p.block;
     const int T = (N + BK - 1) / BK;
     const uint64_t Tp = (uint64_t)T * BK;
@@ -180,6 +182,7 @@ vc_status attn_impl(const void* Q, const vc_prep& pr, const vc_shape& s, const v
     a.v_mean = pr.v_mean;
     a.v_scale = pr.v_scale;
     a.v_bscale = pr.v_bscale;
+    a.tile_mask = tile_mask;
     a.out = static_cast<__nv_bfloat16*>(O);
     a.N = N;
     a.T = T;
@@ -301,6 +304,21 @@ vc_status vc_attn_fwd(const void* Q, const vc_prep* prep, const vc_shape* shape,
     if ((st = check_device()) != VC_OK) return st;
     return attn_impl(Q, *prep, *shape, *params, O, static_cast<uint8_t*>(workspace), L,
                      static_cast<cudaStream_t>(stream));
+}
+
+vc_status vc_attn_fwd_masked(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params,
+                             const uint8_t* tile_mask, void* O, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    vc_status st = check_shape_params(shape, params);
+    if (st != VC_OK) return st;
+    if (!aligned16(Q) || !aligned16(O) || !aligned16(workspace) || !tile_mask) return VC_ERR_INVALID_ARG;
+    if (params->resid_fmt != 0) return VC_ERR_UNSUPPORTED;  // the mask is read by the 8-bit kernel only
+    if ((st = check_prep_ptrs(prep, params, false)) != VC_OK) return st;
+    const WsLayout L = ws_layout(*shape, *params);
+    if (workspace_bytes < L.total) return VC_ERR_WORKSPACE;
+    if ((st = check_device()) != VC_OK) return st;
+    return attn_impl(Q, *prep, *shape, *params, O, static_cast<uint8_t*>(workspace), L,
+                     static_cast<cudaStream_t>(stream), tile_mask);
 }
 
 vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_shape* shape, const vc_params* params,

@@ -101,7 +101,33 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, const 
     }
 }
 
-template <int D, int BK>
+// Block-sparse key tiles: the first kept tile at or after `from` in a query
+// tile's mask row (T if none); every tile when there is no mask.
+__device__ __forceinline__ int next_kept(const uint8_t* row, int from, int T) {
+    if (!row) return from;
+    while (from < T && row[from] == 0) ++from;
+    return from;
+}
+
+// Kept tiles of a mask row, counted by one warp with 16-byte loads (bytes
+// past T are read only inside the row's 16-byte-aligned span, never past it).
+__device__ __forceinline__ int count_kept(const uint8_t* row, int T, int lane) {
+    int n = 0;
+    for (int t = lane * 16; t < T; t += 32 * 16) {
+        if (t + 16 <= T && (reinterpret_cast<uintptr_t>(row + t) & 15u) == 0) {
+            const uint4 w = *reinterpret_cast<const uint4*>(row + t);
+            n += __popc(__vcmpne4(w.x, 0u)) / 8 + __popc(__vcmpne4(w.y, 0u)) / 8 + __popc(__vcmpne4(w.z, 0u)) / 8 +
+                 __popc(__vcmpne4(w.w, 0u)) / 8;
+        } else {
+            for (int u = t; u < t + 16 && u < T; ++u) n += row[u] != 0;
+        }
+    }
+    return __reduce_add_sync(0xffffffffu, n);
+}
+
+// SPARSE: the block-sparse instantiation (a tile mask is read); the dense one
+// compiles without any of it.
+template <int D, int BK, bool SPARSE>
 __global__ void __launch_bounds__(320, 1)
     vc_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const AttnArgs args) {
@@ -119,7 +145,9 @@ __global__ void __launch_bounds__(320, 1)
     const int q0 = blockIdx.x * Cfg::BM;
     const int bh = blockIdx.y;
     const int N = args.N;
-    const int T = args.T;
+    const int T = args.T;  // key tiles of the head
+    // block-sparse: this query tile's row of the mask (null: every tile)
+    const uint8_t* mrow = SPARSE ? args.tile_mask + ((size_t)bh * gridDim.x + blockIdx.x) * T : nullptr;
 
     auto bar = [&](int i) -> uint32_t { return base + Cfg::OFF_BAR + 8u * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
@@ -146,6 +174,11 @@ __global__ void __launch_bounds__(320, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    int* ta_slot = reinterpret_cast<int*>(smem + Cfg::OFF_MISC + 8);
+    if (SPARSE && warp == 2) {  // the number of key tiles this CTA visits
+        const int ta = count_kept(mrow, T, lane);
+        if (lane == 0) *ta_slot = ta;
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
         tmem_relinquish();
@@ -162,6 +195,9 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const DevCtl ctl = args.ctl;
+    // TA tiles are visited; visit i counts barrier phases and ring stages, and
+    // loads the i-th kept tile (next_kept walks the mask row to it)
+    const int TA = SPARSE ? *ta_slot : T;
 
     if (warp == 0) {
         // -------------------------------------------------------- producer
@@ -169,17 +205,20 @@ __global__ void __launch_bounds__(320, 1)
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             int issued_k = 0, issued_v = 0;
-            for (int t = 0; t < T; ++t) {
+            int cursor = SPARSE ? next_kept(mrow, 0, T) : 0;  // the sparse instantiation walks the mask
+            for (int t = 0; t < TA; ++t) {
+                const int tile = SPARSE ? cursor : t;
+                if constexpr (SPARSE) cursor = next_kept(mrow, cursor + 1, T);
                 const int st = t % STAGES;
                 const int n = t / STAGES;
                 if (n > 0 && !mbar_wait(bar(Cfg::B_KEMPTY + st), (n - 1) & 1, ctl, abort_flag)) break;
                 mbar_expect_tx_arrive(bar(Cfg::B_KFULL + st), Cfg::K_BYTES);
-                tma_load_3d(base + Cfg::OFF_K + st * Cfg::K_BYTES, &tm_k, bar(Cfg::B_KFULL + st), 0, t * BK, bh);
+                tma_load_3d(base + Cfg::OFF_K + st * Cfg::K_BYTES, &tm_k, bar(Cfg::B_KFULL + st), 0, tile * BK, bh);
                 issued_k = t + 1;
                 if (n > 0 && !mbar_wait(bar(Cfg::B_VEMPTY + st), (n - 1) & 1, ctl, abort_flag)) break;
                 mbar_expect_tx_arrive(bar(Cfg::B_VFULL + st), Cfg::V_BYTES + Cfg::MU_BYTES);
-                tma_load_3d(base + Cfg::OFF_V + st * Cfg::VX_BYTES, &tm_v, bar(Cfg::B_VFULL + st), t * BK, 0, bh);
-                bulk_load(base + Cfg::OFF_MU + st * Cfg::MU_BYTES, args.v_mean + ((size_t)bh * T + t) * D,
+                tma_load_3d(base + Cfg::OFF_V + st * Cfg::VX_BYTES, &tm_v, bar(Cfg::B_VFULL + st), tile * BK, 0, bh);
+                bulk_load(base + Cfg::OFF_MU + st * Cfg::MU_BYTES, args.v_mean + ((size_t)bh * T + tile) * D,
                           Cfg::MU_BYTES, bar(Cfg::B_VFULL + st));
                 issued_v = t + 1;
             }
@@ -232,9 +271,9 @@ __global__ void __launch_bounds__(320, 1)
             mma_commit_warp(bar(Cfg::B_VEMPTY + st));
             return true;
         };
-        if (ok) ok = issue_qk(0);
-        for (int t = 0; ok && t < T; ++t) {
-            if (t + 1 < T && !issue_qk(t + 1)) break;
+        if (ok && TA > 0) ok = issue_qk(0);
+        for (int t = 0; ok && t < TA; ++t) {
+            if (t + 1 < TA && !issue_qk(t + 1)) break;
             if (!issue_pv(t)) break;
         }
         mma_commit_warp(bar(Cfg::B_MMADONE));
@@ -269,11 +308,16 @@ __global__ void __launch_bounds__(320, 1)
         const float aq = __fmul_rn(args.kappa, sqv);
         const float c0 = 56.0f + (float)args.beta;
         float M = 0.0f;
-        float sk_next = args.k_scale[(size_t)bh * T];
-        for (int t = 0; t < T; ++t) {
+        int tile_next = SPARSE ? next_kept(mrow, 0, T) : 0;  // the sparse instantiation walks the mask
+        float sk_next = TA > 0 ? args.k_scale[(size_t)bh * T + tile_next] : 0.0f;
+        for (int t = 0; t < TA; ++t) {
             const int sb = t & 1;
+            const int tile = SPARSE ? tile_next : t;
             const float sk = sk_next;
-            if (t + 1 < T) sk_next = args.k_scale[(size_t)bh * T + t + 1];
+            if (t + 1 < TA) {
+                if constexpr (SPARSE) tile_next = next_kept(mrow, tile + 1, T);
+                sk_next = args.k_scale[(size_t)bh * T + (SPARSE ? tile_next : t + 1)];
+            }
             if (!warp_wait(bar(Cfg::B_SFULL + sb), (t >> 1) & 1, ctl, abort_flag)) break;
             tc_fence_after();
             float s[BK];
@@ -281,7 +325,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int c = 0; c < BK / 32; ++c) tmem_ld32(lane_tmem + Cfg::S_COL0 + sb * BK + 32 * c, s + 32 * c);
             tmem_wait_ld();
 
-            const int valid = N - t * BK;
+            const int valid = N - tile * BK;
             if (valid < BK) {
 #pragma unroll
                 for (int j = 0; j < BK; ++j)
@@ -359,16 +403,16 @@ __global__ void __launch_bounds__(320, 1)
         float l = 0.0f;  // running row sum after the last tile seen
         // k of tile 0 (always 0); each later tile's k is read one iteration
         // early, to scale l before that tile's PV.
-        bool ok = T == 0 || warp_wait(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag);
+        bool ok = TA == 0 || warp_wait(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag);
         int kinc = 0;
-        for (int t = 0; ok && t < T; ++t) {
+        for (int t = 0; ok && t < TA; ++t) {
             const int st = t % STAGES;
             if (!(ok = warp_wait(bar(Cfg::B_PVDONE + (t & 1)), (t >> 1) & 1, ctl, abort_flag))) break;
             tc_fence_after();
             const float lt = tmem_ld1(lane_tmem + Cfg::L_COL);
             tmem_wait_ld();
             const int kt = kinc;  // this tile's k
-            if (t + 1 < T) {
+            if (t + 1 < TA) {
                 // l(t) * 2^-k(t+1) into O's l column (exact), before PV(t+1),
                 // which waits for l_read(t); the softmax scales the rest of O
                 const int tn = t + 1;
@@ -409,8 +453,8 @@ __global__ void __launch_bounds__(320, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(Cfg::B_VEMPTY + st));
         }
-        if (ok && T > 0) {
-            // The last PV (tile T-1) has completed, so O is final.
+        if (ok && TA > 0) {
+            // The last PV has completed, so O is final.
             tc_fence_after();
             const float inv_l = 1.0f / l;
             const float* vsc = args.v_scale + (size_t)bh * D;
@@ -435,6 +479,10 @@ __global__ void __launch_bounds__(320, 1)
                     dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                 }
             }
+        } else if (SPARSE && ok && TA == 0 && qrow < N) {  // a block-sparse row with no key tile: 0
+            uint4* dst = reinterpret_cast<uint4*>(args.out + ((size_t)bh * N + qrow) * D);
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
 
@@ -456,13 +504,19 @@ cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const At
     using Cfg = AttnCfg<D, BK>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(vc_attn_kernel<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Cfg::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(vc_attn_kernel<D, BK, false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(vc_attn_kernel<D, BK, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     dim3 grid((a.N + Cfg::BM - 1) / Cfg::BM, BH);
-    vc_attn_kernel<D, BK><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tk, tv, a);
+    if (a.tile_mask)
+        vc_attn_kernel<D, BK, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tk, tv, a);
+    else
+        vc_attn_kernel<D, BK, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tk, tv, a);
     return cudaGetLastError();
 }
 

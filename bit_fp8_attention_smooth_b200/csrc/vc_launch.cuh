@@ -13,6 +13,7 @@ struct AttnArgs {
     const float* v_mean;   // [BH, T, D]
     const float* v_scale;  // [BH, D]
     const uint8_t* v_bscale;  // 4-bit path: [BH, T, D, BK/16] UE4M3 block scales of the V residual
+    const uint8_t* tile_mask; // block-sparse: [BH, Tq, T], nonzero keeps key tile t for query tile q; null: dense
     __nv_bfloat16* out;    // [BH, N, D]
     int N, T;
     float kappa;  // fp32(8 * log2(e) / sqrt(D))

@@ -167,6 +167,22 @@ vc_status vc_smooth_prepare(const void* K, const void* V, const vc_shape* shape,
 vc_status vc_attn_fwd(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params, void* O,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * vc_attn_fwd over a block-sparse subset of key tiles (chooseai.io news 7051,
+ * 意义与局限: VC-Attention stacks with sparse attention).
+ *   tile_mask  uint8 [B, H, Tq, T] device input, Tq = ceil(N / 128) query
+ *              tiles of 128 rows, T = ceil(N / block) key tiles in regrouped
+ *              order (the hardware blocks of vc_smooth_prepare); nonzero keeps
+ *              key tile t for every row of query tile q.
+ * A dropped tile takes no part in the row's max, ExpCast weights, row sums or
+ * mean restore; a row whose tiles are all dropped outputs 0.  All ones is
+ * vc_attn_fwd.  resid_fmt 1 is not supported (VC_ERR_UNSUPPORTED).  The mask
+ * must not change until the call has run.
+ */
+vc_status vc_attn_fwd_masked(const void* Q, const vc_prep* prep, const vc_shape* shape, const vc_params* params,
+                             const uint8_t* tile_mask, void* O, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
 /* vc_smooth_prepare followed by vc_attn_fwd on the same stream: the drop-in
  * attention call.  `scratch` receives the prep outputs. */
 vc_status vc_attention(const void* Q, const void* K, const void* V, const vc_shape* shape, const vc_params* params,
