@@ -77,30 +77,6 @@ struct AttnCfg {
     static_assert((K_BYTES % 1024) == 0 && (VX_BYTES % 1024) == 0, "swizzled tiles stay 1024-byte aligned");
 };
 
-__device__ __forceinline__ float exp2_neg_int(int k) {
-    // 2^-k for an integer k >= 0, exactly (0 below the normal range).
-    return k < 127 ? __uint_as_float((uint32_t)(127 - k) << 23) : 0.0f;
-}
-
-// Wait with a warp-uniform verdict: the warp continues only if every lane saw
-// the phase complete.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DevCtl& ctl, volatile int* abort_flag) {
-    const bool ok = mbar_wait(bar, parity, ctl, abort_flag);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Bounded wait that ignores the abort flag (used to drain in-flight copies and
-// MMAs before the CTA exits).
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, const DevCtl& ctl) {
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity)) {
-        if ((int64_t)(globaltimer() - t0) > kDrainNs) {
-            record_error(ctl, VC_ERR_DEVICE_TIMEOUT);
-            return;
-        }
-    }
-}
-
 // Block-sparse key tiles: the first kept tile at or after `from` in a query
 // tile's mask row (T if none); every tile when there is no mask.
 __device__ __forceinline__ int next_kept(const uint8_t* row, int from, int T) {

@@ -91,26 +91,6 @@ struct Attn4Cfg {
                   "swizzled tiles stay 1024-byte aligned");
 };
 
-__device__ __forceinline__ float exp2_neg_int4(int k) {
-    return k < 127 ? __uint_as_float((uint32_t)(127 - k) << 23) : 0.0f;
-}
-
-__device__ __forceinline__ bool warp_wait4(uint32_t bar, uint32_t parity, const DevCtl& ctl,
-                                           volatile int* abort_flag) {
-    const bool ok = mbar_wait(bar, parity, ctl, abort_flag);
-    return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ void drain_wait4(uint32_t bar, uint32_t parity, const DevCtl& ctl) {
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity)) {
-        if ((int64_t)(globaltimer() - t0) > kDrainNs) {
-            record_error(ctl, VC_ERR_DEVICE_TIMEOUT);
-            return;
-        }
-    }
-}
-
 // Barrier of the four softmax warps (named barrier 1, 128 threads) that also
 // ANDs a verdict across them: all four see the same result, so a warp never
 // waits there for one that has left.
@@ -277,18 +257,18 @@ __global__ void __launch_bounds__(320, 1)
                 issued_v = t + 1;
             }
             for (int t = issued_k - STAGES < 0 ? 0 : issued_k - STAGES; t < issued_k; ++t)
-                drain_wait4(bar(Cfg::B_KFULL + t % STAGES), (t / STAGES) & 1, ctl);
+                drain_wait(bar(Cfg::B_KFULL + t % STAGES), (t / STAGES) & 1, ctl);
             for (int t = issued_v - STAGES < 0 ? 0 : issued_v - STAGES; t < issued_v; ++t)
-                drain_wait4(bar(Cfg::B_VFULL + t % STAGES), (t / STAGES) & 1, ctl);
+                drain_wait(bar(Cfg::B_VFULL + t % STAGES), (t / STAGES) & 1, ctl);
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
         const uint32_t id_qk = idesc_e4m3_f32(BK);
         const uint32_t id_pv = idesc_nvf4_f32(D + 16);
-        bool ok = warp_wait4(bar(Cfg::B_QREADY), 0, ctl, abort_flag);
+        bool ok = warp_wait(bar(Cfg::B_QREADY), 0, ctl, abort_flag);
         auto issue_qk = [&](int t) -> bool {
             const int st = t % STAGES, sb = t & 1;
-            if (!warp_wait4(bar(Cfg::B_KFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
+            if (!warp_wait(bar(Cfg::B_KFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint64_t dk = smem_desc(base + Cfg::OFF_K + st * Cfg::K_BYTES, D);
 #pragma unroll
@@ -300,11 +280,11 @@ __global__ void __launch_bounds__(320, 1)
         };
         auto issue_pv = [&](int t) -> bool {
             const int st = t % STAGES, pb = t & 1;
-            if (!warp_wait4(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
+            if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
             // l(t-1) read and SFB(t) in TMEM (the correction warps, before l_read(t-1))
-            if (t > 0 && !warp_wait4(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag))
+            if (t > 0 && !warp_wait(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag))
                 return false;
-            if (!warp_wait4(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
+            if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint64_t dp = smem_desc(base + Cfg::OFF_P + pb * Cfg::P_BYTES, Cfg::VROW);
             const uint64_t dv = smem_desc(base + Cfg::OFF_V + st * Cfg::VX_BYTES, Cfg::VROW);
@@ -323,7 +303,7 @@ __global__ void __launch_bounds__(320, 1)
             if (!issue_pv(t)) break;
         }
         mma_commit_warp(bar(Cfg::B_MMADONE));
-        drain_wait4(bar(Cfg::B_MMADONE), 0, ctl);
+        drain_wait(bar(Cfg::B_MMADONE), 0, ctl);
     } else if (warp < 6) {
         // -------------------------------------------------------- softmax
         const int qd = warp & 3;
@@ -361,7 +341,7 @@ __global__ void __launch_bounds__(320, 1)
             const int sb = t & 1;
             const float sk = sk_next;
             if (t + 1 < T) sk_next = args.k_scale[(size_t)bh * T + t + 1];
-            const bool ok = warp_wait4(bar(Cfg::B_SFULL + sb), (t >> 1) & 1, ctl, abort_flag);
+            const bool ok = warp_wait(bar(Cfg::B_SFULL + sb), (t >> 1) & 1, ctl, abort_flag);
             int kinc = 0;
             if (ok) {
                 tc_fence_after();
@@ -435,9 +415,9 @@ __global__ void __launch_bounds__(320, 1)
                 // O holds PV of tiles < t: wait for it, then scale O by 2^-kinc
                 // (l is scaled by the correction warps).  A failed wait skips the
                 // work; the warps stop together at the next tile's barrier.
-                if (warp_wait4(bar(Cfg::B_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) {
+                if (warp_wait(bar(Cfg::B_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag)) {
                     tc_fence_after();
-                    const float f = exp2_neg_int4(kinc);
+                    const float f = exp2_neg_int(kinc);
                     float o[D];
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_tmem + Cfg::O_COL + 32 * c, o + 32 * c);
@@ -479,7 +459,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int c = 0; c < D; ++c) acc[c] = 0.0f;
         float l = 0.0f;
-        bool ok = T == 0 || warp_wait4(bar(Cfg::B_VFULL + 0), 0, ctl, abort_flag);
+        bool ok = T == 0 || warp_wait(bar(Cfg::B_VFULL + 0), 0, ctl, abort_flag);
         if (ok && T > 0) {  // SFB(0) before the first MMA (it waits on q_ready)
             write_sfb(0);
             tmem_wait_st();
@@ -487,11 +467,11 @@ __global__ void __launch_bounds__(320, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(Cfg::B_QREADY));
         }
-        ok = ok && (T == 0 || warp_wait4(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag));
+        ok = ok && (T == 0 || warp_wait(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag));
         int kinc = 0;
         for (int t = 0; ok && t < T; ++t) {
             const int st = t % STAGES;
-            if (!(ok = warp_wait4(bar(Cfg::B_PVDONE + (t & 1)), (t >> 1) & 1, ctl, abort_flag))) break;
+            if (!(ok = warp_wait(bar(Cfg::B_PVDONE + (t & 1)), (t >> 1) & 1, ctl, abort_flag))) break;
             tc_fence_after();
             const float lt = tmem_ld1(lane_tmem + Cfg::L_COL);
             tmem_wait_ld();
@@ -501,20 +481,20 @@ __global__ void __launch_bounds__(320, 1)
                 // O's l column, and the V block scales of tile t+1 (their TMEM
                 // buffer was last read by PV(t-1), complete with PV(t))
                 const int tn = t + 1;
-                if (!(ok = warp_wait4(bar(Cfg::B_KINC + (tn & 3)), (tn >> 2) & 1, ctl, abort_flag))) break;
+                if (!(ok = warp_wait(bar(Cfg::B_KINC + (tn & 3)), (tn >> 2) & 1, ctl, abort_flag))) break;
                 kinc = kinc_ring[(tn & 3) * Cfg::BM + row];
-                if (__any_sync(0xffffffffu, kinc > 0)) tmem_st1(lane_tmem + Cfg::L_COL, lt * exp2_neg_int4(kinc));
-                if (!(ok = warp_wait4(bar(Cfg::B_VFULL + tn % STAGES), (tn / STAGES) & 1, ctl, abort_flag))) break;
+                if (__any_sync(0xffffffffu, kinc > 0)) tmem_st1(lane_tmem + Cfg::L_COL, lt * exp2_neg_int(kinc));
+                if (!(ok = warp_wait(bar(Cfg::B_VFULL + tn % STAGES), (tn / STAGES) & 1, ctl, abort_flag))) break;
                 write_sfb(tn);
                 tmem_wait_st();
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(Cfg::B_LREAD + (t & 1)));
-            if (!(ok = warp_wait4(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag))) break;
+            if (!(ok = warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag))) break;
             float lb;
             if (kt > 0) {
-                const float f = exp2_neg_int4(kt);
+                const float f = exp2_neg_int(kt);
 #pragma unroll
                 for (int c = 0; c < D; ++c) acc[c] *= f;
                 lb = lt - l * f;
