@@ -59,8 +59,7 @@ struct AttnCfg {
     static constexpr int B_SFULL = B_VEMPTY + STAGES;
     static constexpr int B_PFULL = B_SFULL + 2;
     static constexpr int B_PVDONE = B_PFULL + 2;
-    static constexpr int B_LREAD = B_PVDONE + 2;  // correction has read O's l column for the tile
-    static constexpr int B_KINC = B_LREAD + 2;
+    static constexpr int B_KINC = B_PVDONE + 2;
     static constexpr int B_MMADONE = B_KINC + 4;
     static constexpr int NBAR = B_MMADONE + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -141,9 +140,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(Cfg::B_SFULL + i), 1);
-            mbar_init(bar(Cfg::B_PFULL + i), 4);
+            // P(t) posted by the 4 softmax warps, and l(t-1) read (then scaled)
+            // by the 4 correction warps
+            mbar_init(bar(Cfg::B_PFULL + i), 4 + 4);
             mbar_init(bar(Cfg::B_PVDONE + i), 1);
-            mbar_init(bar(Cfg::B_LREAD + i), 4);
         }
         for (int i = 0; i < 4; ++i) mbar_init(bar(Cfg::B_KINC + i), 4);
         mbar_init(bar(Cfg::B_MMADONE), 1);
@@ -231,11 +231,8 @@ __global__ void __launch_bounds__(320, 1)
             // V(t) first (it lands long before the softmax finishes), so PV(t)
             // is issued as soon as p_full(t) completes
             if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
-            // PV(t) adds into O's l column: the correction warps must have read
-            // l(t-1) first (they do so as soon as PV(t-1) lands, long before
-            // the softmax posts P(t))
-            if (t > 0 && !warp_wait(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag))
-                return false;
+            // p_full(t) also carries the correction warps' read of l(t-1): PV(t)
+            // adds into O's l column
             if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint32_t ap = tmem + Cfg::P_COL0 + pb * (BK / 4);
@@ -380,6 +377,7 @@ __global__ void __launch_bounds__(320, 1)
         // k of tile 0 (always 0); each later tile's k is read one iteration
         // early, to scale l before that tile's PV.
         bool ok = TA == 0 || warp_wait(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag);
+        if (ok && TA > 0 && lane == 0) mbar_arrive(bar(Cfg::B_PFULL + 0));  // no l to read before PV(0)
         int kinc = 0;
         for (int t = 0; ok && t < TA; ++t) {
             const int st = t % STAGES;
@@ -390,7 +388,8 @@ __global__ void __launch_bounds__(320, 1)
             const int kt = kinc;  // this tile's k
             if (t + 1 < TA) {
                 // l(t) * 2^-k(t+1) into O's l column (exact), before PV(t+1),
-                // which waits for l_read(t); the softmax scales the rest of O
+                // which waits for these warps on p_full(t+1); the softmax scales
+                // the rest of O
                 const int tn = t + 1;
                 if (!(ok = warp_wait(bar(Cfg::B_KINC + (tn & 3)), (tn >> 2) & 1, ctl, abort_flag))) break;
                 kinc = kinc_ring[(tn & 3) * Cfg::BM + row];
@@ -401,7 +400,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(Cfg::B_LREAD + (t & 1)));
+            if (lane == 0 && t + 1 < TA) mbar_arrive(bar(Cfg::B_PFULL + ((t + 1) & 1)));
             if (!(ok = warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag))) break;
             float lb;
             if (kt > 0) {
