@@ -70,8 +70,7 @@ struct Attn4Cfg {
     static constexpr int B_SFULL = B_VEMPTY + STAGES;
     static constexpr int B_PFULL = B_SFULL + 2;
     static constexpr int B_PVDONE = B_PFULL + 2;
-    static constexpr int B_LREAD = B_PVDONE + 2;
-    static constexpr int B_KINC = B_LREAD + 2;
+    static constexpr int B_KINC = B_PVDONE + 2;
     static constexpr int B_MMADONE = B_KINC + 4;
     static constexpr int NBAR = B_MMADONE + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -198,7 +197,7 @@ __global__ void __launch_bounds__(320, 1)
 
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
-        mbar_init(bar(Cfg::B_QREADY), 4 + 4);  // softmax: Q in TMEM; correction: SFB(0) in TMEM
+        mbar_init(bar(Cfg::B_QREADY), 4);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar(Cfg::B_KFULL + s), 1);
             mbar_init(bar(Cfg::B_KEMPTY + s), 1);
@@ -207,9 +206,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(Cfg::B_SFULL + i), 1);
-            mbar_init(bar(Cfg::B_PFULL + i), 4);
+            // P(t) and its scales posted by the 4 softmax warps; l(t-1) read
+            // and SFB(t) written by the 4 correction warps
+            mbar_init(bar(Cfg::B_PFULL + i), 4 + 4);
             mbar_init(bar(Cfg::B_PVDONE + i), 1);
-            mbar_init(bar(Cfg::B_LREAD + i), 4);
         }
         for (int i = 0; i < 4; ++i) mbar_init(bar(Cfg::B_KINC + i), 4);
         mbar_init(bar(Cfg::B_MMADONE), 1);
@@ -281,9 +281,8 @@ __global__ void __launch_bounds__(320, 1)
         auto issue_pv = [&](int t) -> bool {
             const int st = t % STAGES, pb = t & 1;
             if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
-            // l(t-1) read and SFB(t) in TMEM (the correction warps, before l_read(t-1))
-            if (t > 0 && !warp_wait(bar(Cfg::B_LREAD + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl, abort_flag))
-                return false;
+            // p_full(t): P(t) and SFA(t) from the softmax warps, l(t-1) read and
+            // SFB(t) written by the correction warps
             if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint64_t dp = smem_desc(base + Cfg::OFF_P + pb * Cfg::P_BYTES, Cfg::VROW);
@@ -460,12 +459,12 @@ __global__ void __launch_bounds__(320, 1)
         for (int c = 0; c < D; ++c) acc[c] = 0.0f;
         float l = 0.0f;
         bool ok = T == 0 || warp_wait(bar(Cfg::B_VFULL + 0), 0, ctl, abort_flag);
-        if (ok && T > 0) {  // SFB(0) before the first MMA (it waits on q_ready)
+        if (ok && T > 0) {  // SFB(0) before PV(0), which waits on p_full(0)
             write_sfb(0);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(Cfg::B_QREADY));
+            if (lane == 0) mbar_arrive(bar(Cfg::B_PFULL + 0));
         }
         ok = ok && (T == 0 || warp_wait(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag));
         int kinc = 0;
@@ -477,7 +476,7 @@ __global__ void __launch_bounds__(320, 1)
             tmem_wait_ld();
             const int kt = kinc;
             if (t + 1 < T) {
-                // before PV(t+1), which waits for l_read(t): l(t) * 2^-k(t+1) into
+                // before PV(t+1), which waits for p_full(t+1): l(t) * 2^-k(t+1) into
                 // O's l column, and the V block scales of tile t+1 (their TMEM
                 // buffer was last read by PV(t-1), complete with PV(t))
                 const int tn = t + 1;
@@ -490,7 +489,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(Cfg::B_LREAD + (t & 1)));
+            if (lane == 0 && t + 1 < T) mbar_arrive(bar(Cfg::B_PFULL + ((t + 1) & 1)));
             if (!(ok = warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag))) break;
             float lb;
             if (kt > 0) {
