@@ -50,25 +50,35 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def kernel_code_hash() -> str:
+    """First 16 hex digits of sha256 over vc_attn.cu and vc_device.cuh with
+    // comments and blank lines removed: the code the profiled kernel was
+    built from, indifferent to edits of its comments."""
+    import hashlib
+
+    csrc = os.path.join(ROOT, "bit_fp8_attention_smooth_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("vc_attn.cu", "vc_device.cuh"):
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            lines = (line.split("//", 1)[0].rstrip() for line in f.read().splitlines())
+            h.update("\n".join(line for line in lines if line).encode())
+    return h.hexdigest()[:16]
+
+
 def attn_traffic_bytes(heads: int):
     """DRAM bytes (read + write) of one attention-kernel launch over `heads`
     heads, from the ncu capture summarised in profiles/; None when the kernel
-    sources have changed since that capture (its counters no longer apply)."""
-    import hashlib
+    code has changed since that capture (its counters no longer apply)."""
     import re
 
     prof = os.path.join(ROOT, "profiles", "vc_attn_kernel_mid_32k_h8.md")
-    csrc = os.path.join(ROOT, "bit_fp8_attention_smooth_b200", "csrc")
     try:
         text = open(prof).read()
-        h = hashlib.sha256()
-        for name in ("vc_attn.cu", "vc_device.cuh"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+        code = kernel_code_hash()
     except OSError:
         return None
     m = re.search(r"roofline-traffic: kernel=\S+ sources_sha256_16=([0-9a-f]{16}) dram_bytes_per_head=(\d+)", text)
-    if not m or m.group(1) != h.hexdigest()[:16]:
+    if not m or m.group(1) != code:
         return None
     return int(m.group(2)) * heads
 

@@ -8,7 +8,8 @@
 // softmax (same page, V-Smooth section; theclarity.today: restored during the
 // online softmax, one pass over the values).
 //
-// One CTA computes a 128-row query tile of one (b, h) against all T key tiles.
+// One CTA computes a 128-row query tile of one (b, h) against all T key tiles
+// (the block-sparse instantiation: against the tiles its mask row keeps).
 // The A operands of every MMA live in tensor memory, so shared memory only
 // feeds the B operands (K tile, V^T tile, a constant tile of ones):
 //   TMEM (columns): S0, S1 [BK each] | O [D + 16] | Q [D/4] | P0, P1 [BK/4 each]
@@ -23,11 +24,13 @@
 //   warps 2..5  softmax, one warp per TMEM lane quadrant, a thread per query
 //               row: it first writes the row's E4M3 Q into TMEM; per tile: row
 //               max of S, integer row reference M (raised online; a rise by k
-//               rescales O and l by 2^-k, exactly), ExpCast bytes stored to
-//               TMEM as the A operand of the PV MMA.
-//   warps 6..9  correction, one warp per quadrant: the tile's row sum
-//               l_t = l(t) - 2^-k l(t-1) from O's column D, acc += l_t * mu_t
-//               (the block-mean restore), rescaled with O; epilogue
+//               rescales O by 2^-k, exactly, once PV(t-1) has landed), ExpCast
+//               bytes stored to TMEM as the A operand of the PV MMA.
+//   warps 6..9  correction, one warp per quadrant: after PV(t), the tile's
+//               row sum l_t = l(t) - 2^-k l(t-1) from O's column D; l(t) scaled
+//               by the next tile's 2^-k before that tile's PV (both signal
+//               p_full with the softmax warps); acc += l_t * mu_t (the
+//               block-mean restore), rescaled with O; epilogue
 //               O = (v_scale * O + acc) / l in bf16, original token order.
 // Every wait is bounded (DevCtl); on a timeout the CTA drains its copies and
 // MMAs, frees TMEM and exits with the status word set.  A CTA does nothing
