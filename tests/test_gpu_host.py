@@ -24,20 +24,21 @@ def _inputs(B, H, N, d, seed):
     return w, [synth.tensor_bf16(w, t) for t in "qkv"]
 
 
-def _device_reference(vc, w, q, k, v):
-    params = vc.Params.for_workload(w, beta=64)
+def _device_reference(vc, w, q, k, v, resid_fmt=0):
+    params = vc.Params.for_workload(w, beta=64, resid_fmt=resid_fmt)
     ws = vc.alloc_workspace(tuple(q.shape), params)
     out = vc.attention(q.cuda(), k.cuda(), v.cuda(), params, workspace=ws)
     vc.check(ws)
     return out.cpu()
 
 
-@pytest.mark.parametrize("B,H,N,d,groups", [(1, 6, 1000, 128, 1), (1, 6, 1000, 128, 4), (2, 3, 777, 64, 6),
-                                            (1, 5, 2100, 128, 64)])
-def test_host_call_equals_device_call(vc, B, H, N, d, groups):
+@pytest.mark.parametrize("B,H,N,d,groups,resid_fmt", [(1, 6, 1000, 128, 1, 0), (1, 6, 1000, 128, 4, 0),
+                                                      (2, 3, 777, 64, 6, 0), (1, 5, 2100, 128, 64, 0),
+                                                      (2, 3, 1300, 128, 4, 1)])
+def test_host_call_equals_device_call(vc, B, H, N, d, groups, resid_fmt):
     w, (q, k, v) = _inputs(B, H, N, d, 51)
-    ref = _device_reference(vc, w, q, k, v)
-    params = vc.Params.for_workload(w, beta=64)
+    ref = _device_reference(vc, w, q, k, v, resid_fmt)
+    params = vc.Params.for_workload(w, beta=64, resid_fmt=resid_fmt)
     call = vc.HostAttention(tuple(q.shape), params, groups=groups)
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     oh = torch.empty_like(q).pin_memory()

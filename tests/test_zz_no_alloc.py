@@ -27,15 +27,15 @@ def _metrics(a, b):
     return rel, cos
 
 
-@pytest.mark.parametrize("N,d,block", [(3000, 128, 128), (1000, 64, 64)])
-def test_noalloc_matches_workspace_entry_point(N, d, block):
+@pytest.mark.parametrize("N,d,block,resid_fmt", [(3000, 128, 128, 0), (1000, 64, 64, 0), (2100, 128, 128, 1)])
+def test_noalloc_matches_workspace_entry_point(N, d, block, resid_fmt):
     import bit_fp8_attention_smooth_b200 as vc
     from bit_fp8_attention_smooth_b200 import synth
 
     L = vc.lib()
     w = synth.custom(f"noalloc_{N}_{d}", 1, 2, N, d, 31, pool=8, C=8, iters=4, block=block)
     q, k, v = (synth.tensor_bf16(w, t).cuda() for t in "qkv")
-    params = vc.Params.for_workload(w, beta=64)
+    params = vc.Params.for_workload(w, beta=64, resid_fmt=resid_fmt)
     ws = vc.alloc_workspace(tuple(q.shape), params)
     prep = vc.smooth_prepare(k, v, params, workspace=ws)
     ref = vc.attn_fwd(q, prep, params, workspace=ws)
