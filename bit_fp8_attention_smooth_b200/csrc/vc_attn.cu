@@ -231,11 +231,8 @@ __global__ void __launch_bounds__(320, 1)
         };
         auto issue_pv = [&](int t) -> bool {
             const int st = t % STAGES, pb = t & 1;
-            // V(t) first (it lands long before the softmax finishes), so PV(t)
-            // is issued as soon as p_full(t) completes
-            if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
-            // p_full(t) also carries the correction warps' read of l(t-1): PV(t)
-            // adds into O's l column
+            // p_full(t) also carries the correction warps' read of l(t-1) (PV(t)
+            // adds into O's l column) and their wait for V(t): one wait here
             if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint32_t ap = tmem + Cfg::P_COL0 + pb * (BK / 4);
@@ -380,7 +377,8 @@ __global__ void __launch_bounds__(320, 1)
         // k of tile 0 (always 0); each later tile's k is read one iteration
         // early, to scale l before that tile's PV.
         bool ok = TA == 0 || warp_wait(bar(Cfg::B_KINC + 0), 0, ctl, abort_flag);
-        if (ok && TA > 0 && lane == 0) mbar_arrive(bar(Cfg::B_PFULL + 0));  // no l to read before PV(0)
+        ok = ok && (TA == 0 || warp_wait(bar(Cfg::B_VFULL + 0), 0, ctl, abort_flag));
+        if (ok && TA > 0 && lane == 0) mbar_arrive(bar(Cfg::B_PFULL + 0));  // V(0) landed; no l to read yet
         int kinc = 0;
         for (int t = 0; ok && t < TA; ++t) {
             const int st = t % STAGES;
@@ -401,10 +399,14 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_wait_st();
                 }
             }
+            // V(t+1) landed too before p_full(t+1) (the MMA warp relies on it);
+            // V(t), read below, was waited for one iteration earlier
+            if (t + 1 < TA &&
+                !(ok = warp_wait(bar(Cfg::B_VFULL + (t + 1) % STAGES), ((t + 1) / STAGES) & 1, ctl, abort_flag)))
+                break;
             tc_fence_before();
             __syncwarp();
             if (lane == 0 && t + 1 < TA) mbar_arrive(bar(Cfg::B_PFULL + ((t + 1) & 1)));
-            if (!(ok = warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag))) break;
             float lb;
             if (kt > 0) {
                 const float f = exp2_neg_int(kt);

@@ -280,9 +280,9 @@ __global__ void __launch_bounds__(320, 1)
         };
         auto issue_pv = [&](int t) -> bool {
             const int st = t % STAGES, pb = t & 1;
-            if (!warp_wait(bar(Cfg::B_VFULL + st), (t / STAGES) & 1, ctl, abort_flag)) return false;
             // p_full(t): P(t) and SFA(t) from the softmax warps, l(t-1) read and
-            // SFB(t) written by the correction warps
+            // SFB(t) written by the correction warps, which waited for V(t) to
+            // land before writing SFB(t): one wait here
             if (!warp_wait(bar(Cfg::B_PFULL + pb), (t >> 1) & 1, ctl, abort_flag)) return false;
             tc_fence_after();
             const uint64_t dp = smem_desc(base + Cfg::OFF_P + pb * Cfg::P_BYTES, Cfg::VROW);
