@@ -73,15 +73,16 @@ def test_prep_timeout_is_reported_and_blocks_later_kernels(vc):
     assert torch.equal(out, ref)
 
 
+@pytest.mark.parametrize("resid_fmt", [0, 1], ids=["e4m3", "nvfp4"])
 @pytest.mark.parametrize("limit_ns", [1, 3000, 30000])
-def test_attention_timeout_then_recovers(vc, limit_ns):
+def test_attention_timeout_then_recovers(vc, limit_ns, resid_fmt):
     w, q, k, v = _case(vc)
-    params = vc.Params.for_workload(w, beta=64)
+    params = vc.Params.for_workload(w, beta=64, resid_fmt=resid_fmt)
     ref = _reference(vc, q, k, v, params)
     ws = vc.alloc_workspace(tuple(q.shape), params)
     prep = vc.smooth_prepare(k, v, params, workspace=ws)
     vc.check(ws)
-    fast = vc.Params.for_workload(w, beta=64, wait_limit_ns=limit_ns)
+    fast = vc.Params.for_workload(w, beta=64, wait_limit_ns=limit_ns, resid_fmt=resid_fmt)
     for _ in range(3):
         out = vc.attn_fwd(q, prep, fast, workspace=ws)
         try:
