@@ -74,3 +74,32 @@ def test_oracle_builds_independently():
     path = oracle.build()
     out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
     assert "vo_attn_emul" in out and "vc_" not in out
+
+
+def test_argument_checks_run_before_any_device_call(libpath):
+    """Host-side validation of the entry points answers without a GPU: the
+    checks come before any CUDA call (the pointers below are never used)."""
+    import bit_fp8_attention_smooth_b200 as vc
+
+    L = vc.lib()
+    fake = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced
+    shape = vc._Shape(1, 2, 1000, 128)
+    prep = vc._Prep(*([fake.value] * 8))
+    dense = vc.Params(C=8, iters=2, block=128)
+
+    def masked(params, mask):
+        return L.vc_attn_fwd_masked(fake, ctypes.byref(prep), ctypes.byref(shape), ctypes.byref(params.c()), mask,
+                                    fake, fake, ctypes.c_size_t(1 << 40), None)
+
+    assert masked(dense, None) == vc.VC_ERR_INVALID_ARG  # a mask is required
+    assert masked(vc.Params(C=8, iters=2, block=128, resid_fmt=1), fake) == vc.VC_ERR_UNSUPPORTED
+    assert masked(vc.Params(C=8, iters=2, block=96), fake) == vc.VC_ERR_UNSUPPORTED
+    assert masked(vc.Params(C=8, iters=2, block=128, smooth=3), fake) == vc.VC_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.vc_attn_fwd_masked(odd, ctypes.byref(prep), ctypes.byref(shape), ctypes.byref(dense.c()), fake, fake,
+                                fake, ctypes.c_size_t(1 << 40), None) == vc.VC_ERR_INVALID_ARG
+    # the 4-bit prep needs its block-scale buffer
+    p4 = vc.Params(C=8, iters=2, block=128, resid_fmt=1)
+    no_scales = vc._Prep(*([fake.value] * 7 + [None]))
+    assert L.vc_attn_fwd(fake, ctypes.byref(no_scales), ctypes.byref(shape), ctypes.byref(p4.c()), fake, fake,
+                         ctypes.c_size_t(1 << 40), None) == vc.VC_ERR_INVALID_ARG
