@@ -2,8 +2,8 @@
 // scores as in vc_attn.cu, then a PV product of NVFP4 operands on sm_100a
 // tensor cores (tcgen05 kind::mxf4nvf4, block16 UE4M3 scales).
 //
-// Method: the zerohour.day summary names a 4-bit residual ("per-channel
-// E4M3/NVFP4 residuals") beside the E4M3 one.  A kind::mxf4nvf4 product needs
+// Method: the zerohour.day summary gives NVFP4 beside E4M3 as a format of
+// the per-channel V residual.  A kind::mxf4nvf4 product needs
 // both operands in E2M1, so P is re-coded to NVFP4 in the softmax stage: each
 // run of 16 keys of a row takes the UE4M3 scale E4M3(max/6) of its ExpCast
 // values, and each value the E2M1 code of p * (1/scale).  QK^T stays FP8.

@@ -94,8 +94,8 @@ typedef struct {
  *                                 UE4M3 scale of each 16-token run of a channel:
  *                                 V[perm[i]][c] ~= v_mean[i / block][c] + v_scale[c] *
  *                                   E4M3(v_bscale[i / block][c][(i % block) / 16]) * E2M1(code)
- *   (4-bit residual: the zerohour.day summary's "per-channel E4M3/NVFP4
- *   residuals"; E2M1 and UE4M3 as in the OCP MX formats.)
+ *   (4-bit residual: the zerohour.day summary lists NVFP4 beside E4M3 for
+ *   the per-channel residual; E2M1 and UE4M3 as in the OCP MX formats.)
  */
 typedef struct {
     int32_t* perm;
@@ -150,8 +150,8 @@ vc_status vc_smooth_prepare(const void* K, const void* V, const vc_shape* shape,
 
 /*
  * ExpCast-FP8 attention forward over prepped K/V (chooseai.io news 7051,
- * ExpCast-FP8 section; theclarity.today: the mean goes back in during the
- * online softmax, one pass over the values).
+ * ExpCast-FP8 section; theclarity.today: block means are restored inside
+ * the online softmax, so V is read once).
  *   Q     bf16 [B,H,N,d] device input, original token order
  *   prep  outputs of vc_smooth_prepare for the same shape and block
  *   O     bf16 [B,H,N,d] device output, original token order

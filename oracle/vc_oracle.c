@@ -39,8 +39,8 @@
  *     beta an integer, a single rounding of the exact value.
  *   - Mean restore: O += l_b * mu_b per tile with l_b = sum of the decoded
  *     bytes of the tile, all terms rescaled by 2^-k when M rises by k.
- *   - NVFP4 (the 4-bit residual [MarkTechPost]: "per-channel E4M3/NVFP4
- *     residuals"): E2M1 values (OCP MX FP4: sign, 2 exponent bits with bias 1,
+ *   - NVFP4 (the 4-bit residual [MarkTechPost]: the V residual is quantised
+ *     per channel to E4M3 or to NVFP4): E2M1 values (OCP MX FP4: sign, 2 exponent bits with bias 1,
  *     1 mantissa bit; max 6) in blocks of 16 along the reduction axis, each
  *     block with a UE4M3 scale s = E4M3(amax/6); a value x is coded
  *     E2M1(x * (1/s)), with 1/s and the product rounded to fp32, E2M1 rounding
@@ -222,8 +222,8 @@ VO_API void vo_expcast_array(const float* A, const float* s, const float* cb, in
 }
 
 /* ------------------------------------------------------------------------ */
-/* k-means over one head's value tokens [ChooseAI/V-Smooth] ("lightweight    */
-/* k-means") and [Clarity] ("clusters similar value tokens").  Plain Lloyd.  */
+/* k-means over one head's value tokens [ChooseAI/V-Smooth] (a lightweight  */
+/* k-means) and [Clarity] (like value tokens share a cluster). Plain Lloyd. */
 /* ------------------------------------------------------------------------ */
 VO_API void vo_kmeans(const uint16_t* v, int n, int d, int C, int iters, int32_t* labels, double* cent) {
     double* sums = (double*)calloc((size_t)C * d, sizeof(double));
@@ -370,7 +370,7 @@ VO_API void vo_smooth_v(const uint16_t* v, int n, int d, int bk, const int32_t* 
     free(inv);
 }
 
-/* The 4-bit residual [MarkTechPost] ("per-channel E4M3/NVFP4 residuals"): the
+/* The 4-bit residual [MarkTechPost] (per-channel scales, NVFP4 codes): the
  * same block means and residuals as vo_smooth_v; per channel one fp32 scale
  * s_c = amax_c/(6*448), y = r * (6*448/amax_c); then NVFP4 blocks of 16
  * consecutive tokens of a channel inside each hardware block (bk a multiple of

@@ -7,8 +7,8 @@ Independent references:
 - a small online replay in Python on top of the pinned primitives, for the
   P re-coding inside the attention replay.
 
-The 4-bit residual is the one the pages name as "per-channel E4M3/NVFP4
-residuals" (zerohour.day summary, key facts).
+The 4-bit residual is the NVFP4 option the pages give beside E4M3 for the
+per-channel V residual (zerohour.day summary, key facts).
 """
 import ml_dtypes
 import numpy as np
