@@ -175,3 +175,71 @@ def test_attn_replay_nvfp4_p_vs_python_replay():
     ref_norm = np.linalg.norm(exact)
     assert np.linalg.norm(out - exact) / ref_norm < 0.2
     assert np.linalg.norm(out - r8) / ref_norm < 0.2
+
+
+def torch_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 values -> bf16 bit patterns (uint16), rounded by torch."""
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).bfloat16().view(torch.int16).numpy().view(np.uint16)
+
+
+def _pin_head():
+    w = synth.custom("nvfp4_pin", 1, 1, 200, 64, 5, pool=6, C=6, iters=3, block=64)
+    return w, [synth.head_bits(w, t, 0, 0) for t in "qkv"]
+
+
+@pytest.mark.parametrize("resid_fmt", [0, 1])
+def test_q_zero_closed_form(resid_fmt):
+    """Q = 0 makes every score 0, so M = 0 and every ExpCast byte is 56 + beta
+    = 120 (value 256).  In the 8-bit path P = 256.  In the 4-bit path each
+    16-key block of 256s takes the scale E4M3(256/6) = 44 (nearest of 40, 44)
+    and the code E2M1(256/44 = 5.82) = 6, so P = 264, worked out by hand.  P is
+    the same for every key, so the output is the plain mean of the dequantised
+    V, and l = P * n.  The 200 keys leave a ragged last block of 8."""
+    w, (q, k, v) = _pin_head()
+    n, d = k.shape
+    rows = np.arange(0, n, 9)
+    r = oracle.forward_head(np.zeros((n, d), np.uint16), k, v, rows, C=w.C, iters=w.iters, bk=64, beta=64,
+                            resid_fmt=resid_fmt)
+    np.testing.assert_array_equal(r["M"], 0)
+    np.testing.assert_array_equal(r["l"], (264.0 if resid_fmt else 256.0) * n)
+    prep = r["prep"]
+    rv = oracle.nvfp4_v_values(prep["vq"], prep["vgs"]) if resid_fmt else oracle.e4m3_value(prep["vhat"])
+    deq = np.repeat(prep["vmu"].astype(np.float64), 64, 0)[:n] + prep["vsc"] * rv[:n]
+    np.testing.assert_allclose(r["out"], np.broadcast_to(deq.mean(0), r["out"].shape), rtol=1e-12, atol=1e-12)
+    # and near the mean of V itself: each coded residual lies within half an
+    # E2M1 step (at most one block-scale unit, 6.25% more for the scale's own
+    # rounding) of the true one, and E4M3 within 1/16 of amax
+    if resid_fmt:
+        unit = prep["vsc"] * np.repeat(oracle.e4m3_value(prep["vgs"]), 16, axis=1).reshape(-1, d).max(0)
+        tol = unit * 1.07
+    else:
+        tol = prep["vsc"] * 448.0 / 16
+    assert np.all(np.abs(r["out"][0] - bf16_values(v).mean(0)) <= tol + 1e-9)
+
+
+@pytest.mark.parametrize("resid_fmt", [0, 1])
+def test_v_constant_per_channel_closed_form(resid_fmt):
+    """V constant along the tokens: every block mean is that constant, the
+    residual is 0 (all codes 0), and O = sum_b l_b mu / sum_b l_b is the
+    constant again, whatever Q and K are."""
+    w, (q, k, _) = _pin_head()
+    n, d = k.shape
+    c = (np.random.default_rng(8).standard_normal(d)).astype(np.float32)
+    cb = torch_bf16_bits(c)
+    v = np.broadcast_to(cb, (n, d)).copy()
+    r = oracle.forward_head(q, k, v, np.arange(0, n, 7), C=w.C, iters=w.iters, bk=64, beta=64, resid_fmt=resid_fmt)
+    prep = r["prep"]
+    assert not np.any(prep["vq"] if resid_fmt else prep["vhat"])
+    np.testing.assert_allclose(r["out"], np.broadcast_to(bf16_values(cb), r["out"].shape), rtol=1e-12, atol=0)
+
+
+@pytest.mark.parametrize("resid_fmt", [0, 1])
+def test_single_token_returns_its_value(resid_fmt):
+    """One key: the block mean is the token itself, the residual is 0, and the
+    output is v_0 exactly (bf16 values, products by P exact in fp64)."""
+    rng = np.random.default_rng(9)
+    q, k, v = (torch_bf16_bits(rng.standard_normal((1, 128)).astype(np.float32)) for _ in range(3))
+    r = oracle.forward_head(q, k, v, np.arange(1), C=1, iters=2, bk=128, beta=64, resid_fmt=resid_fmt)
+    np.testing.assert_array_equal(r["out"], bf16_values(v))
