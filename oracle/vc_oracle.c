@@ -21,7 +21,7 @@
  *                        and FP8 softmax casting", section "The arithmetic
  *                        behind the speedup"
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent (the CUDA path takes the same ones):
  *   - E4M3 is the OCP FP8 E4M3 ("fn") format: bias 7, no infinities, 0x7F NaN,
  *     max 448, subnormals m * 2^-9.  Encoding rounds to nearest, ties to even,
  *     and saturates to +-448.
