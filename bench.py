@@ -237,8 +237,12 @@ def launches_per_step(p) -> int:
     shows the same sequence): km_init; per k-means pass km_assign, km_refine,
     km_scan, km_scatter; between passes km_update, km_finalize; then
     prep_kv_block, prep_v_quant, quant_q and the attention kernel.  V-Smooth
-    off: identity_order, prep_kv_block, prep_v_quant (plus a memset)."""
-    prep = (1 + 4 * p.iters + 2 * (p.iters - 1) + 2) if p.smooth else 3
+    off (smooth 0): identity_order, prep_kv_block, prep_v_quant (plus a
+    memset).  A kept regroup (smooth 2): prep_kv_block and prep_v_quant."""
+    if p.smooth == 1:
+        prep = 1 + 4 * p.iters + 2 * (p.iters - 1) + 2
+    else:
+        prep = 3 if p.smooth == 0 else 2
     return prep + 2
 
 

@@ -1,0 +1,133 @@
+"""Host logic of bench.py, on the CPU: the launch count it claims, the traffic
+figure it takes from the committed ncu summary (and drops once the kernel
+code changes), the peak denominators, and the clock-sample parser that
+decides whether a run is kept."""
+import os
+import re
+import shutil
+
+import pytest
+
+import bench
+import bit_fp8_attention_smooth_b200 as vc
+from bit_fp8_attention_smooth_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_launches_per_step_matches_the_launch_list():
+    """The committed launch list records one timed step of the 32K workload
+    as a fixed number of launches (its -c); the bench claims the same."""
+    text = open(os.path.join(ROOT, "profiles", "launch_list_mid_32k_d128.md")).read()
+    count = int(re.search(r"-c (\d+)", text).group(1))
+    p = vc.Params.for_workload(synth.WORKLOADS["mid_32k_d128"], beta=64)
+    assert bench.launches_per_step(p) == count
+
+
+@pytest.mark.parametrize("iters", [1, 2, 10])
+def test_launches_per_step_by_mode(iters):
+    base = vc.Params(C=16, iters=iters, block=128)
+    # k-means: init, 4 per pass, 2 between passes, then K/V block quantisation
+    assert bench.launches_per_step(base) == 1 + 4 * iters + 2 * (iters - 1) + 2 + 2
+    import dataclasses
+
+    assert bench.launches_per_step(dataclasses.replace(base, smooth=0)) == 3 + 2
+    assert bench.launches_per_step(dataclasses.replace(base, smooth=2)) == 2 + 2
+
+
+def _fake_root(tmp_path, per_head=1000):
+    csrc = tmp_path / "bit_fp8_attention_smooth_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in ("vc_attn.cu", "vc_device.cuh"):
+        shutil.copy(os.path.join(ROOT, "bit_fp8_attention_smooth_b200", "csrc", name), csrc / name)
+    (tmp_path / "profiles").mkdir()
+    return csrc
+
+
+def _write_profile(tmp_path, code_hash, per_head):
+    (tmp_path / "profiles" / "vc_attn_kernel_mid_32k_h8.md").write_text(
+        "summary\n\n    roofline-traffic: kernel=vc_attn_kernel<128,128,false> "
+        f"sources_sha256_16={code_hash} dram_bytes_per_head={per_head}\n")
+
+
+def test_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
+    csrc = _fake_root(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_code_hash()
+    assert h == bench.kernel_code_hash() and re.fullmatch(r"[0-9a-f]{16}", h)
+    _write_profile(tmp_path, h, 1234)
+    assert bench.attn_traffic_bytes(40) == 1234 * 40
+    # comments and blank lines do not change the hash
+    src = csrc / "vc_attn.cu"
+    src.write_text("// a new comment\n\n" + src.read_text().replace("\n", "  // trailing\n", 1))
+    assert bench.kernel_code_hash() == h
+    assert bench.attn_traffic_bytes(8) == 1234 * 8
+    # a code change does: the counters no longer apply
+    src.write_text(src.read_text() + "\nstatic int changed_code = 1;\n")
+    assert bench.kernel_code_hash() != h
+    assert bench.attn_traffic_bytes(40) is None
+
+
+def test_traffic_without_a_profile_is_null(tmp_path, monkeypatch):
+    _fake_root(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.attn_traffic_bytes(40) is None
+    (tmp_path / "profiles" / "vc_attn_kernel_mid_32k_h8.md").write_text("no traffic line here\n")
+    assert bench.attn_traffic_bytes(40) is None
+
+
+def test_committed_traffic_line_is_well_formed():
+    text = open(os.path.join(ROOT, "profiles", "vc_attn_kernel_mid_32k_h8.md")).read()
+    m = re.search(r"roofline-traffic: kernel=\S+ sources_sha256_16=([0-9a-f]{16}) dram_bytes_per_head=(\d+)", text)
+    assert m
+    # at least the fp8 Q, K and V of one 32K x 128 head are read
+    assert int(m.group(2)) >= 3 * 32768 * 128
+
+
+def test_peaks_measured_and_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p = bench.load_peaks()
+    assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0 and p["bf16"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(
+        '{"hbm_gbs": 6538.0, "bf16_tflops": 1606.0, "bf16_tflops_sustained": 1384.2}')
+    p = bench.load_peaks()
+    assert p == dict(hbm_gbs=6538.0, bf16=1606.0, bf16_sustained=1384.2, source="measured")
+
+
+def _sampler(lines):
+    c = bench.ClockSampler(0)
+    c.lines = lines
+    return c
+
+
+def test_clock_summary_median_and_reasons():
+    idle = "Not Active"
+    lines = [
+        f"0, 1335, 1965, 950.1, 0x0000000000000004, {idle}, {idle}, {idle}, Active",
+        f"0, 1965, 1965, 400.0, 0x0000000000000000, {idle}, {idle}, {idle}, {idle}",
+        f"0, 1500, 1965, 990.0, 0x0000000000000004, {idle}, {idle}, {idle}, Active",
+        "garbage line",
+        "0, [N/A], 1965, 1.0, 0x0, x, x, x, x",
+    ]
+    s = _sampler(lines).summary()
+    assert s == {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_clock_summary_flags_slowdowns():
+    idle = "Not Active"
+    s = _sampler([f"0, 900, 1965, 700, 0x8, Active, {idle}, Active, {idle}"]).summary()
+    assert s["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+
+
+def test_clock_summary_without_samples_is_null():
+    assert _sampler([]).summary() is None
+
+
+def test_config_names_the_workload_and_its_l2_rule():
+    w = synth.WORKLOADS["mid_32k_d128"]
+    c = bench.config_of(w)
+    assert c["workload"] == w.name and (c["B"], c["H"], c["N"], c["d"]) == (w.B, w.H, w.N, w.d)
+    assert c["residual"] == "e4m3"
+    gb = float(re.search(r"inputs ([0-9.]+) GB", c["l2"]).group(1))
+    assert gb * 1e9 > 126e6
+    assert bench.config_of(synth.WORKLOADS["nvfp4_32k_d128"])["residual"].startswith("nvfp4")
