@@ -103,3 +103,37 @@ def test_argument_checks_run_before_any_device_call(libpath):
     no_scales = vc._Prep(*([fake.value] * 7 + [None]))
     assert L.vc_attn_fwd(fake, ctypes.byref(no_scales), ctypes.byref(shape), ctypes.byref(p4.c()), fake, fake,
                          ctypes.c_size_t(1 << 40), None) == vc.VC_ERR_INVALID_ARG
+
+
+def test_product_path_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    """No CPU fallback: with the library absent, the public calls raise."""
+    import torch
+
+    import bit_fp8_attention_smooth_b200 as vc
+
+    monkeypatch.setattr(vc, "LIB_PATH", str(tmp_path / "libvcattn.so"))
+    monkeypatch.setattr(vc, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        vc.lib()
+    params = vc.Params(C=4, iters=2, block=64)
+    # the workspace size comes from the library too
+    with pytest.raises(RuntimeError, match="missing"):
+        vc.alloc_workspace((1, 1, 128, 64), params, "cpu")
+    # host tensors are refused, never computed on the CPU
+    x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises((RuntimeError, ValueError), match="missing|CUDA tensor"):
+        vc.attention(x, x, x, params)
+
+
+def test_package_never_loads_the_oracle():
+    """The product path (binding and kernels) names no oracle module, file or
+    symbol: the oracle is test infrastructure only."""
+    pkg = os.path.join(ROOT, "bit_fp8_attention_smooth_b200")
+    offenders = []
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                if re.search(r"import\s+oracle|from\s+oracle|vc_oracle|liboracle|\bvo_\w+\(", text):
+                    offenders.append(f)
+    assert not offenders, offenders
