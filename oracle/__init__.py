@@ -19,8 +19,11 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "vc_oracle.c")
-_SO = os.path.join(_HERE, "_build", "libvcoracle.so")
+# VC_ORACLE_SRC points the tests at another copy of the C source (the mutation
+# test plants one mistake in a copy and checks that the pins fail); the
+# library builds beside whichever source is used.
+_SRC = os.environ.get("VC_ORACLE_SRC") or os.path.join(_HERE, "vc_oracle.c")
+_SO = os.path.join(os.path.dirname(os.path.abspath(_SRC)), "_build", "libvcoracle.so")
 _lib = None
 
 

@@ -84,6 +84,44 @@ def test_q_zero_gives_mean_v():
     np.testing.assert_allclose(r["out"][0], bf16_values(v).mean(0), rtol=0, atol=2e-2)
 
 
+def test_scores_round_to_fp32_before_expcast():
+    """Worked by hand, on the replay with A = 1 (kappa = 1, unit scales).  Two
+    keys in one tile: scores 8 and 4.5 + 2^-30.  The max gives M = ceil(8/8) =
+    1, so cb = 56 + 64 - 8 = 112.  Byte 0 is 120 (value 256).  The second
+    score rounds to 4.5 in fp32, t = 116.5 is a tie and goes to the even byte
+    116 (0x74, value 1.5 * 2^7 = 192); unrounded it would be byte 117 (208).
+    So l = 448 and O = (256 v_0 + 192 v_1)/448."""
+    d, bk = 2, 16
+    qv = np.array([[1.0, 1.0]])
+    kv = np.zeros((bk, d))
+    kv[0] = [8.0, 0.0]
+    kv[1] = [4.5, 2.0 ** -30]
+    rv = np.zeros((bk, d))
+    rv[0] = [1.0, 0.0]
+    rv[1] = [0.0, 1.0]
+    out, M, l = oracle.attn_emul(qv, np.ones(1, np.float32), kv, np.ones(1, np.float32), rv, np.zeros((1, d)),
+                                 np.ones(d, np.float32), n=2, bk=bk, beta=BETA, kappa_value=1.0)
+    assert M[0] == 1 and l[0] == 448.0
+    np.testing.assert_array_equal(out[0], [256.0 / 448.0, 192.0 / 448.0])
+
+
+def test_row_reference_of_a_row_of_negative_scores():
+    """Worked by hand, A = 1: scores -20 and -24 in the first (only) tile give
+    M = ceil(-20/8) = -2, taken as it is (not raised from 0), so cb = 56 + 64
+    + 16 = 136 and the bytes are 116 (192) and 112 (0x70, 128): l = 320 and
+    O = (192 v_0 + 128 v_1)/320."""
+    d, bk = 2, 16
+    kv = np.zeros((bk, d))
+    kv[0, 0], kv[1, 0] = -20.0, -24.0
+    rv = np.zeros((bk, d))
+    rv[0] = [1.0, 0.0]
+    rv[1] = [0.0, 1.0]
+    out, M, l = oracle.attn_emul(np.array([[1.0, 0.0]]), np.ones(1, np.float32), kv, np.ones(1, np.float32), rv,
+                                 np.zeros((1, d)), np.ones(d, np.float32), n=2, bk=bk, beta=BETA, kappa_value=1.0)
+    assert M[0] == -2 and l[0] == 320.0
+    np.testing.assert_array_equal(out[0], [0.6, 0.4])
+
+
 def test_joint_permutation_invariance():
     q, k, v = heads()
     n = k.shape[0]

@@ -133,3 +133,17 @@ def test_kappa_constants():
     assert oracle.kappa(64) == float(np.float32(math.log2(math.e)))
     assert oracle.kappa(128) == float(np.float32(math.log2(math.e) / math.sqrt(2.0)))
     assert np.float32(oracle.kappa(64)).view(np.uint32) == 0x3FB8AA3B
+
+
+def test_expcast_rounds_once():
+    """A constructed witness: A * s lies 1.7e-7 above -9.5, so A * s + 120 is
+    just above the tie 110.5 and rounds once to byte 111.  Rounding the
+    product to fp32 first would give exactly -9.5, whose tie goes to the even
+    byte 110.  The single FMA of the method has one rounding."""
+    A = np.float32(float.fromhex("0x1.1787cep+0"))
+    s = np.float32(float.fromhex("-0x1.1668e2p+3"))
+    exact = Fraction(float(A)) * Fraction(float(s))
+    assert Fraction(-19, 2) < exact < Fraction(-19, 2) + Fraction(1, 2 ** 20)
+    assert np.float32(A * s) == np.float32(-9.5)  # the product alone rounds onto the tie
+    b = oracle.expcast_bytes(np.array([A]), np.array([s]), np.array([120.0], np.float32))
+    assert b[0] == 111

@@ -243,3 +243,22 @@ def test_single_token_returns_its_value(resid_fmt):
     q, k, v = (torch_bf16_bits(rng.standard_normal((1, 128)).astype(np.float32)) for _ in range(3))
     r = oracle.forward_head(q, k, v, np.arange(1), C=1, iters=2, bk=128, beta=64, resid_fmt=resid_fmt)
     np.testing.assert_array_equal(r["out"], bf16_values(v))
+
+
+def test_nvfp4_code_uses_the_fp32_reciprocal_of_the_scale():
+    """Worked by hand.  The block {22.5, 4.6875} has amax/6 = 3.75, an E4M3
+    value (code 0x47), so the scale is exact.  Divided exactly, 4.6875/3.75 =
+    1.25 is an E2M1 tie that goes to the even code 2 (value 1.0).  The reading
+    taken codes x * RN(1/s): RN(1/3.75) lies above 1/3.75, the product
+    rounds to 1.2500001 in fp32, past the tie, and the code is 3 (value 1.5)."""
+    from fractions import Fraction
+
+    x = np.zeros(16, np.float32)
+    x[0], x[1] = 22.5, 4.6875
+    codes, scale = oracle.nvfp4_blocks(x[None])
+    assert scale[0] == 0x47 and oracle.e4m3_value(scale)[0] == 3.75
+    assert Fraction(4.6875) / Fraction(3.75) == Fraction(5, 4)  # the exact quotient is the tie
+    r = np.float32(1.0) / np.float32(3.75)
+    assert np.float32(np.float32(4.6875) * r) > np.float32(1.25)
+    np.testing.assert_array_equal(codes[0][:2], [7, 3])
+    assert not codes[0][2:].any()

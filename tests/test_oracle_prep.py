@@ -97,6 +97,31 @@ def test_kmeans_single_cluster_and_tiny_bruteforce():
         assert np.array_equal(lab, np.where(d1 < d0, 1, 0))
 
 
+def _bits(x):
+    return torch.tensor(np.asarray(x, np.float32)).bfloat16().view(torch.int16).numpy().view(np.uint16)
+
+
+def test_kmeans_equidistant_token_goes_to_the_lowest_cluster():
+    """Worked by hand.  Tokens 0, 2, 1 with C = 2: the strided init gives
+    c_0 = v[0] = 0 and c_1 = v[floor(3/2)] = 2, and token 2 (value 1) is at
+    distance 1 from both, so it takes the lower index.  One update moves c_0
+    to 0.5 and leaves c_1 at 2, and the second pass keeps those labels.
+    Ties to the higher index would give [0, 1, 1] and c_1 = 1.5."""
+    v = _bits([[0.0], [2.0], [1.0]])
+    labels, cent = oracle.kmeans(v, 2, 1)
+    np.testing.assert_array_equal(labels, [0, 1, 0])
+    labels, cent = oracle.kmeans(v, 2, 2)
+    np.testing.assert_array_equal(labels, [0, 1, 0])
+    np.testing.assert_array_equal(cent[:, 0], [0.5, 2.0])
+    # in 4 channels with C = 3: the init takes rows 0, 2 and 4, so c_0 and c_2
+    # are both the origin and c_1 = (0, 4, 0, 0).  Tokens 1, 4 and 5 tie
+    # between c_0 and c_2, and token 3 = (2, 2, 0, 0) is at squared distance 8
+    # from all three: every tie goes to cluster 0.
+    v = _bits([[0, 0, 0, 0], [4, 0, 0, 0], [0, 4, 0, 0], [2, 2, 0, 0], [0, 0, 0, 0], [0, 0, 0, 0]])
+    labels, _ = oracle.kmeans(v, 3, 1)
+    np.testing.assert_array_equal(labels, [0, 0, 1, 0, 0, 0])
+
+
 def test_stable_perm_vs_numpy():
     rng = np.random.default_rng(10)
     for C in (1, 3, 64):
