@@ -5,6 +5,7 @@ import pytest
 import torch
 
 import oracle
+from conftest import expcast_rounding_witnesses
 
 pytestmark = pytest.mark.gpu
 
@@ -49,6 +50,9 @@ def test_expcast_bit_exact(vc):
     # the map's domain: 8z + 56 + beta <= 126 (the row reference keeps z <= 0)
     over = A.astype(np.float64) * s + cb > 126
     s[over] = 0.0
+    # products within half an fp32 ulp of a tie: one rounding and two disagree
+    wa, ws, wc, _ = expcast_rounding_witnesses(12)
+    A, s, cb = np.concatenate([A, wa]), np.concatenate([s, ws]), np.concatenate([cb, wc])
     dev = [torch.from_numpy(a).cuda() for a in (A, s, cb)]
     got = vc.expcast_bytes(*dev).cpu().numpy()
     ref = oracle.expcast_bytes(A, s, cb)

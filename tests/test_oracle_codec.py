@@ -135,6 +135,26 @@ def test_kappa_constants():
     assert np.float32(oracle.kappa(64)).view(np.uint32) == 0x3FB8AA3B
 
 
+def test_expcast_rounds_once_on_constructed_witnesses():
+    """Thousands of inputs where one rounding and two disagree: the oracle's
+    byte is the exact rational A*s + cb rounded once, never the byte that an
+    fp32 product would give."""
+    from conftest import expcast_rounding_witnesses
+
+    A, s, cb, prod = expcast_rounding_witnesses(11, 20_000)
+    assert A.size > 10_000
+    got = oracle.expcast_bytes(A, s, cb)
+    for i in range(0, A.size, 7):
+        t = Fraction(float(A[i])) * Fraction(float(s[i])) + int(cb[i])
+        assert t.denominator > 2  # never an exact tie
+        assert got[i] == max(0, round(t)), (i, float(A[i]), float(s[i]), float(cb[i]))
+    d32 = (A * s).astype(np.float64)  # the product rounded to fp32 first: a tie
+    assert np.all(d32 - np.floor(d32) == 0.5)
+    two = d32 + cb.astype(np.float64)
+    two = np.where(np.floor(two) % 2 == 0, np.floor(two), np.ceil(two))
+    assert np.all(got != two)
+
+
 def test_expcast_rounds_once():
     """A constructed witness: A * s lies 1.7e-7 above -9.5, so A * s + 120 is
     just above the tie 110.5 and rounds once to byte 111.  Rounding the
