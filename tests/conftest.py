@@ -42,3 +42,34 @@ def expcast_rounding_witnesses(seed: int, n: int = 400_000):
     # above the tie (the tie would go down), odd when below (it would go up)
     cb = 60 - fl + 2 * rng.integers(-25, 30, fl.size) + (prod < D)
     return A, s, cb.astype(np.float32), prod
+
+
+NVFP4_TIE_SCALES = (2.0, 3.75, 3.5, 1.875, 7.5, 0.75, 13.0, 15.0, 0.5, 1.625, 0.013671875, 0.0390625, 104.0, 240.0)
+E2M1_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def nvfp4_tie_values(seed: int, N: int = 256, d: int = 128):
+    """Seeded V values [N, d] (float32, all bf16-exact) whose 4-bit residual
+    without V-Smooth lands on E2M1 ties.  Token 0 of every channel is 2688,
+    so the channel scale amax/2688 is exactly 1 and y = v.  Each 16-token
+    block leads with 6*s, so its scale E4M3(6s/6) is exactly s, one of
+    NVFP4_TIE_SCALES (448 in the first block).  The other 15 tokens are
+    +-s * m, m an E2M1 midpoint (mostly) or grid value.  Input construction
+    only (test helper, not method arithmetic); returns (v, scale per block
+    [N/16, d])."""
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    assert N % 16 == 0
+    nb = N // 16
+    scales = np.empty((nb, d))
+    v = np.empty((N, d))
+    for j in range(nb):
+        for c in range(d):
+            s = 448.0 if j == 0 else NVFP4_TIE_SCALES[(j + 3 * c) % len(NVFP4_TIE_SCALES)]
+            scales[j, c] = s
+            m = np.where(rng.random(15) < 0.8, rng.choice(E2M1_MIDPOINTS, 15), rng.choice(E2M1_GRID, 15))
+            v[16 * j, c] = 6.0 * s
+            v[16 * j + 1:16 * j + 16, c] = s * m * rng.choice([-1.0, 1.0], 15)
+    return v.astype(np.float32), scales

@@ -150,3 +150,30 @@ def test_four_bit_rejects_block_64(vc):
     with pytest.raises(vc.VcError) as e:
         vc.attention(qd, kd, vd, vc.Params(C=16, iters=8, block=64, resid_fmt=1))
     assert e.value.status == vc.VC_ERR_UNSUPPORTED
+
+
+def test_prep_nvfp4_ties_bit_exact(vc):
+    """The crafted tie workload (V-Smooth off, channel scales 1, block scales
+    set by construction): every code, including thousands of exact E2M1 ties
+    of y * RN(1/s) and of values that only the exact quotient puts on a tie,
+    matches the oracle."""
+    from conftest import nvfp4_tie_values
+
+    v, _ = nvfp4_tie_values(21)
+    n, d = v.shape
+    rng = torch.Generator().manual_seed(5)
+    k = torch.randn((1, 1, n, d), generator=rng).bfloat16()
+    vt = torch.from_numpy(v).bfloat16().reshape(1, 1, n, d)
+    params = vc.Params(C=4, iters=2, block=128, smooth=0, resid_fmt=1)
+    ws = vc.alloc_workspace((1, 1, n, d), params)
+    prep = vc.smooth_prepare(k.cuda(), vt.cuda(), params, workspace=ws)
+    vc.check(ws)
+    prep = prep_to_host(prep)
+    vq, vgs, vmu, vsc = oracle.smooth_v_nvfp4(bits(vt[0, 0]), np.arange(n, dtype=np.int32), 128, False)
+    assert np.array_equal(prep["perm"][0, 0].numpy(), np.arange(n))
+    assert np.array_equal(prep["v_scale"][0, 0].numpy(), vsc)
+    assert np.array_equal(prep["v_mean"][0, 0].numpy(), vmu)
+    assert np.array_equal(prep["v_bscale"][0, 0].numpy().transpose(0, 2, 1), vgs)
+    got = unpack_codes(prep["vt_fp8"][0, 0].numpy())
+    bad = np.argwhere(got != vq)
+    assert bad.size == 0, (bad[:5], got[got != vq][:5], vq[got != vq][:5])

@@ -262,3 +262,36 @@ def test_nvfp4_code_uses_the_fp32_reciprocal_of_the_scale():
     assert np.float32(np.float32(4.6875) * r) > np.float32(1.25)
     np.testing.assert_array_equal(codes[0][:2], [7, 3])
     assert not codes[0][2:].any()
+
+
+def test_crafted_tie_blocks():
+    """On the crafted tie workload (V-Smooth off) the channel scales are 1,
+    each block takes the scale it was built with, and every code follows
+    the reading: an exact E2M1 tie of y * RN(1/s) goes to the even code, and
+    a value that only the exact quotient would put on a tie rounds from the
+    fp32 product.  Both kinds occur by the thousand."""
+    from conftest import nvfp4_tie_values
+
+    v, scales = nvfp4_tie_values(21)
+    vb = torch_bf16_bits(v)
+    assert np.array_equal(bf16_values(vb), v.astype(np.float64))  # bf16-exact
+    n, d = v.shape
+    vq, vgs, vmu, vsc = oracle.smooth_v_nvfp4(vb, np.arange(n, dtype=np.int32), 128, False)
+    assert np.all(vsc == 1.0) and not vmu.any()
+    np.testing.assert_array_equal(oracle.e4m3_value(vgs).reshape(-1, d), scales)
+    sv = np.repeat(scales, 16, axis=0).astype(np.float32)
+    prod = (v * (np.float32(1.0) / sv)).astype(np.float32).astype(np.float64)
+    quotient = v.astype(np.float64) / sv
+    mags = np.abs(prod)
+    tie = np.isin(mags, (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0))
+    witness = ~tie & np.isin(np.abs(quotient), (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0))
+    assert tie.sum() > 1000 and witness.sum() > 1000, (tie.sum(), witness.sum())
+    got = oracle.e2m1_value(vq)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    lo = grid[np.searchsorted(grid, mags, side="right") - 1]
+    hi = grid[np.minimum(np.searchsorted(grid, mags, side="right"), 7)]
+    lo_even = np.isin(lo, (0.0, 1.0, 2.0, 4.0))  # codes 0, 2, 4, 6
+    want_tie = np.where(lo_even, lo, hi) * np.sign(prod)
+    np.testing.assert_array_equal(got[tie], want_tie[tie])
+    nearest = np.where(mags - lo < hi - mags, lo, hi) * np.sign(prod)
+    np.testing.assert_array_equal(got[witness], nearest[witness])
