@@ -37,11 +37,6 @@ __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { retur
 // to 16; pad rows are zero), plus fp32 squared norms [BH, Cp]: v.c is computed
 // on tensor cores as v.hi + v.lo (v is exact in bf16), so the distance
 // |c|^2 - 2 v.c carries about 2^-16 relative error in c.
-__device__ __forceinline__ void store_centroid(float c, __nv_bfloat16* hi, __nv_bfloat16* lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(c);
-    *hi = h;
-    *lo = __float2bfloat16_rn(c - __bfloat162float(h));
-}
 
 // Sum over the D threads of a block (D = blockDim.x, 64 or 128).
 __device__ __forceinline__ float block_sum_d(float x, float* red) {
