@@ -218,26 +218,61 @@ def alloc_workspace(shape, params: Params, device="cuda") -> torch.Tensor:
     return torch.zeros(workspace_bytes(shape, params), dtype=torch.uint8, device=device)
 
 
-def alloc_prep(shape, params: Params, device="cuda") -> Dict[str, torch.Tensor]:
-    """Caller-owned prep buffers with their logical shapes and dtypes (the
-    4-bit residual, resid_fmt 1: vt_fp8 holds two E2M1 codes a byte and
-    v_bscale the UE4M3 block scales)."""
+def prep_layout(shape, params: Params) -> Dict[str, tuple]:
+    """Logical shape and dtype of each prep buffer (the 4-bit residual,
+    resid_fmt 1: vt_fp8 holds two E2M1 codes a byte and v_bscale the UE4M3
+    block scales; v_bscale exists only then)."""
     B, H, N, d = shape
     T = -(-N // params.block)
     Tp = T * params.block
     fp4 = params.resid_fmt == 1
-    prep = {
-        "perm": torch.empty((B, H, N), dtype=torch.int32, device=device),
-        "labels": torch.empty((B, H, N), dtype=torch.int32, device=device),
-        "k_fp8": torch.empty((B, H, Tp, d), dtype=torch.uint8, device=device),
-        "k_scale": torch.empty((B, H, T), dtype=torch.float32, device=device),
-        "vt_fp8": torch.empty((B, H, d, Tp // 2 if fp4 else Tp), dtype=torch.uint8, device=device),
-        "v_mean": torch.empty((B, H, T, d), dtype=torch.float32, device=device),
-        "v_scale": torch.empty((B, H, d), dtype=torch.float32, device=device),
+    layout = {
+        "perm": ((B, H, N), torch.int32),
+        "labels": ((B, H, N), torch.int32),
+        "k_fp8": ((B, H, Tp, d), torch.uint8),
+        "k_scale": ((B, H, T), torch.float32),
+        "vt_fp8": ((B, H, d, Tp // 2 if fp4 else Tp), torch.uint8),
+        "v_mean": ((B, H, T, d), torch.float32),
+        "v_scale": ((B, H, d), torch.float32),
     }
     if fp4:
-        prep["v_bscale"] = torch.empty((B, H, T, d, params.block // 16), dtype=torch.uint8, device=device)
-    return prep
+        layout["v_bscale"] = ((B, H, T, d, params.block // 16), torch.uint8)
+    return layout
+
+
+def alloc_prep(shape, params: Params, device="cuda") -> Dict[str, torch.Tensor]:
+    """Caller-owned prep buffers with their logical shapes and dtypes."""
+    return {n: torch.empty(sh, dtype=dt, device=device) for n, (sh, dt) in prep_layout(shape, params).items()}
+
+
+def _check_like(t, name: str, shape, dtype, device):
+    """The library indexes raw pointers by the problem shape, so every buffer
+    it touches must have exactly that shape and dtype, contiguous, on the
+    device of the call."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or tuple(t.shape) != tuple(shape) \
+            or not t.is_contiguous() or t.device != device:
+        got = (f"{t.dtype} {tuple(t.shape)} on {t.device}" + ("" if t.is_contiguous() else ", not contiguous")
+               if isinstance(t, torch.Tensor) else type(t).__name__)
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device} "
+                         f"(got {got})")
+
+
+def _check_prep(prep, shape, params: Params, device):
+    for n, (sh, dt) in prep_layout(shape, params).items():
+        if n not in prep:
+            raise ValueError(f"prep buffer {n!r} is missing (resid_fmt {params.resid_fmt})")
+        _check_like(prep[n], f"prep[{n!r}]", sh, dt, device)
+
+
+def _check_out(out, Q: torch.Tensor):
+    _check_like(out, "out", Q.shape, torch.bfloat16, Q.device)
+
+
+def _ws_args(ws: torch.Tensor, device):
+    """Workspace pointer and size in bytes (the library checks the size)."""
+    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous() or ws.device != device:
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+    return ws.data_ptr(), ws.numel() * ws.element_size()
 
 
 def _prep_struct(prep: Dict[str, torch.Tensor]) -> _Prep:
@@ -251,12 +286,13 @@ def _prep_struct(prep: Dict[str, torch.Tensor]) -> _Prep:
 def smooth_prepare(K: torch.Tensor, V: torch.Tensor, params: Params, prep=None, workspace=None, stream=None):
     """V-Smooth prep; returns the prep buffers (k-means labels included)."""
     _check_input(K, "K")
-    _check_input(V, "V")
+    _check_like(V, "V", K.shape, torch.bfloat16, K.device)
     shape = tuple(K.shape)
     prep = alloc_prep(shape, params, K.device) if prep is None else prep
-    ws = alloc_workspace(shape, params, K.device) if workspace is None else workspace
+    _check_prep(prep, shape, params, K.device)
+    ws_ptr, ws_bytes = _ws_args(alloc_workspace(shape, params, K.device) if workspace is None else workspace, K.device)
     st = lib().vc_smooth_prepare(K.data_ptr(), V.data_ptr(), ctypes.byref(_shape(K)), ctypes.byref(params.c()),
-                                 ctypes.byref(_prep_struct(prep)), ws.data_ptr(), ws.numel(), _stream(stream))
+                                 ctypes.byref(_prep_struct(prep)), ws_ptr, ws_bytes, _stream(stream))
     _ok(st, "vc_smooth_prepare")
     return prep
 
@@ -268,11 +304,13 @@ def attn_fwd(Q: torch.Tensor, prep, params: Params, out=None, workspace=None, st
     block-sparse: nonzero keeps a key tile for a query tile."""
     _check_input(Q, "Q")
     shape = tuple(Q.shape)
+    _check_prep(prep, shape, params, Q.device)
     out = torch.empty_like(Q) if out is None else out
-    ws = alloc_workspace(shape, params, Q.device) if workspace is None else workspace
+    _check_out(out, Q)
+    ws_ptr, ws_bytes = _ws_args(alloc_workspace(shape, params, Q.device) if workspace is None else workspace, Q.device)
     if tile_mask is None:
         st = lib().vc_attn_fwd(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
-                               ctypes.byref(params.c()), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+                               ctypes.byref(params.c()), out.data_ptr(), ws_ptr, ws_bytes, _stream(stream))
         _ok(st, "vc_attn_fwd")
         return out
     B, H, N, _ = shape
@@ -281,23 +319,26 @@ def attn_fwd(Q: torch.Tensor, prep, params: Params, out=None, workspace=None, st
             or tile_mask.device != Q.device:
         raise ValueError(f"tile_mask must be a contiguous uint8 {want} tensor on {Q.device}")
     st = lib().vc_attn_fwd_masked(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
-                                  ctypes.byref(params.c()), tile_mask.data_ptr(), out.data_ptr(), ws.data_ptr(),
-                                  ws.numel(), _stream(stream))
+                                  ctypes.byref(params.c()), tile_mask.data_ptr(), out.data_ptr(), ws_ptr,
+                                  ws_bytes, _stream(stream))
     _ok(st, "vc_attn_fwd_masked")
     return out
 
 
 def attention(Q, K, V, params: Params, out=None, prep=None, workspace=None, stream=None) -> torch.Tensor:
     """The drop-in call: V-Smooth prep then ExpCast-FP8 attention."""
-    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
-        _check_input(t, n)
+    _check_input(Q, "Q")
+    for t, n in ((K, "K"), (V, "V")):
+        _check_like(t, n, Q.shape, torch.bfloat16, Q.device)
     shape = tuple(Q.shape)
     out = torch.empty_like(Q) if out is None else out
+    _check_out(out, Q)
     prep = alloc_prep(shape, params, Q.device) if prep is None else prep
-    ws = alloc_workspace(shape, params, Q.device) if workspace is None else workspace
+    _check_prep(prep, shape, params, Q.device)
+    ws_ptr, ws_bytes = _ws_args(alloc_workspace(shape, params, Q.device) if workspace is None else workspace, Q.device)
     st = lib().vc_attention(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(_shape(Q)),
                             ctypes.byref(params.c()), ctypes.byref(_prep_struct(prep)), out.data_ptr(),
-                            ws.data_ptr(), ws.numel(), _stream(stream))
+                            ws_ptr, ws_bytes, _stream(stream))
     _ok(st, "vc_attention")
     return out
 
@@ -311,7 +352,9 @@ def attn_fwd_noalloc(Q: torch.Tensor, prep, params: Params, out=None, stream=Non
     Problems larger than the scratch raise VcError(VC_ERR_WORKSPACE); calls
     that overlap on the GPU race on the shared scratch."""
     _check_input(Q, "Q")
+    _check_prep(prep, tuple(Q.shape), params, Q.device)
     out = torch.empty_like(Q) if out is None else out
+    _check_out(out, Q)
     st = lib().vc_attn_fwd_noalloc(Q.data_ptr(), ctypes.byref(_prep_struct(prep)), ctypes.byref(_shape(Q)),
                                    ctypes.byref(params.c()), out.data_ptr(), _stream(stream))
     _ok(st, "vc_attn_fwd_noalloc")
@@ -320,19 +363,23 @@ def attn_fwd_noalloc(Q: torch.Tensor, prep, params: Params, out=None, stream=Non
 
 def check(workspace: torch.Tensor, stream=None) -> None:
     """Synchronise and raise VcError if a kernel recorded a device-side timeout."""
-    _ok(lib().vc_check(workspace.data_ptr(), _stream(stream)), "vc_check")
+    ws_ptr, _ = _ws_args(workspace, workspace.device)
+    _ok(lib().vc_check(ws_ptr, _stream(stream)), "vc_check")
 
 
 def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
-    assert x.dtype == torch.float32 and x.is_cuda and x.is_contiguous()
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
     out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _ok(lib().vc_e4m3_encode(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)), "vc_e4m3_encode")
     return out
 
 
 def expcast_bytes(A: torch.Tensor, s: torch.Tensor, cb: torch.Tensor, stream=None) -> torch.Tensor:
-    for t in (A, s, cb):
-        assert t.dtype == torch.float32 and t.is_cuda and t.is_contiguous() and t.shape == A.shape
+    if not A.is_cuda:
+        raise ValueError("A, s and cb must be CUDA tensors")
+    for t, n in ((A, "A"), (s, "s"), (cb, "cb")):
+        _check_like(t, n, A.shape, torch.float32, A.device)
     out = torch.empty(A.shape, dtype=torch.uint8, device=A.device)
     _ok(lib().vc_expcast_bytes(A.data_ptr(), s.data_ptr(), cb.data_ptr(), out.data_ptr(), A.numel(), _stream(stream)),
         "vc_expcast_bytes")
