@@ -5,7 +5,7 @@ attention output) is carved out of a larger allocation whose margins hold a
 known byte pattern.  After the prep, the dense attention and the block-sparse
 attention, the margins must still hold it.  This stands in for a memory
 checker on ragged shapes, both residual formats, both block sizes and
-V-Smooth on and off.  Not yet run on a GPU when written.  The
+V-Smooth on and off.  The
 margins keep every base address aligned to 4 KiB, as an ordinary allocation
 would be."""
 import math
