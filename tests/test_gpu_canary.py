@@ -6,8 +6,8 @@ known byte pattern.  After the prep, the dense attention and the block-sparse
 attention, the margins must still hold it.  This stands in for a memory
 checker on ragged shapes, both residual formats, both block sizes and
 V-Smooth on and off.  The
-margins keep every base address aligned to 4 KiB, as an ordinary allocation
-would be."""
+margins are 16 KiB, so every base address keeps the alignment of an ordinary
+allocation (512 bytes from the caching allocator; TMA needs 16)."""
 import math
 
 import pytest
