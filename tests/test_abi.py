@@ -137,3 +137,28 @@ def test_package_never_loads_the_oracle():
                 if re.search(r"import\s+oracle|from\s+oracle|vc_oracle|liboracle|\bvo_\w+\(", text):
                     offenders.append(f)
     assert not offenders, offenders
+
+
+@pytest.mark.parametrize("shape", [(1, 40, 32768, 128), (2, 3, 777, 64), (1, 1, 1, 128), (1, 2, 300, 128)])
+@pytest.mark.parametrize("block,resid_fmt", [(64, 0), (128, 0), (128, 1)])
+def test_binding_layout_matches_the_library_sizes(libpath, shape, block, resid_fmt):
+    """The binding checks buffers against its own table of prep shapes; the
+    library sizes them with vc_prep_buffer_bytes.  Both must agree byte for
+    byte, field by field, or a buffer the binding accepts could be too small."""
+    import torch
+
+    import bit_fp8_attention_smooth_b200 as vc
+
+    params = vc.Params(C=min(16, shape[2]), iters=3, block=block, resid_fmt=resid_fmt)  # C <= N
+    sizes = vc.prep_sizes(shape, params)
+    layout = vc.prep_layout(shape, params)
+    for i, name in enumerate(vc.PREP_FIELDS):
+        want = sizes[i]
+        if name not in layout:
+            assert want == 0, name
+            continue
+        sh, dt = layout[name]
+        n = 1
+        for x in sh:
+            n *= x
+        assert n * torch.empty((), dtype=dt).element_size() == want, (name, sh, dt, want)
