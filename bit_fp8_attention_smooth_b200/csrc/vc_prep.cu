@@ -17,6 +17,8 @@
 //             km_scatter      perm[position] = token (stable within a cluster)
 //             km_update       fp64 member sums over fixed slices of the stable order
 //             km_finalize     c_k = sum / count (empty clusters keep c_k)
+//   identity_order            V-Smooth off (smooth 0): perm = identity, labels 0, no k-means
+//   (smooth 2 runs no k-means kernel and keeps the perm already in the prep buffers)
 //   prep_kv_block             per block: K amax scale + E4M3 K, V block mean (fp64 sum),
 //                             residual channel amax
 //   prep_v_quant              per-channel residual scale, E4M3 residual, transposed
@@ -27,7 +29,6 @@
 #include "vc_launch.cuh"
 
 namespace vc {
-
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
 __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
