@@ -1,7 +1,7 @@
 """ctypes front end of the plain C oracle (vc_oracle.c).
 
-TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the
-benchmark's CPU-baseline leg are the only users.  It takes numpy arrays and
+TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check, and the
+benchmark's CPU-baseline leg and `--impl reference` arm are the only users.  It takes numpy arrays and
 returns numpy arrays; it imports nothing from the CUDA package, and the CUDA
 package never imports it.
 

@@ -2,8 +2,8 @@
  * vc_oracle.c -- plain, slow CPU reference for VC-Attention (V-Smooth prep +
  * ExpCast-FP8 attention forward).
  *
- * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check and
- * the benchmark's CPU-baseline leg may load this library.  The CUDA path never
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check,
+ * and the benchmark's CPU-baseline leg and reference arm may load this library.  The CUDA path never
  * calls it, and it shares no code, header, table or constant with the CUDA
  * path: every format and formula here is written from its definition.
  *
@@ -40,9 +40,10 @@
  *   - Mean restore: O += l_b * mu_b per tile with l_b = sum of the decoded
  *     bytes of the tile, all terms rescaled by 2^-k when M rises by k.
  *   - NVFP4 (the 4-bit residual [MarkTechPost]: the V residual is quantised
- *     per channel to E4M3 or to NVFP4): E2M1 values (OCP MX FP4: sign, 2 exponent bits with bias 1,
- *     1 mantissa bit; max 6) in blocks of 16 along the reduction axis, each
- *     block with a UE4M3 scale s = E4M3(amax/6); a value x is coded
+ *     per channel to E4M3 or to NVFP4): E2M1 values (OCP MX FP4: sign, 2
+ *     exponent bits with bias 1, 1 mantissa bit; max 6) in blocks of 16 along
+ *     the reduction axis, each block with a UE4M3 scale s = E4M3(amax/6); a
+ *     value x is coded
  *     E2M1(x * (1/s)), with 1/s and the product rounded to fp32, E2M1 rounding
  *     to nearest (ties to the even code) and saturating at 6; a zero scale
  *     codes zeros.  The V residual keeps one fp32 scale per channel,
