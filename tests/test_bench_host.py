@@ -1,7 +1,7 @@
 """Host logic of bench.py, on the CPU: the launch count it claims, the traffic
 figure it takes from the committed ncu summary (and drops once the kernel
-code changes), the peak denominators, and the clock-sample parser that
-decides whether a run is kept."""
+code changes), the peak denominators, the clock-sample parser that decides
+whether a run is kept, and the oracle arm (`--impl reference`) end to end."""
 import os
 import re
 import shutil
@@ -131,3 +131,34 @@ def test_config_names_the_workload_and_its_l2_rule():
     gb = float(re.search(r"inputs ([0-9.]+) GB", c["l2"]).group(1))
     assert gb * 1e9 > 126e6
     assert bench.config_of(synth.WORKLOADS["nvfp4_32k_d128"])["residual"].startswith("nvfp4")
+
+
+def _run_reference(env_extra):
+    import json
+    import subprocess
+    import sys
+
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    env.update(env_extra)
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
+                        "--ref-rows", "16"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [line for line in r.stdout.splitlines() if line.startswith("{")]
+    return [json.loads(line) for line in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    """The oracle arm on the host: one JSON line with the contract's keys,
+    its own e2e (no transfers) and a cpu_baseline describing the run."""
+    (line,) = _run_reference({})
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOPS"
+    assert line["metric"] == bench.METRIC and line["higher_is_better"] is True and line["n_gpus"] == 1
+    assert line["config"] == bench.config_of(synth.WORKLOADS["mid_32k_d128"])
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    assert _run_reference({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
