@@ -162,3 +162,65 @@ def test_binding_layout_matches_the_library_sizes(libpath, shape, block, resid_f
         for x in sh:
             n *= x
         assert n * torch.empty((), dtype=dt).element_size() == want, (name, sh, dt, want)
+
+
+def test_shape_and_parameter_checks_of_every_entry_point(libpath):
+    """Every entry point rejects a bad shape, parameter, pointer or workspace
+    size on the host, before any CUDA call (the pointers are never used)."""
+    import bit_fp8_attention_smooth_b200 as vc
+
+    L = vc.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    prep = vc._Prep(*([fake.value] * 8))
+    big = ctypes.c_size_t(1 << 40)
+
+    def sh(B=1, H=2, N=1000, d=128):
+        return vc._Shape(B, H, N, d)
+
+    def pr(**kw):
+        base = dict(C=8, iters=2, block=128)
+        base.update(kw)
+        return vc.Params(**base).c()
+
+    def prepare(shape, params, K=fake, V=fake, p=prep, ws=fake, nbytes=big):
+        return L.vc_smooth_prepare(K, V, ctypes.byref(shape), ctypes.byref(params), ctypes.byref(p) if p else None,
+                                   ws, nbytes, None)
+
+    def attention(shape, params, O=fake, ws=fake, nbytes=big):
+        return L.vc_attention(fake, fake, fake, ctypes.byref(shape), ctypes.byref(params), ctypes.byref(prep), O,
+                              ws, nbytes, None)
+
+    INV, UNS, WS = vc.VC_ERR_INVALID_ARG, vc.VC_ERR_UNSUPPORTED, vc.VC_ERR_WORKSPACE
+    cases = [
+        (sh(d=96), pr(), UNS), (sh(), pr(block=96), UNS), (sh(), pr(block=64, resid_fmt=1), UNS),
+        (sh(N=0), pr(), INV), (sh(B=0), pr(), INV), (sh(N=(1 << 24) + 1), pr(), INV),
+        (sh(B=256, H=257), pr(), INV),
+        (sh(), pr(resid_fmt=2), INV), (sh(), pr(smooth=3), INV), (sh(), pr(smooth=-1), INV),
+        (sh(), pr(beta=71), INV), (sh(), pr(beta=-1), INV), (sh(), pr(wait_limit_ns=-1), INV),
+        (sh(), pr(C=0), INV), (sh(), pr(C=257), INV), (sh(N=7), pr(C=8), INV),
+        (sh(), pr(iters=0), INV), (sh(), pr(iters=65), INV),
+    ]
+    for shape, params, want in cases:
+        got = (prepare(shape, params), attention(shape, params))
+        assert got == (want, want), (shape.B, shape.H, shape.N, shape.d, params.C, params.iters, params.block,
+                                     params.beta, params.smooth, params.resid_fmt, got)
+    ok_shape, ok = sh(), pr()
+    assert prepare(ok_shape, ok, K=None) == INV
+    assert prepare(ok_shape, ok, V=odd) == INV
+    assert prepare(ok_shape, ok, p=None) == INV
+    assert prepare(ok_shape, ok, p=vc._Prep(*([fake.value] * 4 + [odd.value] + [fake.value] * 3))) == INV
+    assert prepare(ok_shape, ok, ws=odd) == INV
+    assert prepare(ok_shape, ok, nbytes=ctypes.c_size_t(1024)) == WS
+    assert attention(ok_shape, ok, O=None) == INV
+    assert attention(ok_shape, ok, nbytes=ctypes.c_size_t(1024)) == WS
+    # from host buffers: host pointers must be given
+    assert L.vc_attention_host(None, fake, fake, fake, ctypes.byref(ok_shape), ctypes.byref(ok), 4, fake, fake,
+                               fake, fake, ctypes.byref(prep), fake, big, None, None, None) == INV
+    # allocation-free: a problem larger than the static scratch is refused up front
+    huge = sh(H=8, N=32768)
+    assert L.vc_attn_fwd_noalloc(fake, ctypes.byref(prep), ctypes.byref(huge), ctypes.byref(ok), fake,
+                                 None) == WS
+    assert L.vc_attn_fwd_noalloc(odd, ctypes.byref(prep), ctypes.byref(ok_shape), ctypes.byref(ok), fake,
+                                 None) == INV
+    assert L.vc_check(odd, None) == INV
