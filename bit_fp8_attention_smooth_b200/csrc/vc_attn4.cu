@@ -561,12 +561,13 @@ template <int D>
 cudaError_t launch_attn4_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int BH,
                            cudaStream_t stream) {
     using Cfg = Attn4Cfg<D>;
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceOnce configured;
+    const int dev = PerDeviceOnce::current();
+    if (!configured.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(vc_attn4_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured.mark(dev);
     }
     dim3 grid((a.N + Cfg::BM - 1) / Cfg::BM, BH);
     vc_attn4_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tk, tv, a);

@@ -2,9 +2,27 @@
 // (vc_api.cu) and the kernels (vc_attn.cu, vc_prep.cu).
 #pragma once
 
+#include <atomic>
+
 #include "vc_device.cuh"
 
 namespace vc {
+
+// Kernel attributes such as the dynamic shared-memory limit belong to one
+// device: a launcher sets them once for each device it runs on (a bit per
+// device, ordinals 0..63).  Two threads may both set them the first time,
+// which is harmless.
+struct PerDeviceOnce {
+    std::atomic<uint64_t> mask{0};
+    static int current() {
+        int d = -1;
+        return cudaGetDevice(&d) == cudaSuccess ? d : -1;
+    }
+    bool done(int dev) const { return dev >= 0 && dev < 64 && ((mask.load() >> dev) & 1u); }
+    void mark(int dev) {
+        if (dev >= 0 && dev < 64) mask.fetch_or(uint64_t(1) << dev);
+    }
+};
 
 struct AttnArgs {
     const uint8_t* q_fp8;  // [BH, N, D] E4M3 Q

@@ -964,13 +964,14 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     const int64_t slots = 148LL * cps * 4;
     const int tpc = (int)imin64(16, (tiles + slots - 1) / slots);
     const int nchunk = (nblk + tpc - 1) / tpc;
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceOnce configured;
+    const int dev = PerDeviceOnce::current();
+    if (!configured.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(km_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, KM_SCAN_CHUNK * sizeof(int));
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured.mark(dev);
     }
     CUtensorMap tv, th, tl;
     if (!make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.V, D, p.N, p.BH, 64, KM_TOK) ||
@@ -1011,8 +1012,9 @@ static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
         cudaError_t e = cudaMemsetAsync(p.vamax, 0, sizeof(uint32_t) * (size_t)p.BH * D, s);
         if (e != cudaSuccess) return e;
     }
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceOnce configured;
+    const int dev = PerDeviceOnce::current();
+    if (!configured.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(prep_kv_block<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kv_block_smem<D, BK>());
         if (e != cudaSuccess) return e;
@@ -1022,7 +1024,7 @@ static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
         e = cudaFuncSetAttribute(prep_v_quant_nvfp4<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  v_quant_smem<D, BK>());
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured.mark(dev);
     }
     prep_kv_block<D, BK><<<dim3(T, p.BH), PREP_THREADS, kv_block_smem<D, BK>(), s>>>(
         p.K, p.V, p.perm, p.smooth, p.k_fp8, p.k_scale, p.v_mean, p.vamax, p.N, T, p.ctl.status);
