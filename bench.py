@@ -232,6 +232,30 @@ def config_of(w):
             "l2": f"inputs {3 * w.B * w.H * w.N * w.d * 2 / 1e9:.2f} GB per step > 126 MB L2 (no flush needed)"}
 
 
+def prep_roofline(w, prep_ms: float, peaks) -> dict:
+    """The V-Smooth prep against its floor.  Compulsory bytes per head: K and
+    V read as bf16 (4Nd); the quantised K (Tp d) and V residual (Tp d, or half
+    plus the 16-token block scales on the 4-bit path) written; perm (4N),
+    block means (4Td), K block scales (4T) and channel scales (4d).  Flops: the
+    k-means assignment, 2 N C d per pass.  The floor is the slower of the
+    bytes at the HBM copy rate and the flops at the bf16 tensor rate."""
+    T = -(-w.N // w.block)
+    Tp = T * w.block
+    fp4 = resid_fmt_of(w) == 1
+    resid = Tp * w.d // 2 + T * w.d * (w.block // 16) if fp4 else Tp * w.d
+    per_head = 4 * w.N * w.d + Tp * w.d + resid + 4 * w.N + 4 * T * w.d + 4 * T + 4 * w.d
+    nbytes = per_head * w.B * w.H
+    flops = 2.0 * w.N * w.C * w.d * w.iters * w.B * w.H
+    tensor = peaks.get("bf16_sustained") or peaks["bf16"]
+    t_bytes = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_flops = flops / (tensor * 1e12)
+    floor_s = max(t_bytes, t_flops)
+    t = prep_ms * 1e-3
+    return {"bound": "hbm" if t_bytes >= t_flops else "tensor", "bytes": nbytes, "flops": flops,
+            "achieved_gbs": nbytes / t / 1e9, "peak_gbs": peaks["hbm_gbs"], "peak_bf16_tflops": tensor,
+            "floor_ms": floor_s * 1e3, "frac": floor_s / t}
+
+
 def launches_per_step(p) -> int:
     """Kernels of the library one step launches (the launch list in profiles/
     shows the same sequence): km_init; per k-means pass km_assign, km_refine,
@@ -378,6 +402,7 @@ def run_ours(args, w):
             "config": dict(config_of(full), **({"heads_per_rank": w.H} if args.split_heads else {}),
                            **({"tile_density": density} if tile_mask is not None else {})),
             "attn_ms": attn_ms, "prep_ms": prep_ms, "prep_reuse_ms": prep_reuse_ms, "attn_tflops": attn_tflops,
+            "prep_roofline": prep_roofline(w, prep_ms, peaks),
             "frac_of_nominal_fp8_4500": value / 4500.0, "attn_frac_of_nominal_fp8_4500": attn_tflops / 4500.0,
             "roofline": {
                 "bound": "tensor", "kernel": kernel,

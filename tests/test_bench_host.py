@@ -162,3 +162,27 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_other_ranks_do_no_work():
     assert _run_reference({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_prep_roofline_against_the_workload_arithmetic():
+    """The compulsory prep bytes and k-means flops of the 40-head 32K
+    workload: 25.43 MB and 5.37 GFLOP a head (1.017 GB and 215 GFLOP in all).
+    At the measured peaks the two floors nearly coincide (about 0.156 ms)."""
+    w = synth.WORKLOADS["mid_32k_d128"]
+    peaks = dict(hbm_gbs=6538.0, bf16=1606.0, bf16_sustained=1384.2)
+    r = bench.prep_roofline(w, 3.45, peaks)
+    per_head = 4 * 32768 * 128 + 2 * 32768 * 128 + 4 * 32768 + 4 * 256 * 128 + 4 * 256 + 4 * 128
+    assert r["bytes"] == 40 * per_head and abs(r["bytes"] / 1e9 - 1.017) < 0.001
+    assert r["flops"] == 2.0 * 32768 * 64 * 128 * 10 * 40 and abs(r["flops"] / 1e9 - 214.7) < 0.1
+    t_bytes, t_flops = r["bytes"] / 6538e9, r["flops"] / 1384.2e12
+    assert r["floor_ms"] == pytest.approx(max(t_bytes, t_flops) * 1e3)
+    assert r["frac"] == pytest.approx(r["floor_ms"] / 3.45) and 0 < r["frac"] < 1
+    assert r["achieved_gbs"] == pytest.approx(r["bytes"] / 3.45e-3 / 1e9)
+    # the 4-bit workload writes half the residual bytes plus one scale byte per 16
+    w4 = synth.WORKLOADS["nvfp4_32k_d128"]
+    r4 = bench.prep_roofline(w4, 2.0, peaks)
+    per_head4 = per_head - 32768 * 128 // 2 + 256 * 128 * 8
+    assert r4["bytes"] == 24 * per_head4
+    # without a sustained figure the burst one is used
+    assert bench.prep_roofline(w, 3.45, dict(hbm_gbs=6538.0, bf16=1606.0, bf16_sustained=None))["peak_bf16_tflops"] \
+        == 1606.0
