@@ -2,7 +2,6 @@
 quantisation) against library routines (scipy, scikit-learn, numpy, torch),
 Lloyd's invariants and closed forms."""
 import numpy as np
-import pytest
 import torch
 
 import oracle
