@@ -224,3 +224,40 @@ def test_shape_and_parameter_checks_of_every_entry_point(libpath):
     assert L.vc_attn_fwd_noalloc(odd, ctypes.byref(prep), ctypes.byref(ok_shape), ctypes.byref(ok), fake,
                                  None) == INV
     assert L.vc_check(odd, None) == INV
+
+
+def test_header_is_plain_c_and_a_c_program_links_the_library(libpath, tmp_path):
+    """include/vc_attention.h compiles as strict C99 and as C++17, and a plain
+    C program links libvcattn.so and answers the host queries (no torch, no
+    Python): the boundary is usable from C."""
+    inc = os.path.join(ROOT, "include")
+    hdr = os.path.join(inc, "vc_attention.h")
+    for cmd in (["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-x", "c", hdr],
+                ["g++", "-std=c++17", "-Wall", "-Werror", "-fsyntax-only", "-x", "c++", hdr]):
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+    prog = tmp_path / "abi.c"
+    prog.write_text(r"""
+#include <stdio.h>
+#include "vc_attention.h"
+int main(void) {
+    vc_shape s = {1, 40, 32768, 128};
+    vc_params p = {64, 10, 128, 64, 1, 0, 0};
+    size_t b[8], ws = 0;
+    if (vc_abi_version() != VC_ABI_VERSION) return 1;
+    if (vc_prep_buffer_bytes(&s, &p, b) != VC_OK || vc_workspace_bytes(&s, &p, &ws) != VC_OK) return 2;
+    p.block = 96;
+    if (vc_prep_buffer_bytes(&s, &p, b) != VC_ERR_UNSUPPORTED) return 3;
+    printf("%zu %zu %s\n", b[2], ws, vc_status_string(VC_ERR_WORKSPACE));
+    return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(libpath)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(prog), "-o", str(exe), "-L", libdir,
+                        "-lvcattn", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    k_bytes, ws, msg = r.stdout.split(maxsplit=2)
+    assert int(k_bytes) == 40 * 32768 * 128 and int(ws) > 0 and msg.strip()
