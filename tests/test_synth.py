@@ -48,3 +48,23 @@ def test_grid_patches_share_a_centroid():
         rows = v[ids == p]
         med = np.median(rows, axis=0)
         assert np.median(np.abs(rows - med)) < 0.5
+
+
+def test_generator_holds_no_method_arithmetic():
+    """Both the oracle and the CUDA path are fed from synth.py, so it must not
+    load either of them or compute any step of the method: it imports only
+    numpy, torch and the standard library, and calls no quantiser, ExpCast,
+    k-means or library routine."""
+    import ast
+    import os
+
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "bit_fp8_attention_smooth_b200", "synth.py"), encoding="utf-8").read()
+    tree = ast.parse(src)
+    mods = {a.name.split(".")[0] for n in ast.walk(tree) if isinstance(n, ast.Import) for a in n.names}
+    mods |= {(n.module or "").split(".")[0] for n in ast.walk(tree) if isinstance(n, ast.ImportFrom)}
+    assert mods <= {"__future__", "dataclasses", "typing", "numpy", "torch"}, mods
+    calls = {n.func.attr if isinstance(n.func, ast.Attribute) else getattr(n.func, "id", "")
+             for n in ast.walk(tree) if isinstance(n, ast.Call)}
+    banned = {c for c in calls if any(w in c.lower() for w in ("e4m3", "e2m1", "expcast", "kmeans", "quant", "lib"))}
+    assert not banned, banned
