@@ -65,22 +65,20 @@ def kernel_code_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def attn_traffic_bytes(heads: int):
+def attn_traffic_bytes(heads: int, kernel: str = "vc_attn_kernel"):
     """DRAM bytes (read + write) of one attention-kernel launch over `heads`
-    heads, from the ncu capture summarised in profiles/; None when the kernel
-    code has changed since that capture (its counters no longer apply)."""
-    import re
-
-    prof = os.path.join(ROOT, "profiles", "vc_attn_kernel_mid_32k_h8.md")
+    heads, from the ncu capture recorded in profiles/attn_traffic.json; None
+    when there is no record for the kernel or its code has changed since the
+    capture (the counters no longer apply)."""
     try:
-        text = open(prof).read()
+        with open(os.path.join(ROOT, "profiles", "attn_traffic.json")) as f:
+            rec = json.load(f).get(kernel)
         code = kernel_code_hash()
-    except OSError:
+    except (OSError, ValueError):
         return None
-    m = re.search(r"roofline-traffic: kernel=\S+ sources_sha256_16=([0-9a-f]{16}) dram_bytes_per_head=(\d+)", text)
-    if not m or m.group(1) != code:
+    if not rec or rec.get("sources_sha256_16") != code:
         return None
-    return int(m.group(2)) * heads
+    return int(rec["dram_bytes_per_head"]) * heads
 
 
 # ----------------------------------------------------------------- distributed
@@ -166,7 +164,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- CPU oracle
-def oracle_sample(w, rows: int, threads: int):
+def oracle_sample(w, rows: int, threads: int, smooth: bool = True):
     """Time the oracle (prep of one head + replay of `rows` query rows over all
     keys) and extrapolate to the per-head attention throughput in TFLOPS."""
     import oracle
@@ -175,14 +173,27 @@ def oracle_sample(w, rows: int, threads: int):
     sel = np.linspace(0, w.N - 1, rows).astype(np.int64)
     t0 = time.perf_counter()
     rf = resid_fmt_of(w)
-    prep = oracle.prep_head(k, v, C=w.C, iters=w.iters, bk=w.block, resid_fmt=rf)
+    prep = oracle.prep_head(k, v, C=w.C, iters=w.iters, bk=w.block, smooth=smooth, resid_fmt=rf)
     t1 = time.perf_counter()
-    oracle.forward_head(q, k, v, sel, C=w.C, iters=w.iters, bk=w.block, beta=BETA, resid_fmt=rf, prep=prep,
-                        threads=threads)
+    oracle.forward_head(q, k, v, sel, C=w.C, iters=w.iters, bk=w.block, beta=BETA, smooth=smooth, resid_fmt=rf,
+                        prep=prep, threads=threads)
     t2 = time.perf_counter()
     head_s = (t1 - t0) + (t2 - t1) * (w.N / rows)
     head_flops = 4.0 * float(w.N) ** 2 * w.d
     return dict(value=head_flops / head_s / 1e12, prep_s=t1 - t0, rows_s=t2 - t1, head_s=head_s)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
 
 
 def cpu_cores() -> int:
@@ -194,27 +205,39 @@ def cpu_cores() -> int:
 
 # ----------------------------------------------------------------- arms
 def run_reference(args, w):
+    """The oracle as it stands, timed on the host cores.  One step is one
+    bounded sample of the workload: the full prep of head 0 plus the replay of
+    `--ref-rows` strided query rows over all keys.  ms_per_step is the measured
+    time of that sample; value is the workload's attention flops over the time
+    the sample extrapolates to (the head's prep plus all its rows, times the
+    heads)."""
     world, rank, _ = dist_env()
     if rank != 0:
         return
     cores = cpu_cores()
     rows = args.ref_rows
     for _ in range(args.warmup):
-        oracle_sample(w, max(8, rows // 8), cores)
-    vals, secs = [], []
+        oracle_sample(w, max(8, rows // 8), cores, args.smooth)
+    samples = []
+    t0 = time.perf_counter()
     for _ in range(args.steps):
-        r = oracle_sample(w, rows, cores)
-        vals.append(r["value"])
-        secs.append(r["head_s"])
-    value = statistics.median(vals)
+        samples.append(oracle_sample(w, rows, cores, args.smooth))
+    wall = time.perf_counter() - t0
+    head_s = statistics.median(r["head_s"] for r in samples)
+    full_s = head_s * w.B * w.H
+    value = w.attn_flops / full_s / 1e12
     sample = (f"head 0 of {w.name}: full k-means/regroup/quantise prep + replay of {rows} strided query rows "
-              f"over all {w.N} keys, extrapolated to the head's {w.N} rows")
+              f"over all {w.N} keys; value extrapolates to all {w.N} rows of each of the {w.B * w.H} heads")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(secs) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 emulation of e4m3",
-        "data": "synthetic", "config": config_of(w),
-        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
+        "data": "synthetic", "config": config_of(w, args.smooth),
+        "sample_s": {"prep": statistics.median(r["prep_s"] for r in samples),
+                     "rows": statistics.median(r["rows_s"] for r in samples)},
+        "extrapolated_head_s": head_s, "extrapolated_step_s": full_s,
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "cpu_model": cpu_model(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -225,14 +248,21 @@ def resid_fmt_of(w) -> int:
     return 1 if w.resid_fmt == "nvfp4" else 0
 
 
-def config_of(w):
+def config_of(w, smooth: bool):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "C": w.C, "kmeans_iters": w.iters,
-            "block": w.block, "beta": BETA, "v_smooth": True,
+            "block": w.block, "beta": BETA, "v_smooth": smooth,
             "residual": "nvfp4 (E2M1 + UE4M3 per 16)" if resid_fmt_of(w) else "e4m3",
-            "l2": f"inputs {3 * w.B * w.H * w.N * w.d * 2 / 1e9:.2f} GB per step > 126 MB L2 (no flush needed)"}
+            "l2": l2_note(w)}
 
 
-def prep_roofline(w, prep_ms: float, peaks) -> dict:
+def l2_note(w) -> str:
+    gb = 3 * w.B * w.H * w.N * w.d * 2 / 1e9
+    if gb > 0.126:
+        return f"inputs {gb:.2f} GB per step > 126 MB L2 (no flush needed)"
+    return f"inputs {gb * 1e3:.1f} MB per step fit in the 126 MB L2 (a parity-size case, not a throughput workload)"
+
+
+def prep_roofline(w, prep_ms: float, peaks, timed_s: float) -> dict:
     """The V-Smooth prep against its floor.  Compulsory bytes per head: K and
     V read as bf16 (4Nd); the quantised K (Tp d) and V residual (Tp d, or half
     plus the 16-token block scales on the 4-bit path) written; perm (4N),
@@ -246,7 +276,7 @@ def prep_roofline(w, prep_ms: float, peaks) -> dict:
     per_head = 4 * w.N * w.d + Tp * w.d + resid + 4 * w.N + 4 * T * w.d + 4 * T + 4 * w.d
     nbytes = per_head * w.B * w.H
     flops = 2.0 * w.N * w.C * w.d * w.iters * w.B * w.H
-    tensor = peaks.get("bf16_sustained") or peaks["bf16"]
+    tensor, _ = tensor_peak(peaks, timed_s)
     t_bytes = nbytes / (peaks["hbm_gbs"] * 1e9)
     t_flops = flops / (tensor * 1e12)
     floor_s = max(t_bytes, t_flops)
@@ -270,6 +300,41 @@ def launches_per_step(p) -> int:
     return prep + 2
 
 
+def accuracy_vs_exact(q, k, v, out, heads, rows: int = 64) -> dict:
+    """Error of the output against exact attention softmax(q k^T / sqrt(d)) v
+    on the bf16 inputs, computed in fp64 with torch on sampled query rows of
+    the given heads (the benchmark spec's rel-L2 and PSNR, plus cosine)."""
+    B, H, N, d = q.shape
+    sel = torch.unique(torch.cat([torch.linspace(0, N - 1, rows).long(), torch.tensor([N - 1])])).to(q.device)
+    num, den, dot, nrm_o, peak, sq, cnt = 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0
+    for h in heads:
+        qh = q[0, h, sel].double()
+        kh, vh = k[0, h].double(), v[0, h].double()
+        ref = torch.softmax(qh @ kh.T / d ** 0.5, dim=-1) @ vh
+        got = out[0, h, sel].double()
+        e = got - ref
+        num += float((e * e).sum())
+        den += float((ref * ref).sum())
+        dot += float((got * ref).sum())
+        nrm_o += float((got * got).sum())
+        peak = max(peak, float(ref.abs().max()))
+        sq += float((e * e).sum())
+        cnt += e.numel()
+    rmse = (sq / cnt) ** 0.5
+    return {"vs": "exact softmax attention on the bf16 inputs (fp64)", "heads": list(heads), "rows_per_head": len(sel),
+            "rel_l2": (num / den) ** 0.5, "cos": dot / (den * nrm_o) ** 0.5,
+            "psnr_db": 20.0 * float(np.log10(peak / rmse)) if rmse > 0 else float("inf")}
+
+
+def tensor_peak(peaks, timed_s: float):
+    """The measured bf16 tensor rate that applies to a kernel timed inside a
+    region of timed_s seconds: the burst figure for a short region (the clocks
+    stay near max), the power-capped sustained one for a region of seconds."""
+    if timed_s < 2.0 or not peaks.get("bf16_sustained"):
+        return peaks["bf16"], "burst"
+    return peaks["bf16_sustained"], "sustained"
+
+
 def run_ours(args, w):
     import bit_fp8_attention_smooth_b200 as vc
 
@@ -289,7 +354,7 @@ def run_ours(args, w):
             raise SystemExit(f"--split-heads needs at most {w.H} ranks")
         h0, h1 = vc.head_range(rank, world, w.H)
         w = dataclasses.replace(w, H=h1 - h0)
-    params = vc.Params.for_workload(w, beta=BETA)
+    params = vc.Params.for_workload(w, beta=BETA, smooth=int(args.smooth))
     shape = (w.B, w.H, w.N, w.d)
 
     # inputs resident in HBM (pinned host copies kept for the end-to-end leg)
@@ -380,37 +445,46 @@ def run_ours(args, w):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     e2e.check()
+    # error against exact attention on sampled rows of the first and last head
+    acc = accuracy_vs_exact(qd, kd, vd, out, sorted({0, w.H - 1})) if rank == 0 and tile_mask is None else None
 
     if rank == 0:
         peaks = load_peaks()
-        fp8_peak = peaks["bf16_sustained"] * FP8_PER_BF16
+        timed_s = total_ms * 1e-3
+        bf16, which = tensor_peak(peaks, timed_s)
+        fp8_peak = bf16 * FP8_PER_BF16
         four_bit = resid_fmt_of(w) == 1
         if four_bit:
             # QK^T (half the flops) at the FP8 rate, PV (the other half) at the
             # FP4 rate, twice FP8: the time at peak is 3/4 of the all-FP8 time
-            peak, kernel = fp8_peak * 4.0 / 3.0, "vc_attn_fwd (Q quantise + vc_attn4_kernel)"
-            peak_src = (f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16) for QK^T, "
-                        f"x 4 (fp4:bf16) for PV; harmonic over the two halves")
+            peak, kernel = fp8_peak * 4.0 / 3.0, "vc_attn_fwd (vc_attn4_kernel)"
+            nominal = 4500.0 * 4.0 / 3.0
+            peak_src = (f"{peaks['source']} bf16 {which} {bf16} TFLOP/s x 2 (fp8:bf16) for QK^T, x 4 (fp4:bf16) "
+                        f"for PV; harmonic over the two halves")
         else:
-            peak, kernel = fp8_peak, "vc_attn_fwd (Q quantise + vc_attn_kernel)"
-            peak_src = f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x 2 (fp8:bf16)"
+            peak, kernel, nominal = fp8_peak, "vc_attn_fwd (vc_attn_kernel)", 4500.0
+            peak_src = f"{peaks['source']} bf16 {which} {bf16} TFLOP/s x 2 (fp8:bf16)"
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if args.split_heads else "weak",
             "vs_baseline": None, "dtype": "e4m3+e2m1" if four_bit else "e4m3", "data": "synthetic",
-            "config": dict(config_of(full), **({"heads_per_rank": w.H} if args.split_heads else {}),
+            "config": dict(config_of(full, bool(args.smooth)),
+                           **({"heads_per_rank": w.H} if args.split_heads else {}),
                            **({"tile_density": density} if tile_mask is not None else {})),
             "attn_ms": attn_ms, "prep_ms": prep_ms, "prep_reuse_ms": prep_reuse_ms, "attn_tflops": attn_tflops,
-            "prep_roofline": prep_roofline(w, prep_ms, peaks),
-            "frac_of_nominal_fp8_4500": value / 4500.0, "attn_frac_of_nominal_fp8_4500": attn_tflops / 4500.0,
+            "prep_roofline": prep_roofline(w, prep_ms, peaks, timed_s) if args.smooth else None,
+            "frac_of_nominal_fp8_4500": value / 4500.0,
             "roofline": {
                 "bound": "tensor", "kernel": kernel,
                 "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                "peak_source": peak_src,
-                "traffic": None if four_bit or tile_mask is not None else attn_traffic_bytes(w.B * w.H),
-                "traffic_unit": "bytes per launch (ncu capture on 8 heads, scaled by heads)",
+                "peak_source": peak_src, "timed_region_s": timed_s,
+                "frac_of_nominal": attn_tflops / nominal, "nominal_peak": nominal,
+                "traffic": None if tile_mask is not None else attn_traffic_bytes(
+                    w.B * w.H, "vc_attn4_kernel" if four_bit else "vc_attn_kernel"),
+                "traffic_unit": "DRAM bytes per launch (ncu capture on fewer heads, scaled by heads)",
             },
+            "accuracy": acc,
             "e2e": {"value": dense_job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": e2e.h2d_bytes, "d2h_bytes_per_step": e2e.d2h_bytes},
             "gpu_launches": launches_per_step(params) * args.steps,
@@ -418,9 +492,10 @@ def run_ours(args, w):
         }
         if world == 1 and not args.no_cpu_baseline:
             cores = cpu_cores()
-            r = oracle_sample(w, args.ref_rows, cores)
+            r = oracle_sample(w, args.ref_rows, cores, bool(args.smooth))
             line["cpu_baseline"] = {
-                "value": r["value"], "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                "value": r["value"], "unit": "TFLOPS", "cores": cores,
+                "cpu_model": cpu_model(), "kind": "oracle",
                 "sample": (f"head 0: full prep ({r['prep_s']:.1f} s) + {args.ref_rows} strided query rows over all "
                            f"keys ({r['rows_s']:.1f} s), extrapolated to the head's {w.N} rows"),
             }
@@ -440,6 +515,8 @@ def main():
     ap.add_argument("--workload", default="mid_32k_d128", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--smooth", choices=["on", "off"], default="on",
+                    help="V-Smooth on (k-means regroup, block means) or off (plain per-channel FP8 V)")
     ap.add_argument("--tile-density", type=float, default=1.0,
                     help="block-sparse attention: the share of key tiles each query tile keeps (seeded random mask; "
                          "flops count the kept tiles only)")
@@ -449,6 +526,7 @@ def main():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads of the workload (profiling captures on a smaller case)")
     args = ap.parse_args()
+    args.smooth = args.smooth == "on"
     w = synth.WORKLOADS[args.workload]
     if args.heads:
         w = dataclasses.replace(w, name=f"{w.name}_h{args.heads}", H=args.heads)

@@ -51,6 +51,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
     cmd = [
         nvcc(), "-shared", "-Xcompiler", "-fPIC", "-std=c++17", "-O3", "-lineinfo",
         "-gencode", "arch=compute_100a,code=sm_100a",
+        # IEEE fp32 throughout: the ExpCast byte map reads a rounded integer
+        # out of an fp32 subnormal, so denormals must not be flushed; divisions
+        # and square roots are the correctly rounded ones the quantisers use.
+        # (--use_fast_math would turn all three off, so it is never passed.)
+        "--ftz=false", "--prec-div=true", "--prec-sqrt=true",
         "--expt-relaxed-constexpr", "-Xptxas", "-v" if verbose else "-O3",
         "-I", INCLUDE, "-I", CSRC,
         "-o", tmp, *sources(),

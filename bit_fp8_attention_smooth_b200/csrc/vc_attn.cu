@@ -339,6 +339,14 @@ __global__ void __launch_bounds__(320, 1)
                     const float* sp = s + 64 * c + 4 * q;
                     pw[q] = expcast4(A, sp[0], sp[1], sp[2], sp[3], cbm);
                 }
+                if (valid < BK) {
+                    // Keys past N carry no weight.  Their scores are -inf, which
+                    // codes to 0 only while A > 0: with A = 0 (a zero Q row or
+                    // an all-zero K block) the FMA gives 0 * -inf = NaN, so the
+                    // bytes are cleared here instead.
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) pw[q] &= tail_keep_mask(valid - (64 * c + 4 * q));
+                }
                 tmem_st16(pcol + 16 * c, pw);
             }
             if (t > 0 && __any_sync(0xffffffffu, kinc > 0)) {
@@ -482,15 +490,16 @@ template <int D, int BK>
 cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int BH,
                           cudaStream_t stream) {
     using Cfg = AttnCfg<D, BK>;
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceOnce configured;
+    const int dev = PerDeviceOnce::current();
+    if (!configured.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(vc_attn_kernel<D, BK, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(vc_attn_kernel<D, BK, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured.mark(dev);
     }
     dim3 grid((a.N + Cfg::BM - 1) / Cfg::BM, BH);
     if (a.tile_mask)
@@ -521,7 +530,8 @@ __global__ void vc_expcast_kernel(const float* A, const float* s, const float* c
 cudaError_t launch_expcast(const float* A, const float* s, const float* cb, uint8_t* out, int64_t n,
                            cudaStream_t stream) {
     if (n == 0) return cudaSuccess;
-    const unsigned grid = (unsigned)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
+    const int64_t cap = 16LL * sm_count();
+    const unsigned grid = (unsigned)((n + 255) / 256 < cap ? (n + 255) / 256 : cap);
     vc_expcast_kernel<<<grid, 256, 0, stream>>>(A, s, cb, out, n);
     return cudaGetLastError();
 }

@@ -436,4 +436,11 @@ __device__ __forceinline__ uint32_t expcast4(float A, float s0, float s1, float 
     return pack2_sat_u8(__float_as_int(w01.y), __float_as_int(w01.x), hi);
 }
 
+// Mask of the bytes of a word of four codes that belong to keys inside the
+// sequence: `left` keys remain from the word's first key on (<= 0: none, >= 4:
+// all four, else the low `left` bytes).
+__device__ __forceinline__ uint32_t tail_keep_mask(int left) {
+    return left >= 4 ? 0xFFFFFFFFu : (left <= 0 ? 0u : (1u << (8 * left)) - 1u);
+}
+
 }  // namespace vc

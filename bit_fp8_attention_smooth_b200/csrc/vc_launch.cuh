@@ -24,6 +24,20 @@ struct PerDeviceOnce {
     }
 };
 
+// Streaming multiprocessors of the current device, queried once per device
+// (grid sizes of the grid-stride kernels scale with it).
+inline int sm_count() {
+    static std::atomic<int> cache[64];
+    const int dev = PerDeviceOnce::current();
+    if (dev < 0 || dev >= 64) return 148;
+    int n = cache[dev].load();
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev].store(n);
+    }
+    return n;
+}
+
 struct AttnArgs {
     const uint8_t* q_fp8;  // [BH, N, D] E4M3 Q
     const float* sq;       // [BH, N] per-token Q scale

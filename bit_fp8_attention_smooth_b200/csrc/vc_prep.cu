@@ -959,9 +959,10 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     while (cps > 1 && ((size_t)cps * lay.bytes > 227 * 1024 || cps * ncols > 512)) --cps;
     const size_t smem = lay.bytes > (size_t)(228 * 1024 / (cps + 1) + 1024) ? lay.bytes
                                                                              : (size_t)(228 * 1024 / (cps + 1) + 1024);
-    // Tiles per CTA: about four waves of CTAs over the 148 SMs.
+    // Tiles per CTA: about four waves of CTAs over the SMs.
+    const int sms = sm_count();
     const int64_t tiles = (int64_t)nblk * p.BH;
-    const int64_t slots = 148LL * cps * 4;
+    const int64_t slots = (int64_t)sms * cps * 4;
     const int tpc = (int)imin64(16, (tiles + slots - 1) / slots);
     const int nchunk = (nblk + tpc - 1) / tpc;
     static PerDeviceOnce configured;
@@ -984,7 +985,7 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
         km_assign<D><<<dim3(nchunk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.vnorm2, p.labels,
                                                             p.hist, p.ties, p.tie_count, p.state, p.N, p.C, Cp,
                                                             it, tpc, p.ctl);
-        km_refine<D><<<148 * 8, 256, 0, s>>>(p.ties, p.tie_count, p.V, p.cent64, p.labels, p.hist, p.state, p.N,
+        km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, p.V, p.cent64, p.labels, p.hist, p.state, p.N,
                                               p.C, Cp, it, p.ctl.status);
         km_scan<<<p.BH, 1024, KM_SCAN_CHUNK * sizeof(int), s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it,
                                       p.ctl.status);
@@ -1006,7 +1007,7 @@ static cudaError_t blocks_t(const PrepLaunch& p, cudaStream_t s) {
     if (p.smooth != 1) {  // no k-means this call: the channel maxima start from zero here
         if (p.smooth == 0) {  // plain per-channel FP8 V: identity order
             const int64_t total = (int64_t)p.BH * p.N;
-            identity_order<<<(unsigned)imin64((total + 255) / 256, 148 * 32), 256, 0, s>>>(p.perm, p.labels,
+            identity_order<<<(unsigned)imin64((total + 255) / 256, 32LL * sm_count()), 256, 0, s>>>(p.perm, p.labels,
                                                                                                  total, p.N);
         }  // smooth == 2: the regroup already in perm is kept
         cudaError_t e = cudaMemsetAsync(p.vamax, 0, sizeof(uint32_t) * (size_t)p.BH * D, s);
@@ -1064,7 +1065,7 @@ cudaError_t launch_quant_q(const __nv_bfloat16* Q, uint8_t* q_fp8, float* sq, in
 
 cudaError_t launch_e4m3_encode(const float* x, uint8_t* out, int64_t n, cudaStream_t s) {
     if (n == 0) return cudaSuccess;
-    const unsigned grid = (unsigned)imin64((n + 255) / 256, 148 * 16);
+    const unsigned grid = (unsigned)imin64((n + 255) / 256, 16LL * sm_count());
     e4m3_encode_kernel<<<grid, 256, 0, s>>>(x, out, n);
     return cudaGetLastError();
 }

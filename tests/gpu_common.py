@@ -79,6 +79,47 @@ def oracle_prep_to_gpu(preps, shape, bk, device="cuda"):
     return out
 
 
+def oracle_prep_on_perm(k_bits, v_bits, perm, bk, smooth=True, resid_fmt=0):
+    """The oracle's quantisers (K, V-Smooth residual) applied in a given
+    regroup order -- the GPU's own, so that byte parity of the quantisers does
+    not hinge on the two k-means agreeing on every near tie."""
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    khat, ksc = oracle.quant_k(k_bits, perm, bk)
+    if resid_fmt == 1:
+        vq, vgs, vmu, vsc = oracle.smooth_v_nvfp4(v_bits, perm, bk, smooth)
+        return dict(perm=perm, khat=khat, ksc=ksc, vq=vq, vgs=vgs, vmu=vmu, vsc=vsc)
+    vhat, vmu, vsc = oracle.smooth_v(v_bits, perm, bk, smooth)
+    return dict(perm=perm, khat=khat, ksc=ksc, vhat=vhat, vmu=vmu, vsc=vsc)
+
+
+# k-means decisions the tensor-core distance leaves open are re-decided in
+# fp64 when two clusters lie within this fraction of (|v| + max|c|)^2.
+KMEANS_MARGIN = 2.0 ** -12
+
+
+def check_labels_valid(v_bits, gpu_labels, ref_labels, centroids):
+    """Where the GPU's k-means label differs from the oracle's, the GPU's
+    cluster must still be a valid argmin: its fp64 squared distance (to the
+    oracle's final centroids) lies within the near-tie margin of the minimum."""
+    diff = np.nonzero(np.asarray(gpu_labels) != np.asarray(ref_labels))[0]
+    if diff.size == 0:
+        return 0
+    v = bits_to_f64(v_bits[diff])
+    c = np.asarray(centroids, dtype=np.float64)
+    d2 = ((v[:, None, :] - c[None, :, :]) ** 2).sum(-1)
+    got = d2[np.arange(diff.size), np.asarray(gpu_labels)[diff]]
+    rad = np.linalg.norm(v, axis=1) + np.linalg.norm(c, axis=1).max()
+    excess = got - d2.min(1)
+    assert np.all(excess <= KMEANS_MARGIN * rad ** 2), (diff[:5], excess[:5], (KMEANS_MARGIN * rad ** 2)[:5])
+    return int(diff.size)
+
+
+def bits_to_f64(b: np.ndarray) -> np.ndarray:
+    """uint16 bf16 bit patterns -> float64 values (test helper)."""
+    u = np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
 def check_perm(perm: np.ndarray, labels: np.ndarray, n: int):
     """perm is a bijection, labels[perm] is non-decreasing, and stable."""
     assert np.array_equal(np.sort(perm), np.arange(n))

@@ -1,7 +1,8 @@
 """Host logic of bench.py, on the CPU: the launch count it claims, the traffic
-figure it takes from the committed ncu summary (and drops once the kernel
-code changes), the peak denominators, the clock-sample parser that decides
-whether a run is kept, and the oracle arm (`--impl reference`) end to end."""
+figure it takes from the committed ncu record (and drops once the kernel code
+changes), the peak denominators, the clock-sample parser that decides whether
+a run is kept, and the oracle arm (`--impl reference`) end to end."""
+import json
 import os
 import re
 import shutil
@@ -13,15 +14,6 @@ import bit_fp8_attention_smooth_b200 as vc
 from bit_fp8_attention_smooth_b200 import synth
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-
-
-def test_launches_per_step_matches_the_launch_list():
-    """The committed launch list records one timed step of the 32K workload
-    as a fixed number of launches (its -c); the bench claims the same."""
-    text = open(os.path.join(ROOT, "profiles", "launch_list_mid_32k_d128.md")).read()
-    count = int(re.search(r"-c (\d+)", text).group(1))
-    p = vc.Params.for_workload(synth.WORKLOADS["mid_32k_d128"], beta=64)
-    assert bench.launches_per_step(p) == count
 
 
 @pytest.mark.parametrize("iters", [1, 2, 10])
@@ -44,10 +36,9 @@ def _fake_root(tmp_path, per_head=1000):
     return csrc
 
 
-def _write_profile(tmp_path, code_hash, per_head):
-    (tmp_path / "profiles" / "vc_attn_kernel_mid_32k_h8.md").write_text(
-        "summary\n\n    roofline-traffic: kernel=vc_attn_kernel<128,128,false> "
-        f"sources_sha256_16={code_hash} dram_bytes_per_head={per_head}\n")
+def _write_profile(tmp_path, code_hash, per_head, kernel="vc_attn_kernel"):
+    (tmp_path / "profiles" / "attn_traffic.json").write_text(json.dumps(
+        {kernel: {"sources_sha256_16": code_hash, "dram_bytes_per_head": per_head}}))
 
 
 def test_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
@@ -72,16 +63,25 @@ def test_traffic_without_a_profile_is_null(tmp_path, monkeypatch):
     _fake_root(tmp_path)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.attn_traffic_bytes(40) is None
-    (tmp_path / "profiles" / "vc_attn_kernel_mid_32k_h8.md").write_text("no traffic line here\n")
+    (tmp_path / "profiles" / "attn_traffic.json").write_text("{}")
     assert bench.attn_traffic_bytes(40) is None
+    (tmp_path / "profiles" / "attn_traffic.json").write_text("not json")
+    assert bench.attn_traffic_bytes(40) is None
+    # a record of another kernel does not apply
+    _write_profile(tmp_path, bench.kernel_code_hash(), 99, kernel="vc_attn4_kernel")
+    assert bench.attn_traffic_bytes(40) is None
+    assert bench.attn_traffic_bytes(40, "vc_attn4_kernel") == 99 * 40
 
 
-def test_committed_traffic_line_is_well_formed():
-    text = open(os.path.join(ROOT, "profiles", "vc_attn_kernel_mid_32k_h8.md")).read()
-    m = re.search(r"roofline-traffic: kernel=\S+ sources_sha256_16=([0-9a-f]{16}) dram_bytes_per_head=(\d+)", text)
-    assert m
-    # at least the fp8 Q, K and V of one 32K x 128 head are read
-    assert int(m.group(2)) >= 3 * 32768 * 128
+def test_committed_traffic_records_are_well_formed():
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(path):
+        pytest.skip("no traffic record committed")
+    recs = json.load(open(path))
+    for kernel, rec in recs.items():
+        assert re.fullmatch(r"[0-9a-f]{16}", rec["sources_sha256_16"]), kernel
+        # at least the fp8 Q and K and the V residual of one head are read
+        assert int(rec["dram_bytes_per_head"]) >= 2 * 32768 * 128, kernel
 
 
 def test_peaks_measured_and_fallback(tmp_path, monkeypatch):
@@ -125,12 +125,15 @@ def test_clock_summary_without_samples_is_null():
 
 def test_config_names_the_workload_and_its_l2_rule():
     w = synth.WORKLOADS["mid_32k_d128"]
-    c = bench.config_of(w)
+    c = bench.config_of(w, True)
+    assert c["v_smooth"] is True and bench.config_of(w, False)["v_smooth"] is False
     assert c["workload"] == w.name and (c["B"], c["H"], c["N"], c["d"]) == (w.B, w.H, w.N, w.d)
     assert c["residual"] == "e4m3"
     gb = float(re.search(r"inputs ([0-9.]+) GB", c["l2"]).group(1))
     assert gb * 1e9 > 126e6
-    assert bench.config_of(synth.WORKLOADS["nvfp4_32k_d128"])["residual"].startswith("nvfp4")
+    assert bench.config_of(synth.WORKLOADS["nvfp4_32k_d128"], True)["residual"].startswith("nvfp4")
+    # a parity-size case is named as one, not passed off as L2-exceeding
+    assert "fit in the 126 MB L2" in bench.config_of(synth.WORKLOADS["tiny_1k_d64"], True)["l2"]
 
 
 def _run_reference(env_extra):
@@ -153,9 +156,15 @@ def test_reference_arm_prints_one_contract_line():
     (line,) = _run_reference({})
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOPS"
     assert line["metric"] == bench.METRIC and line["higher_is_better"] is True and line["n_gpus"] == 1
-    assert line["config"] == bench.config_of(synth.WORKLOADS["mid_32k_d128"])
+    assert line["config"] == bench.config_of(synth.WORKLOADS["mid_32k_d128"], True)
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert cb["cpu_model"]
+    # ms_per_step is the measured sample; the full-workload time is an extrapolation beside it
+    samp = line["sample_s"]["prep"] + line["sample_s"]["rows"]
+    assert line["ms_per_step"] >= 0.9 * samp * 1e3
+    assert line["extrapolated_step_s"] == pytest.approx(line["extrapolated_head_s"] * 40)
+    assert line["value"] == pytest.approx(40 * 4.0 * 32768 ** 2 * 128 / line["extrapolated_step_s"] / 1e12)
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
 
@@ -170,7 +179,7 @@ def test_prep_roofline_against_the_workload_arithmetic():
     At the measured peaks the two floors nearly coincide (about 0.156 ms)."""
     w = synth.WORKLOADS["mid_32k_d128"]
     peaks = dict(hbm_gbs=6538.0, bf16=1606.0, bf16_sustained=1384.2)
-    r = bench.prep_roofline(w, 3.45, peaks)
+    r = bench.prep_roofline(w, 3.45, peaks, timed_s=5.0)
     per_head = 4 * 32768 * 128 + 2 * 32768 * 128 + 4 * 32768 + 4 * 256 * 128 + 4 * 256 + 4 * 128
     assert r["bytes"] == 40 * per_head and abs(r["bytes"] / 1e9 - 1.017) < 0.001
     assert r["flops"] == 2.0 * 32768 * 64 * 128 * 10 * 40 and abs(r["flops"] / 1e9 - 214.7) < 0.1
@@ -180,9 +189,18 @@ def test_prep_roofline_against_the_workload_arithmetic():
     assert r["achieved_gbs"] == pytest.approx(r["bytes"] / 3.45e-3 / 1e9)
     # the 4-bit workload writes half the residual bytes plus one scale byte per 16
     w4 = synth.WORKLOADS["nvfp4_32k_d128"]
-    r4 = bench.prep_roofline(w4, 2.0, peaks)
+    r4 = bench.prep_roofline(w4, 2.0, peaks, timed_s=5.0)
     per_head4 = per_head - 32768 * 128 // 2 + 256 * 128 * 8
     assert r4["bytes"] == 24 * per_head4
     # without a sustained figure the burst one is used
-    assert bench.prep_roofline(w, 3.45, dict(hbm_gbs=6538.0, bf16=1606.0, bf16_sustained=None))["peak_bf16_tflops"] \
-        == 1606.0
+    assert bench.prep_roofline(w, 3.45, dict(hbm_gbs=6538.0, bf16=1606.0, bf16_sustained=None),
+                               timed_s=5.0)["peak_bf16_tflops"] == 1606.0
+    # and so it is for a timed region under two seconds
+    assert bench.prep_roofline(w, 3.45, peaks, timed_s=0.3)["peak_bf16_tflops"] == 1606.0
+
+
+def test_tensor_peak_by_timed_region():
+    peaks = dict(hbm_gbs=6538.0, bf16=1606.0, bf16_sustained=1384.2)
+    assert bench.tensor_peak(peaks, 0.35) == (1606.0, "burst")
+    assert bench.tensor_peak(peaks, 3.0) == (1384.2, "sustained")
+    assert bench.tensor_peak(dict(peaks, bf16_sustained=None), 3.0) == (1606.0, "burst")

@@ -11,7 +11,8 @@ import torch
 
 import oracle
 from bit_fp8_attention_smooth_b200 import synth
-from gpu_common import BETA, COS_TOL, REL_L2_TOL, bits, check_perm, gpu_prep_head, metrics
+from gpu_common import (BETA, COS_TOL, REL_L2_TOL, check_labels_valid, check_perm, gpu_prep_head, metrics,
+                        oracle_prep_on_perm)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -72,9 +73,14 @@ def _check_workload(vc, w, smooth=True, resid_fmt=0):
         check_perm(got["perm"], got["labels"], w.N)
         agree = (got["labels"] == ref["prep"]["labels"]).mean()
         assert agree >= 0.999, (h, agree)
-        if np.array_equal(got["perm"], ref["prep"]["perm"]):
-            for key in ("khat", "ksc", "vmu", "vsc") + (("vq", "vgs") if resid_fmt == 1 else ("vhat",)):
-                assert np.array_equal(got[key], ref["prep"][key]), (h, key)
+        vb, kb = synth.head_bits(w, "v", 0, h), synth.head_bits(w, "k", 0, h)
+        if smooth:
+            check_labels_valid(vb, got["labels"], ref["prep"]["labels"], ref["prep"]["centroids"])
+            assert np.array_equal(got["perm"], oracle.stable_perm(got["labels"], w.C))
+        # quantiser bytes, always: the oracle's quantisers on the GPU's own order
+        own = oracle_prep_on_perm(kb, vb, got["perm"], w.block, smooth, resid_fmt)
+        for key in ("khat", "ksc", "vmu", "vsc") + (("vq", "vgs") if resid_fmt == 1 else ("vhat",)):
+            assert np.array_equal(got[key], own[key]), (h, key)
         rel, cos, _ = metrics(gout[h], ref["out"])
         rel_x, _, psnr_x = metrics(gout[h], ref["exact"])
         print(f"{w.name} smooth={smooth} resid_fmt={resid_fmt} head {h}: labels agree {agree:.5f}, "

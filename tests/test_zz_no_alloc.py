@@ -15,18 +15,6 @@ import torch
 
 pytestmark = pytest.mark.gpu
 
-REL_L2_TOL = 1e-2
-COS_TOL = 0.9995
-
-
-def _metrics(a, b):
-    a = a.double().flatten()
-    b = b.double().flatten()
-    rel = ((a - b).norm() / b.norm()).item()
-    cos = (a @ b / (a.norm() * b.norm())).item()
-    return rel, cos
-
-
 @pytest.mark.parametrize("N,d,block,resid_fmt", [(3000, 128, 128, 0), (1000, 64, 64, 0), (2100, 128, 128, 1)])
 def test_noalloc_matches_workspace_entry_point(N, d, block, resid_fmt):
     import bit_fp8_attention_smooth_b200 as vc
@@ -35,6 +23,8 @@ def test_noalloc_matches_workspace_entry_point(N, d, block, resid_fmt):
     L = vc.lib()
     w = synth.custom(f"noalloc_{N}_{d}", 1, 2, N, d, 31, pool=8, C=8, iters=4, block=block)
     q, k, v = (synth.tensor_bf16(w, t).cuda() for t in "qkv")
+    q[:, :, :3] = 0  # zero rows (padding tokens): score scale 0 over the ragged last key tile too
+    q[:, :, -2:] = 0
     params = vc.Params.for_workload(w, beta=64, resid_fmt=resid_fmt)
     ws = vc.alloc_workspace(tuple(q.shape), params)
     prep = vc.smooth_prepare(k, v, params, workspace=ws)
@@ -50,8 +40,8 @@ def test_noalloc_matches_workspace_entry_point(N, d, block, resid_fmt):
                                    ctypes.byref(params_c), ctypes.c_void_p(out.data_ptr()), stream)
         assert st == vc.VC_OK, vc.status_string(st)
         torch.cuda.synchronize()
-        rel, cos = _metrics(out.float().cpu(), ref.float().cpu())
-        assert rel <= REL_L2_TOL and cos >= COS_TOL, (call, rel, cos)
+        # the same kernels on the same inputs: the same bits
+        assert torch.equal(out, ref), (call, (out.float() - ref.float()).abs().max().item())
 
 
 def test_noalloc_rejects_oversized_problems():
