@@ -71,9 +71,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the phase of parity `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bound on draining a CTA's own in-flight copies and MMAs after an abort; it
 // does not depend on the (possibly tiny) wait limit.
 constexpr int64_t kDrainNs = 2000000000LL;
+
+// Wait limits below this leave no time to wait at all: only a phase already
+// complete at the first (non-blocking) poll passes.  A blocking try_wait can
+// hold a thread for longer than such a limit, and the global timer ticks more
+// coarsely, so a shorter limit could not be told apart from none.
+constexpr int64_t kMinWaitNs = 1000;
 
 // Waits for the phase of parity `parity` to complete.  Gives up when the CTA
 // abort flag is raised by another warp, or after ctl.limit_ns, in which case
@@ -81,7 +100,12 @@ constexpr int64_t kDrainNs = 2000000000LL;
 // gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const DevCtl& ctl,
                                           volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
+    if (ctl.limit_ns < kMinWaitNs) {
+        *abort_flag = 1;
+        record_error(ctl, VC_ERR_DEVICE_TIMEOUT);
+        return false;
+    }
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;

@@ -73,7 +73,8 @@ typedef struct {
                               2 = V-Smooth reusing the regroup already in the prep's perm (from an
                               earlier call on the same shape): no k-means, K/V quantised in that order */
     int32_t resid_fmt;     /* 0 = E4M3 residual; 1 = 4-bit NVFP4 residual (block 128 only) */
-    int64_t wait_limit_ns; /* bound on any single device-side wait; 0 = 2 s */
+    int64_t wait_limit_ns; /* bound on any single device-side wait; 0 = 2 s; below 1000 ns no
+                              wait at all: only a phase complete at its first poll passes */
 } vc_params;
 
 /*

@@ -1,7 +1,8 @@
 """Failure detection on the GPU without a fault.
 
 Every device-side wait in the library is bounded by params.wait_limit_ns.  A
-limit of 1 ns makes the first wait that is not already satisfied run out: the
+limit under 1 us leaves no time to wait: the first wait whose phase is not
+already complete at its first (non-blocking) poll runs out, and the
 kernel records VC_ERR_DEVICE_TIMEOUT in the workspace status word, lets its
 own copies and MMAs land, frees its tensor memory and returns, so the context
 stays usable.  These tests check the status vc_check reports, that kernels
