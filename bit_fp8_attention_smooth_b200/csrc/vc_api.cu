@@ -40,7 +40,7 @@ WsLayout ws_layout(const vc_shape& s, const vc_params& p) {
     w.cent64 = o; o = align256(o + 8 * BH * C * D);
     w.vnorm2 = o; o = align256(o + 4 * BH * N);
     w.ties = o; o = align256(o + sizeof(vc::KmTie) * BH * N);
-    w.tie_count = o; o = align256(o + 2 * sizeof(int));
+    w.tie_count = o; o = align256(o + (2 + 2 * vc::kKmTieRegions) * sizeof(int));  // + km_pass's regions
     w.sums = o; o = align256(o + 8 * BH * C * D);
     w.cstart = o; o = align256(o + 4 * BH * C);
     w.ccount = o; o = align256(o + 4 * BH * C);

@@ -130,6 +130,36 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
     return __all_sync(0xffffffffu, ok);
 }
 
+// mbar_wait for warps off the critical path: between polls the thread sleeps
+// about `sleep_ns`, so a long wait takes almost no issue slots from the warps
+// of its sub-partition that have work.  Same limits and verdicts as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, const DevCtl& ctl,
+                                               volatile int* abort_flag, uint32_t sleep_ns) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (ctl.limit_ns < kMinWaitNs) {
+        *abort_flag = 1;
+        record_error(ctl, VC_ERR_DEVICE_TIMEOUT);
+        return false;
+    }
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        __nanosleep(sleep_ns);
+        if (mbar_test_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if ((int64_t)(globaltimer() - t0) > ctl.limit_ns) {
+            *abort_flag = 1;
+            record_error(ctl, VC_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool warp_wait_idle(uint32_t bar, uint32_t parity, const DevCtl& ctl,
+                                               volatile int* abort_flag, uint32_t sleep_ns) {
+    const bool ok = mbar_wait_idle(bar, parity, ctl, abort_flag, sleep_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait that ignores the abort flag (used to drain in-flight copies and
 // MMAs before the CTA exits).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, const DevCtl& ctl) {

@@ -54,10 +54,14 @@ struct AttnArgs {
 };
 
 struct KmState {  // per (b, h), 16 bytes of workspace
-    int changed;
-    int done;
-    int pad0, pad1;
+    int chg[2];  // labels changed by pass it, in chg[it % 2]
+    int done;    // the labels stopped changing: the regroup is final
+    int pad;
 };
+
+// The fused k-means pass lists near ties in one region per CTA (one CTA per
+// SM); the workspace holds the (start, count) pairs of this many regions.
+constexpr int kKmTieRegions = 1024;
 
 // A k-means near tie: a token whose tensor-core distances leave more than one
 // cluster within the error bound; km_refine decides it in fp64.

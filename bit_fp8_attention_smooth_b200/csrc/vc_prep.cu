@@ -72,7 +72,7 @@ __global__ void km_init(const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __re
     if (k == 0 && bh == 0 && c < 2) tie_count[c] = 0;
     if (k == 0) {
         vamax[(size_t)bh * D + c] = 0u;
-        if (c == 0) state[bh] = KmState{0, 0, 0, 0};
+        if (c == 0) state[bh] = KmState{{0, 0}, 0, 0};
     }
 }
 
@@ -287,15 +287,19 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
                     bestk = k4[e];
                 }
             }
-            // Error bound of the tensor-core distance: bf16 hi/lo centroids carry
-            // 2^-16 relative error, the products are exact and the fp32
-            // accumulation of the 2 D products errs by at most 2^-15 of
-            // sum |v_c c_c|, so |err| <= 2^-14 (|v| + max|c|)^2 with room to
-            // spare.  Clusters within twice that of the best are decided again
-            // in fp64 from the fp64 centroids, as the Lloyd step defines the
-            // distance (sum over channels of (v - c)^2).
+            // Error bound of the tensor-core distance d = |c|^2 - 2 v.c: the bf16
+            // hi/lo centroid carries 2^-16 relative error per channel, the
+            // products are exact, and the fp32 accumulation of the 2 D products
+            // errs by at most 2^-15 of sum |v_c c_c| (one unit of fp32
+            // truncation per addition), so 2 v.c errs by at most
+            // 3 * 2^-15 |v||c| <= 2^-15.4 (|v| + max|c|)^2; |c|^2 in fp32 adds
+            // far less.  If every d errs by at most E, the fp64 argmin lies
+            // within 2E of the tensor-core best, so the clusters within
+            // 2^-13 (|v| + max|c|)^2 of the best (2.6 times 2E) are decided
+            // again in fp64 from the fp64 centroids, as the Lloyd step defines
+            // the distance (sum over channels of (v - c)^2).
             const float rad = sqrtf(vn2) + cmax_r;
-            const float margin = ldexpf(rad * rad, -12);
+            const float margin = ldexpf(rad * rad, -13);
             const bool refine = valid && C > 1 && (second - best) <= margin;
             // Near ties go to the list that km_refine decides in fp64; the
             // label written now is the tensor-core choice.
@@ -356,7 +360,7 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
         for (int k = tid; k < C; k += 128) hist[((size_t)bh * C + k) * nblk + blk0 + j] = hp[k];
     }
     changed = __reduce_add_sync(0xffffffffu, changed);
-    if (lane == 0 && changed) atomicAdd(&state[bh].changed, changed);
+    if (lane == 0 && changed) atomicAdd(&state[bh].chg[it & 1], changed);
     // After an abort thread 0's last copies and MMAs may still be in flight:
     // let them land before shared memory and TMEM are released.
     if (tid == 0 && !ok) {
@@ -378,27 +382,667 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
     }
 }
 
-// fp64 decision of the near ties km_assign listed: one warp a token, each
+// ------------------------------------------------------------------ fused pass
+// One k-means pass for C <= 64, persistent: one CTA per SM takes an equal,
+// contiguous share of the (head, 128-token tile) units of the heads whose
+// labels still change, and reads each V tile once for both halves of the
+// Lloyd step:
+//   assignment  label = argmin_k |c_k|^2 - 2 v.c_k on tensor cores (kind::f16,
+//               v . c_hi + v . c_lo in TMEM), ties to the lowest k, near ties
+//               listed for km_refine, the tile's cluster histogram, and the
+//               tile's tokens grouped by cluster (a counting sort);
+//   update      the member sums from the same V tile in shared memory: update
+//               warp u owns clusters 8u .. 8u + 7, whose tokens are one
+//               contiguous block of the grouped tile; it walks the block four
+//               tokens at a time, adds each run of a cluster in registers and
+//               the run's sum to the CTA's fp64 sums in shared memory; those go
+//               to the head's global sums
+//               (one fp64 atomic each) when the CTA leaves the head.  Every
+//               fp64 addition of bf16 values is exact (for values of typical
+//               range), so the sums do not depend on the order and equal the
+//               oracle's sequential ones.  Loops stay short: with four warp
+//               roles in one CTA, long unrolled code stalls on instruction
+//               fetch.
+// `mode` 1 is that full accumulation (the sums start from zero).  Mode 2 keeps
+// the sums of the previous pass and moves only the tokens whose label changed
+// (the assignment warps subtract the row from the old cluster's global sums
+// and add it to the new one's, fp64 atomics): exact like a fresh sum, and
+// cheap once few labels change.  Mode 0 (the last pass) writes labels and
+// histograms only.
+// Warps: 0 TMA producer (V tiles through a 3-stage ring; a head's centroids
+// when the CTA enters it), 1 MMA issuer (tile i into accumulator i % 2 in
+// TMEM), then KP_GROUPS assignment groups of four warps (group g takes the
+// CTA's tiles i = g mod KP_GROUPS; a thread per token), then 8 update warps
+// (D/32 channels a lane).
+constexpr int KP_GROUPS = 1;
+constexpr int KP_STAGES = 3;
+constexpr int KP_SEG = 68;      // per stage: 65 cluster offsets, padded
+constexpr int KP_UPD = 8;       // update warps
+constexpr int KP_ASG = 4 * KP_GROUPS;  // assignment warps
+constexpr int KP_THREADS = 32 * (2 + KP_ASG + KP_UPD);
+constexpr int KP_MAX_GRID = kKmTieRegions;  // near-tie regions the workspace holds
+
+// Shared-memory plan of km_pass, from a 1024-byte aligned base:
+//   V ring | centroid hi | centroid lo | fp64 sums [64][D] | |c|^2 per group |
+//   tile order and its labels per stage | cluster offsets per stage | label
+//   counts per group x2 | scratch | barriers
+struct KpLayout {
+    uint32_t v_bytes, c_bytes, off_v, off_chi, off_clo, off_sum, off_cn, off_ord, off_slab, off_seg, off_cnt, off_misc,
+        off_bar, bytes;
+    __host__ __device__ KpLayout(int D, int Cp) {
+        v_bytes = KM_TOK * D * 2;
+        c_bytes = Cp * D * 2;
+        off_v = 0;
+        off_chi = off_v + KP_STAGES * v_bytes;
+        off_clo = off_chi + c_bytes;
+        off_sum = off_clo + c_bytes;                 // [64][D] double
+        off_cn = off_sum + 64 * D * 8;               // [2][64] float
+        off_ord = off_cn + 2 * 64 * 4;               // [stage][128] tile rows grouped by cluster
+        off_slab = off_ord + KP_STAGES * KM_TOK;     // [stage][128] their clusters
+        off_seg = off_slab + KP_STAGES * KM_TOK;     // [stage][KP_SEG] first grouped position of each cluster
+        off_cnt = off_seg + KP_STAGES * KP_SEG * 4;  // [2][2][64] label counts of a group's tile
+        off_misc = off_cnt + 2 * 2 * 64 * 4;         // [16] ints, see km_pass
+        off_bar = off_misc + 64;
+        bytes = off_bar + 8 * (3 * KP_STAGES + 7) + 1024;  // + alignment slack
+    }
+};
+
+// All-of over the threads of named barrier `id` (bar.red.and): every thread
+// gets the same answer, so a decision taken on it is uniform.
+__device__ __forceinline__ bool named_barrier_and(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+// The walk over a CTA's units: (bh, tile) in head-major order over the heads
+// not yet final.
+struct KpWalk {
+    int bh, tile;
+    __device__ __forceinline__ void next(const KmState* state, int BH, int nblk) {
+        if (++tile == nblk) {
+            tile = 0;
+            do {
+                ++bh;
+            } while (bh < BH && state[bh].done);
+        }
+    }
+};
+
+// bf16 -> fp64 by placing the bits: a bf16 with sign s, exponent e and
+// mantissa m read as the fp64 with sign s, exponent field e and mantissa m
+// (top bits) is the bf16 value times 2^-896, exactly, for every finite bf16
+// (normal: 2^(e-1023) (1 + m/128) = 2^-896 * 2^(e-127) (1 + m/128); zero and
+// subnormal: m 2^-1029 = 2^-896 * m 2^-133).  Sums of these scaled values are
+// exact whenever the unscaled ones are; multiplying by 2^896 (kBf16Unscale)
+// gives the sum back exactly.  The high word is the bf16's 16 bits moved to
+// the top of a 32-bit word, shifted right by 3 with the sign copied, and the
+// copies of the sign and the bits shifted in from below cleared.
+constexpr double kBf16Unscale = 0x1p896;
+__device__ __forceinline__ double bf16hi_scaled(uint32_t w) {  // bits 16..31 of w
+    return __hiloint2double((int)(((int)w >> 3) & 0x8FFFE000), 0);
+}
+__device__ __forceinline__ double bf16lo_scaled(uint32_t w) {  // bits 0..15 of w
+    return bf16hi_scaled(w << 16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(KP_THREADS, 1)
+    km_pass(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_chi,
+            const __grid_constant__ CUtensorMap tm_clo, const float* __restrict__ cnorm, float* __restrict__ vnorm2,
+            int32_t* __restrict__ labels, int32_t* __restrict__ hist, double* __restrict__ sums,
+            KmTie* __restrict__ ties, int* __restrict__ tie_regions, KmState* __restrict__ state, int BH, int N,
+            int C, int Cp, int it, int mode, DevCtl ctl) {
+    constexpr int S = KP_STAGES;
+    const bool accumulate = mode == 1;
+    if (ctl_failed(ctl.status)) return;
+    const int nblk = (N + KM_TOK - 1) / KM_TOK;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_base);
+    const KpLayout L(D, Cp);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // scratch: [0] TMEM base, [1] abort flag, [2..3] max |c|^2 bits of each
+    // group's head, [4] units, [5] first head, [6] first tile, [7] near ties
+    // listed, [8] near-tie region start
+    int* misc = reinterpret_cast<int*>(smem + L.off_misc);
+    volatile int* abort_flag = misc + 1;
+    int* tie_s = misc + 7;
+    int* cnt_s = reinterpret_cast<int*>(smem + L.off_cnt);
+    const uint32_t bar0 = base + L.off_bar;
+    auto b_vfull = [&](int st) { return bar0 + 8u * st; };
+    auto b_vempty = [&](int st) { return bar0 + 8u * (S + st); };
+    auto b_lfull = [&](int st) { return bar0 + 8u * (2 * S + st); };
+    auto b_accfull = [&](int b) { return bar0 + 8u * (3 * S + b); };
+    auto b_accempty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+    const uint32_t b_cfull = bar0 + 8u * (3 * S + 4), b_cempty = b_cfull + 8, b_mmadone = b_cfull + 16;
+    if (tid == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(b_vfull(st), 1);
+            // the MMA warp's commit, the 4 warps of the assignment group, the update warps
+            mbar_init(b_vempty(st), 1 + 4 + (accumulate ? KP_UPD : 0));
+            mbar_init(b_lfull(st), 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(b_accfull(b), 1);
+            mbar_init(b_accempty(b), 4);
+        }
+        mbar_init(b_cfull, 1);
+        mbar_init(b_cempty, 1);
+        mbar_init(b_mmadone, 1);
+        *abort_flag = 0;
+        *tie_s = 0;
+        fence_mbar_init();
+    }
+    for (int i = tid; i < 2 * 2 * 64; i += blockDim.x) cnt_s[i] = 0;
+    double* sums_s = reinterpret_cast<double*>(smem + L.off_sum);
+    if (accumulate)
+        for (int i = tid; i < 64 * D; i += blockDim.x) sums_s[i] = 0.0;
+    const uint32_t ncols = 2 * Cp <= 32 ? 32 : (2 * Cp <= 64 ? 64 : 128);
+    if (warp == 1) {
+        tmem_alloc(smem_u32(reinterpret_cast<uint32_t*>(misc)), ncols);
+        tmem_relinquish();
+    }
+    if (warp == 2) {
+        // This CTA's share of the live units: the heads still changing, nblk
+        // units each, split evenly over the grid.
+        int live = 0;
+        for (int bh = lane; bh < BH; bh += 32) live += state[bh].done == 0;
+        live = __reduce_add_sync(0xffffffffu, live);
+        const int64_t units = (int64_t)live * nblk;
+        const int64_t lu0 = units * blockIdx.x / gridDim.x, lu1 = units * (blockIdx.x + 1) / gridDim.x;
+        // the head of live unit lu0: the (lu0 / nblk)-th live head
+        const int64_t target = lu0 / nblk;
+        int seen = 0, bh0 = BH;
+        for (int b0 = 0; b0 < BH && lu1 > lu0; b0 += 32) {
+            const int bh = b0 + lane;
+            uint32_t m = __ballot_sync(0xffffffffu, bh < BH && state[bh].done == 0);
+            if (seen + __popc(m) > target) {
+                for (int q = 0; q < (int)(target - seen); ++q) m &= m - 1;
+                bh0 = b0 + __ffs(m) - 1;
+                break;
+            }
+            seen += __popc(m);
+        }
+        if (lane == 0) {
+            misc[4] = (int)(lu1 - lu0);
+            misc[5] = bh0;
+            misc[6] = (int)(lu0 % nblk);
+            // Near ties go to this CTA's region of the list: from the live-token
+            // index of its first unit, as many entries as its units hold tokens.
+            misc[8] = (int)(target * N + (lu0 % nblk) * KM_TOK);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[0];
+    const int nunits = misc[4];
+    const KpWalk start{misc[5], misc[6]};
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (lane 0)
+        if (lane == 0 && nunits > 0) {
+            prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_chi);
+            prefetch_tmap(&tm_clo);
+            KpWalk w = start;
+            int i = 0, hs = -1, cur = -1;
+            for (; i < nunits; ++i, w.next(state, BH, nblk)) {
+                if (w.bh != cur) {  // the head's centroids, once the MMAs of the last head are done
+                    if (hs >= 0 && !mbar_wait(b_cempty, hs & 1, ctl, abort_flag)) break;
+                    ++hs;
+                    cur = w.bh;
+                    mbar_expect_tx_arrive(b_cfull, 2 * L.c_bytes);
+#pragma unroll
+                    for (int kc = 0; kc < D / 64; ++kc) {
+                        tma_load_3d(base + L.off_chi + kc * (Cp * 128), &tm_chi, b_cfull, 64 * kc, 0, w.bh);
+                        tma_load_3d(base + L.off_clo + kc * (Cp * 128), &tm_clo, b_cfull, 64 * kc, 0, w.bh);
+                    }
+                }
+                const int st = i % S;
+                if (i >= S && !mbar_wait(b_vempty(st), ((i / S) - 1) & 1, ctl, abort_flag)) break;
+                mbar_expect_tx_arrive(b_vfull(st), L.v_bytes);
+#pragma unroll
+                for (int kc = 0; kc < D / 64; ++kc)
+                    tma_load_3d(base + L.off_v + st * L.v_bytes + kc * (KM_TOK * 128), &tm_v, b_vfull(st),
+                                64 * kc, w.tile * KM_TOK, w.bh);
+            }
+            // the copies still in flight (the earlier ones were consumed) land
+            // before shared memory is released
+            for (int j = i - S < 0 ? 0 : i - S; j < i; ++j) drain_wait(b_vfull(j % S), (j / S) & 1, ctl);
+            if (hs >= 0) drain_wait(b_cfull, hs & 1, ctl);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (lane 0)
+        if (lane == 0 && nunits > 0) {
+            const uint32_t idesc = idesc_bf16_f32(Cp);
+            KpWalk w = start;
+            int hs = -1, cur = -1;
+            for (int i = 0; i < nunits; ++i, w.next(state, BH, nblk)) {
+                if (w.bh != cur) {
+                    if (hs >= 0) mma_commit(b_cempty);  // the last head's MMAs: its centroids are free
+                    ++hs;
+                    cur = w.bh;
+                    if (!mbar_wait(b_cfull, hs & 1, ctl, abort_flag)) break;
+                }
+                const int st = i % S, b = i & 1;
+                if (!mbar_wait(b_vfull(st), (i / S) & 1, ctl, abort_flag)) break;
+                if (i >= 2 && !mbar_wait(b_accempty(b), ((i >> 1) - 1) & 1, ctl, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t sA = base + L.off_v + st * L.v_bytes, acc = tmem + b * Cp;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;
+                    mma_bf16(acc, smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128),
+                             smem_desc(base + L.off_chi + (kk >> 2) * (Cp * 128) + off, 128), idesc, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;
+                    mma_bf16(acc, smem_desc(sA + (kk >> 2) * (KM_TOK * 128) + off, 128),
+                             smem_desc(base + L.off_clo + (kk >> 2) * (Cp * 128) + off, 128), idesc, 1u);
+                }
+                mma_commit(b_accfull(b));
+                mma_commit(b_vempty(st));
+            }
+            mma_commit(b_mmadone);  // every MMA issued has finished before TMEM is released
+            drain_wait(b_mmadone, 0, ctl);
+        }
+    } else if (warp < 2 + KP_ASG) {
+        // ------------------------------------------------------------ assignment (thread per token)
+        // Group g takes tiles i = g, g + KP_GROUPS, ...  TMEM lane quadrant
+        // q = warp % 4 holds tile rows 32q..32q+31.
+        const int g = (warp - 2) >> 2;
+        const int qd = warp & 3;
+        const int r = qd * 32 + lane;
+        const int bar_id = 1 + g;
+        float* cn_s = reinterpret_cast<float*>(smem + L.off_cn) + g * 64;
+        uint8_t* ord_s = smem + L.off_ord;
+        uint8_t* slab_s = smem + L.off_slab;
+        int* seg_s = reinterpret_cast<int*>(smem + L.off_seg);
+        const int tie_base = misc[8];
+        KpWalk w = start;
+        for (int q = 0; q < g; ++q) w.next(state, BH, nblk);
+        int cur = -1, changed = 0;
+        float cmax_r = 0.0f;
+        auto flush_changed = [&]() {
+            const int t = __reduce_add_sync(0xffffffffu, changed);
+            if (lane == 0 && t) atomicAdd(&state[cur].chg[it & 1], t);
+            changed = 0;
+        };
+        // the previous pass's label and |v|^2 of this thread's token, fetched
+        // one group tile ahead so the loads overlap the work on the current one
+        int32_t nxt_old = -1;
+        float nxt_vn2 = 0.0f;
+        auto fetch = [&](const KpWalk& u) {
+            const int n = u.tile * KM_TOK + r;
+            nxt_old = -1;
+            nxt_vn2 = 0.0f;
+            if (it > 0 && n < N) {
+                nxt_old = labels[(size_t)u.bh * N + n];
+                nxt_vn2 = vnorm2[(size_t)u.bh * N + n];
+            }
+        };
+        if (g < nunits) fetch(w);
+        for (int i = g; i < nunits; i += KP_GROUPS) {
+            const int bh = w.bh, tile = w.tile;
+            if (bh != cur) {  // |c_k|^2 of the new head (pad clusters +inf, never chosen), max_k |c_k|^2
+                if (cur >= 0) flush_changed();
+                cur = bh;
+                named_barrier_sync(bar_id, 128);  // every warp of the group is past the last head's tile
+                if (qd == 0) {
+                    uint32_t mb = 0;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int k = 2 * lane + e;
+                        const float x = k < C ? cnorm[(size_t)bh * Cp + k] : INFINITY;
+                        cn_s[k] = x;
+                        if (k < C) mb = max(mb, __float_as_uint(x));  // x >= 0: bit order is value order
+                    }
+                    mb = __reduce_max_sync(0xffffffffu, mb);
+                    if (lane == 0) misc[2 + g] = (int)mb;
+                }
+                named_barrier_sync(bar_id, 128);
+                cmax_r = sqrtf(__uint_as_float((uint32_t)misc[2 + g]));
+            }
+            const int32_t old_label = nxt_old;
+            float vn2 = nxt_vn2;
+#pragma unroll
+            for (int q = 0; q < KP_GROUPS; ++q) w.next(state, BH, nblk);  // this group's next tile
+            if (i + KP_GROUPS < nunits) fetch(w);
+            const int st = i % S, b = i & 1;
+            int* cnt = cnt_s + (g * 2 + ((i / KP_GROUPS) & 1)) * 64;  // this tile's label counts
+            const int n = tile * KM_TOK + r;
+            const bool valid = n < N;
+            // the accumulator of tile i (its MMA also means V tile i has landed)
+            const bool okj = warp_wait(b_accfull(b), (i >> 1) & 1, ctl, abort_flag);
+            int label = 0, rank = 0;
+            if (okj) {
+                tc_fence_after();
+                const uint32_t lane_tmem = tmem + b * Cp + ((uint32_t)(qd * 32) << 16);
+                float dk[64];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (16 * q < Cp) {
+                        tmem_ld16(lane_tmem + 16 * q, dk + 16 * q);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) dk[16 * q + e] = 0.0f;  // pad clusters: |c|^2 = +inf decides
+                    }
+                }
+                if (it == 0) {  // |v|^2 once per prep, from the V tile (resident until this warp releases it)
+                    const uint8_t* arow = smem + L.off_v + st * L.v_bytes + r * 128;
+                    vn2 = 0.0f;
+#pragma unroll
+                    for (int kc = 0; kc < D / 64; ++kc)
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) {
+                            const uint4 raw = *reinterpret_cast<const uint4*>(arow + kc * (KM_TOK * 128) +
+                                                                              ((ch ^ (r & 7)) << 4));
+                            const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) vn2 = fmaf(bf2f(hv[e]), bf2f(hv[e]), vn2);
+                        }
+                    if (valid) vnorm2[(size_t)bh * N + n] = vn2;
+                }
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_accempty(b));  // the accumulator is free for tile i + 2
+                // best and runner-up of d_k = |c_k|^2 - 2 v.c_k, four chains (k % 4)
+                float b4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+                float s4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+                int k4[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int q4 = 0; q4 < 16; ++q4) {
+                    const float4 cn = reinterpret_cast<const float4*>(cn_s)[q4];
+                    const float cv[4] = {cn.x, cn.y, cn.z, cn.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float d = fmaf(-2.0f, dk[4 * q4 + e], cv[e]);
+                        dk[4 * q4 + e] = d;
+                        const bool lt = d < b4[e];
+                        s4[e] = fminf(s4[e], fmaxf(b4[e], d));
+                        b4[e] = fminf(b4[e], d);
+                        k4[e] = lt ? 4 * q4 + e : k4[e];
+                    }
+                }
+                float best = b4[0], second = s4[0];
+                int bestk = k4[0];
+#pragma unroll
+                for (int e = 1; e < 4; ++e) {
+                    second = fminf(fminf(second, s4[e]), fmaxf(best, b4[e]));
+                    if (b4[e] < best || (b4[e] == best && k4[e] < bestk)) {
+                        best = b4[e];
+                        bestk = k4[e];
+                    }
+                }
+                // Near ties within the error bound derived at km_assign.  The
+                // radius takes an approximate square root (relative error near
+                // 2^-22): the margin sits 2.6 times above the bound, and only
+                // chooses which tokens km_refine decides again in fp64.
+                const float rad = (vn2 > 0.0f ? vn2 * rsqrtf(vn2) : 0.0f) + cmax_r;
+                const float margin = rad * rad * 0x1p-13f;
+                const bool refine = valid && C > 1 && (second - best) <= margin;
+                const uint32_t rmask = __ballot_sync(0xffffffffu, refine);
+                if (rmask != 0) {
+                    int first = 0;
+                    if (lane == 0) first = atomicAdd(tie_s, __popc(rmask));
+                    first = __shfl_sync(0xffffffffu, first, 0);
+                    if (refine) {
+                        KmTie* e = ties + tie_base + first + __popc(rmask & ((1u << lane) - 1));
+                        const float lim = best + margin;
+                        uint32_t m0 = 0, m1 = 0;  // candidates 0..31 and 32..63 (pads are +inf)
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            if (dk[jj] <= lim) m0 |= 1u << jj;
+                            if (dk[32 + jj] <= lim) m1 |= 1u << jj;
+                        }
+                        e->mask[0] = m0;
+                        e->mask[1] = m1;
+                        *reinterpret_cast<int4*>(e) = make_int4(bh, n, old_label, bestk);
+                    }
+                }
+                if (valid) {
+                    label = bestk;
+                    if (it == 0 || old_label != label) ++changed;
+                    labels[(size_t)bh * N + n] = label;
+                    rank = atomicAdd(&cnt[label], 1);  // the token's place among its cluster's in this tile
+                }
+                if (mode == 2) {  // move the tokens that changed cluster, a row at a time over the warp
+                    constexpr int NCH = D / 32;
+                    const int c0 = NCH * lane;
+                    const uint8_t* vtile = smem + L.off_v + st * L.v_bytes + (c0 >> 6) * (KM_TOK * 128) + (c0 & 7) * 2;
+                    const int q16 = (c0 & 63) >> 3;
+                    uint32_t cm = __ballot_sync(0xffffffffu, valid && label != old_label);
+                    while (cm) {
+                        const int src = __ffs(cm) - 1;
+                        cm &= cm - 1;
+                        const int ko = __shfl_sync(0xffffffffu, old_label, src);
+                        const int kn = __shfl_sync(0xffffffffu, label, src);
+                        const int row = qd * 32 + src;
+                        const uint8_t* p2 = vtile + row * 128 + ((q16 ^ (row & 7)) << 4);
+                        double* so = sums + ((size_t)bh * C + ko) * D + c0;
+                        double* sn = sums + ((size_t)bh * C + kn) * D + c0;
+#pragma unroll
+                        for (int h = 0; h < NCH / 2; ++h) {
+                            const uint32_t w2 = reinterpret_cast<const uint32_t*>(p2)[h];
+                            const double x0 = bf16lo_scaled(w2) * kBf16Unscale;  // exact
+                            const double x1 = bf16hi_scaled(w2) * kBf16Unscale;
+                            atomicAdd(so + 2 * h, -x0);
+                            atomicAdd(so + 2 * h + 1, -x1);
+                            atomicAdd(sn + 2 * h, x0);
+                            atomicAdd(sn + 2 * h + 1, x1);
+                        }
+                    }
+                }
+            }
+            // one decision for the four warps: leave together or go on together
+            if (!named_barrier_and(bar_id, 128, okj)) break;
+            int* seg = seg_s + st * KP_SEG;
+            if (qd == 0) {  // the tile's histogram, to global; cluster offsets for the grouping
+                const int k0 = 2 * lane;
+                const int h0 = cnt[k0], h1 = cnt[k0 + 1];
+                cnt[k0] = 0;  // ready for this group's tile after next
+                cnt[k0 + 1] = 0;
+                if (k0 < C) hist[((size_t)bh * C + k0) * nblk + tile] = h0;
+                if (k0 + 1 < C) hist[((size_t)bh * C + k0 + 1) * nblk + tile] = h1;
+                if (accumulate) {
+                    int x = h0 + h1;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(0xffffffffu, x, o);
+                        if (lane >= o) x += y;
+                    }
+                    seg[k0] = x - h0 - h1;
+                    seg[k0 + 1] = x - h1;
+                    if (lane == 31) seg[64] = x;
+                }
+            }
+            if (accumulate) {
+                named_barrier_sync(bar_id, 128);
+                if (valid) {
+                    const int pos = st * KM_TOK + seg[label] + rank;
+                    ord_s[pos] = (uint8_t)r;
+                    slab_s[pos] = (uint8_t)label;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_lfull(st));  // the tile's grouping, for the update warps
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_vempty(st));
+        }
+        if (cur >= 0) flush_changed();
+    } else if (accumulate && nunits > 0) {
+        // ------------------------------------------------------------ update, mode 1 (D/32 channels a lane)
+        constexpr int NCH = D / 32;
+        const int u = warp - 2 - KP_ASG;        // clusters 8u .. 8u + 7
+        const int c0 = NCH * lane;              // channels c0 .. c0 + NCH - 1
+        const int kc = c0 >> 6, q16 = (c0 & 63) >> 3, wo = (c0 & 7) * 2;  // chunk, 16-byte piece, byte
+        const uint8_t* ord_s = smem + L.off_ord;
+        const uint8_t* slab_s = smem + L.off_slab;
+        const int* seg_s = reinterpret_cast<const int*>(smem + L.off_seg);
+        auto flush = [&](int bh) {  // this warp's sums of head bh to the global sums, then zero
+#pragma unroll 1
+            for (int k = 8 * u; k < 8 * u + 8 && k < C; ++k) {
+#pragma unroll
+                for (int e = 0; e < NCH; ++e) {
+                    double* sp = sums_s + k * D + c0 + e;
+                    if (*sp != 0.0) atomicAdd(&sums[((size_t)bh * C + k) * D + c0 + e], *sp * kBf16Unscale);
+                    *sp = 0.0;
+                }
+            }
+        };
+        KpWalk w = start;
+        int cur = -1;
+        bool ok = true;
+        for (int i = 0; i < nunits; ++i, w.next(state, BH, nblk)) {
+            if (w.bh != cur) {
+                if (cur >= 0) flush(cur);
+                cur = w.bh;
+            }
+            const int st = i % S;
+            // the update trails the assignment by a tile: wait without polling hard
+            if (!(ok = warp_wait_idle(b_lfull(st), (i / S) & 1, ctl, abort_flag, 100))) break;
+            const uint8_t* ord = ord_s + st * KM_TOK;
+            const uint8_t* slab = slab_s + st * KM_TOK;
+            const uint8_t* vt = smem + L.off_v + st * L.v_bytes + kc * (KM_TOK * 128) + wo;
+            // clusters 8u .. 8u + 7 hold grouped positions [P0, P1)
+            const int P0 = seg_s[st * KP_SEG + 8 * u], P1 = seg_s[st * KP_SEG + 8 * u + 8];
+            double run[NCH];
+#pragma unroll
+            for (int e = 0; e < NCH; ++e) run[e] = 0.0;
+            int rk = P0 < P1 ? slab[P0] : 0;  // cluster of the run being added
+            auto flush_run = [&]() {
+                double* sp = sums_s + rk * D + c0;
+#pragma unroll
+                for (int e = 0; e < NCH; ++e) {
+                    sp[e] += run[e];
+                    run[e] = 0.0;
+                }
+            };
+#pragma unroll 1
+            for (int p = P0; p < P1; p += 4) {
+                // four positions' rows and clusters first, so their loads overlap
+                int j[4], kk[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int pp = min(p + t, P1 - 1);
+                    j[t] = ord[pp];
+                    kk[t] = p + t < P1 ? (int)slab[pp] : -1;
+                }
+                uint32_t x[4][NCH / 2];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const uint8_t* src = vt + j[t] * 128 + ((q16 ^ (j[t] & 7)) << 4);  // row j, 128-byte swizzle
+                    if constexpr (NCH == 4) {
+                        const uint2 y = *reinterpret_cast<const uint2*>(src);
+                        x[t][0] = y.x;
+                        x[t][1] = y.y;
+                    } else {
+                        x[t][0] = *reinterpret_cast<const uint32_t*>(src);
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if (kk[t] < 0) break;
+                    if (kk[t] != rk) {  // a new cluster's run starts (uniform over the warp)
+                        flush_run();
+                        rk = kk[t];
+                    }
+#pragma unroll
+                    for (int h = 0; h < NCH / 2; ++h) {
+                        run[2 * h] += bf16lo_scaled(x[t][h]);
+                        run[2 * h + 1] += bf16hi_scaled(x[t][h]);
+                    }
+                }
+            }
+            if (P0 < P1) flush_run();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_vempty(st));
+        }
+        if (ok && cur >= 0) flush(cur);
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {  // this CTA's near-tie region for km_refine
+        tie_regions[2 * blockIdx.x] = misc[8];
+        tie_regions[2 * blockIdx.x + 1] = *tie_s;
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
+    }
+}
+
+// fp64 decision of the near ties km_assign or km_pass listed: one warp a token, each
 // candidate's squared distance summed over D/32 channels a lane in fp64 and
 // added across the warp; candidates in ascending cluster order with a strict
 // comparison, so equal distances keep the lowest cluster (as the Lloyd step's
 // argmin).  When the decision differs from the tensor-core label, the label,
 // the tile's cluster counts and the head's change count are corrected.
+// The list is either one run counted in tie_count[it % 2] (km_assign) or, with
+// nreg > 0, km_pass's per-CTA regions: (start, count) pairs in tie_regions.
 template <int D>
 __global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties, int* __restrict__ tie_count,
+                                                 const int* __restrict__ tie_regions, int nreg,
                                                  const __nv_bfloat16* __restrict__ V,
                                                  const double* __restrict__ cent64, int32_t* __restrict__ labels,
-                                                 int32_t* __restrict__ hist, KmState* __restrict__ state, int N,
-                                                 int C, int Cp, int it, const int* __restrict__ status) {
+                                                 int32_t* __restrict__ hist, double* __restrict__ sums,
+                                                 KmState* __restrict__ state, int N, int C, int Cp, int it,
+                                                 int accumulate, const int* __restrict__ status) {
+    __shared__ int pre_s[KP_MAX_GRID + 1];  // entries before each region
+    __shared__ int start_s[KP_MAX_GRID];
     if (ctl_failed(status)) return;
     constexpr int CPL = D / 32;  // channels a lane
-    const int count = tie_count[it & 1];
-    if (blockIdx.x == 0 && threadIdx.x == 0) tie_count[(it + 1) & 1] = 0;  // the next pass's list starts empty
+    int count;
+    if (nreg > 0) {
+        if (threadIdx.x < 32) {  // exclusive prefix of the region counts, 32 at a time
+            int carry = 0;
+            for (int r0 = 0; r0 < nreg; r0 += 32) {
+                const int r = r0 + threadIdx.x;
+                const int c = r < nreg ? tie_regions[2 * r + 1] : 0;
+                if (r < nreg) start_s[r] = tie_regions[2 * r];
+                int x = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, x, o);
+                    if ((int)threadIdx.x >= o) x += y;
+                }
+                if (r < nreg) pre_s[r] = carry + x - c;
+                carry += __shfl_sync(0xffffffffu, x, 31);
+            }
+            if (threadIdx.x == 0) pre_s[nreg] = carry;
+        }
+        __syncthreads();
+        count = pre_s[nreg];
+    } else {
+        count = tie_count[it & 1];
+        if (blockIdx.x == 0 && threadIdx.x == 0) tie_count[(it + 1) & 1] = 0;  // the next pass's list starts empty
+    }
     const int lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     const int nblk = (N + KM_TOK - 1) / KM_TOK;
     const int words = (Cp + 31) >> 5;
-    for (int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; e < count; e += nwarps) {
+    for (int e0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; e0 < count; e0 += nwarps) {
+        int e = e0;
+        if (nreg > 0) {  // the region holding entry e0: the last r with pre_s[r] <= e0 (never an empty one)
+            int lo = 0, hi = nreg - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (pre_s[mid] <= e0) lo = mid; else hi = mid - 1;
+            }
+            e = start_s[lo] + e0 - pre_s[lo];
+        }
         const int4 hd = *reinterpret_cast<const int4*>(ties + e);  // bh, n, old, prov
         const int bh = hd.x, n = hd.y;
         float vx[CPL];
@@ -443,13 +1087,22 @@ __global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties,
                 }
             }
         }
-        if (lane == 0 && kbest != hd.w) {
-            labels[(size_t)bh * N + n] = kbest;
-            const int tile = n / KM_TOK;
-            atomicSub(&hist[((size_t)bh * C + hd.w) * nblk + tile], 1);
-            atomicAdd(&hist[((size_t)bh * C + kbest) * nblk + tile], 1);
-            const int dchg = (kbest != hd.z) - (hd.w != hd.z);
-            if (dchg != 0) atomicAdd(&state[bh].changed, dchg);
+        if (kbest != hd.w) {  // uniform over the warp: every lane holds the same sums
+            if (accumulate) {  // the token's channels move from the tensor-core cluster's sums to the new one's
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) {
+                    atomicAdd(&sums[((size_t)bh * C + hd.w) * D + lane * CPL + i], -(double)vx[i]);
+                    atomicAdd(&sums[((size_t)bh * C + kbest) * D + lane * CPL + i], (double)vx[i]);
+                }
+            }
+            if (lane == 0) {
+                labels[(size_t)bh * N + n] = kbest;
+                const int tile = n / KM_TOK;
+                atomicSub(&hist[((size_t)bh * C + hd.w) * nblk + tile], 1);
+                atomicAdd(&hist[((size_t)bh * C + kbest) * nblk + tile], 1);
+                const int dchg = (kbest != hd.z) - (hd.w != hd.z);
+                if (dchg != 0) atomicAdd(&state[bh].chg[it & 1], dchg);
+            }
         }
     }
 }
@@ -463,19 +1116,22 @@ constexpr int KM_SCAN_CHUNK = 16 * 1024;
 __global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist, int32_t* __restrict__ offs,
                                                 int32_t* __restrict__ cstart, int32_t* __restrict__ ccount,
                                                 KmState* __restrict__ state, int N, int C, int nblk, int it,
-                                                const int* __restrict__ status) {
+                                                int decide, const int* __restrict__ status) {
     extern __shared__ int h_s[];  // [KM_SCAN_CHUNK]
     __shared__ int s_part[1024];
     __shared__ int s_skip;
     if (ctl_failed(status)) return;
     const int bh = blockIdx.x, tid = threadIdx.x;
     if (tid == 0) {
-        int skip = state[bh].done;
-        if (!skip && it > 0 && state[bh].changed == 0) {
-            state[bh].done = 1;  // labels repeat the previous pass: perm is final
-            skip = 1;
+        int skip = 0;
+        if (decide) {  // per pass: a head whose labels repeat the previous pass is final
+            skip = state[bh].done;
+            if (!skip && it > 0 && state[bh].chg[it & 1] == 0) {
+                state[bh].done = 1;
+                skip = 1;
+            }
+            if (!skip) state[bh].chg[it & 1] = 0;  // for pass it + 2
         }
-        if (!skip) state[bh].changed = 0;
         s_skip = skip;
     }
     __syncthreads();
@@ -527,10 +1183,10 @@ __global__ void __launch_bounds__(1024) km_scan(const int32_t* __restrict__ hist
 __global__ void __launch_bounds__(KM_TOK) km_scatter(const int32_t* __restrict__ labels,
                                                      const int32_t* __restrict__ offs, int32_t* __restrict__ perm,
                                                      const KmState* __restrict__ state, int N, int C,
-                                                     const int* __restrict__ status) {
+                                                     int skip_done, const int* __restrict__ status) {
     __shared__ int cnt_s[KM_TOK / 32][256];
     const int bh = blockIdx.y, blk = blockIdx.x, nblk = gridDim.x, r = threadIdx.x;
-    if (ctl_failed(status) || state[bh].done) return;
+    if (ctl_failed(status) || (skip_done && state[bh].done)) return;
     const int warp = r >> 5, lane = r & 31;
     for (int i = r; i < (KM_TOK / 32) * 256; i += KM_TOK) (&cnt_s[0][0])[i] = 0;
     const int j = blk * KM_TOK + r;
@@ -616,18 +1272,44 @@ __global__ void __launch_bounds__(128) km_update(const __nv_bfloat16* __restrict
     }
 }
 
+// Lloyd update: c_k = sum / count in fp64 (empty clusters keep c_k), as bf16
+// hi/lo, fp32 |c_k|^2 and fp64 for km_refine; the sums are zeroed for the next
+// pass, or kept (keep_sums) when the next pass moves only the tokens that
+// change cluster.  The counts come from km_scan (ccount) or, after km_pass, from the
+// tile histograms; then the pass's change count also decides here whether
+// the head is final (its labels repeat the previous pass, so the centroids
+// would not move).
 __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __restrict__ c_lo,
                             float* __restrict__ cnorm, double* __restrict__ cent64, double* __restrict__ sums,
-                            const int32_t* __restrict__ ccount, const KmState* __restrict__ state, int C, int Cp,
-                            int D, const int* __restrict__ status) {
+                            const int32_t* __restrict__ ccount, const int32_t* __restrict__ hist,
+                            KmState* __restrict__ state, int C, int Cp, int D, int nblk, int it, int from_hist,
+                            int keep_sums, const int* __restrict__ status) {
     __shared__ float red[4];
+    __shared__ int red_i[4];
     const int k = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
     if (ctl_failed(status) || state[bh].done) return;
-    const int cnt = ccount[(size_t)bh * C + k];
+    int cnt;
+    if (from_hist) {
+        // every CTA of the head reads the same count (no one writes it during this kernel)
+        if (it >= 1 && state[bh].chg[it & 1] == 0) {
+            if (k == 0 && c == 0) state[bh].done = 1;
+            return;
+        }
+        if (k == 0 && c == 0) state[bh].chg[(it + 1) & 1] = 0;  // read last by the previous pass's finalize
+        int part = 0;
+        for (int t = c; t < nblk; t += D) part += hist[((size_t)bh * C + k) * nblk + t];
+        part = __reduce_add_sync(0xffffffffu, part);
+        if ((c & 31) == 0) red_i[c >> 5] = part;
+        __syncthreads();
+        cnt = 0;
+        for (int w = 0; w < (D >> 5); ++w) cnt += red_i[w];
+    } else {
+        cnt = ccount[(size_t)bh * C + k];
+    }
     if (cnt == 0) return;  // an empty cluster keeps its centroid (sums are still 0)
     double* sp = &sums[((size_t)bh * C + k) * D + c];
     const double mean = __ddiv_rn(*sp, (double)cnt);  // the fp64 member mean
-    *sp = 0.0;
+    if (!keep_sums) *sp = 0.0;
     cent64[((size_t)bh * C + k) * D + c] = mean;
     const size_t row = ((size_t)bh * Cp + k) * D + c;
     const __nv_bfloat16 h = __double2bfloat16(mean);
@@ -970,6 +1652,8 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     if (!configured.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(km_pass<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(km_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, KM_SCAN_CHUNK * sizeof(int));
         if (e != cudaSuccess) return e;
         configured.mark(dev);
@@ -981,21 +1665,48 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
         return cudaErrorInvalidValue;
     km_init<<<dim3(Cp, p.BH), D, 0, s>>>(p.V, p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.state, p.vamax, p.tie_count, p.N, p.C,
                                          Cp, D);
+    if (p.C <= 64) {
+        // One fused pass a sweep (the member sums fit in shared memory); the
+        // regroup is built once, from the last labels.
+        const KpLayout kl(D, Cp);
+        const int grid = sms < KP_MAX_GRID ? sms : KP_MAX_GRID;
+        int* regions = p.tie_count + 2;
+        for (int it = 0; it < p.iters; ++it) {
+            // the first two passes add every token (most labels still move);
+            // later ones move the few tokens that change; the last needs no sums
+            const int mode = it + 1 == p.iters ? 0 : (it < 2 ? 1 : 2);
+            km_pass<D><<<grid, KP_THREADS, kl.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels, p.hist, p.sums,
+                                                           p.ties, regions, p.state, p.BH, p.N, p.C, Cp, it, mode,
+                                                           p.ctl);
+            km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, regions, grid, p.V, p.cent64, p.labels,
+                                                  p.hist, p.sums, p.state, p.N, p.C, Cp, it, mode != 0,
+                                                  p.ctl.status);
+            if (mode != 0)  // the sums stay for a following pass that moves changed tokens only
+                km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.ccount,
+                                                          p.hist, p.state, p.C, Cp, D, nblk, it, 1, it + 1 >= 2,
+                                                          p.ctl.status);
+        }
+        km_scan<<<p.BH, 1024, KM_SCAN_CHUNK * sizeof(int), s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N,
+                                                                 p.C, nblk, p.iters - 1, 0, p.ctl.status);
+        km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C, 0,
+                                                       p.ctl.status);
+        return cudaGetLastError();
+    }
     for (int it = 0; it < p.iters; ++it) {
         km_assign<D><<<dim3(nchunk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.vnorm2, p.labels,
                                                             p.hist, p.ties, p.tie_count, p.state, p.N, p.C, Cp,
                                                             it, tpc, p.ctl);
-        km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, p.V, p.cent64, p.labels, p.hist, p.state, p.N,
-                                              p.C, Cp, it, p.ctl.status);
-        km_scan<<<p.BH, 1024, KM_SCAN_CHUNK * sizeof(int), s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N, p.C, nblk, it,
-                                      p.ctl.status);
-        km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C,
+        km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, nullptr, 0, p.V, p.cent64, p.labels, p.hist,
+                                              p.sums, p.state, p.N, p.C, Cp, it, 0, p.ctl.status);
+        km_scan<<<p.BH, 1024, KM_SCAN_CHUNK * sizeof(int), s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N,
+                                                                 p.C, nblk, it, 1, p.ctl.status);
+        km_scatter<<<dim3(nblk, p.BH), KM_TOK, 0, s>>>(p.labels, p.offs, p.perm, p.state, p.N, p.C, 1,
                                                        p.ctl.status);
         if (it + 1 < p.iters) {
             km_update<D><<<dim3((p.N + KM_UPD_ROWS - 1) / KM_UPD_ROWS, p.BH), 128, 0, s>>>(
                 p.V, p.perm, p.cstart, p.sums, p.state, p.N, p.C, p.ctl.status);
-            km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.ccount, p.state,
-                                                      p.C, Cp, D, p.ctl.status);
+            km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.ccount, p.hist,
+                                                      p.state, p.C, Cp, D, nblk, it, 0, 0, p.ctl.status);
         }
     }
     return cudaGetLastError();

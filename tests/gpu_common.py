@@ -93,8 +93,9 @@ def oracle_prep_on_perm(k_bits, v_bits, perm, bk, smooth=True, resid_fmt=0):
 
 
 # k-means decisions the tensor-core distance leaves open are re-decided in
-# fp64 when two clusters lie within this fraction of (|v| + max|c|)^2.
-KMEANS_MARGIN = 2.0 ** -12
+# fp64 when two clusters lie within this fraction of (|v| + max|c|)^2 (the
+# library's near-tie margin).
+KMEANS_MARGIN = 2.0 ** -13
 
 
 def check_labels_valid(v_bits, gpu_labels, ref_labels, centroids):
