@@ -409,18 +409,23 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
 // and add it to the new one's, fp64 atomics): exact like a fresh sum, and
 // cheap once few labels change.  Mode 0 (the last pass) writes labels and
 // histograms only.
-// Warps: 0 TMA producer (V tiles through a 3-stage ring; a head's centroids
-// when the CTA enters it), 1 MMA issuer (tile i into accumulator i % 2 in
-// TMEM), then KP_GROUPS assignment groups of four warps (group g takes the
-// CTA's tiles i = g mod KP_GROUPS; a thread per token), then 8 update warps
-// (D/32 channels a lane).
-constexpr int KP_GROUPS = 1;
-constexpr int KP_STAGES = 3;
-constexpr int KP_SEG = 68;      // per stage: 65 cluster offsets, padded
-constexpr int KP_UPD = 8;       // update warps
-constexpr int KP_ASG = 4 * KP_GROUPS;  // assignment warps
-constexpr int KP_THREADS = 32 * (2 + KP_ASG + KP_UPD);
+// Warps: 0 TMA producer (V tiles through a ring of stages; a head's centroids
+// when the CTA enters it), 1 MMA issuer (tile i into TMEM accumulator
+// i % kAcc), then G assignment groups of four warps (group g takes the CTA's
+// tiles i = g mod G; a thread per token), then, in the shape that sums every
+// token, 8 update warps (D/32 channels a lane).  Passes that move changed
+// tokens only run three assignment groups and no update warps.
+constexpr int KP_SEG = 68;  // per stage: 65 cluster offsets, padded
 constexpr int KP_MAX_GRID = kKmTieRegions;  // near-tie regions the workspace holds
+
+template <int G, bool UPD>
+struct KpShape {
+    static constexpr int kGroups = G;
+    static constexpr int kUpd = UPD ? 8 : 0;  // update warps
+    static constexpr int kStages = UPD ? 3 : 4;
+    static constexpr int kAcc = G < 2 ? 2 : G;  // TMEM accumulators
+    static constexpr int kThreads = 32 * (2 + 4 * G + kUpd);
+};
 
 // Shared-memory plan of km_pass, from a 1024-byte aligned base:
 //   V ring | centroid hi | centroid lo | fp64 sums [64][D] | |c|^2 per group |
@@ -429,21 +434,21 @@ constexpr int KP_MAX_GRID = kKmTieRegions;  // near-tie regions the workspace ho
 struct KpLayout {
     uint32_t v_bytes, c_bytes, off_v, off_chi, off_clo, off_sum, off_cn, off_ord, off_slab, off_seg, off_cnt, off_misc,
         off_bar, bytes;
-    __host__ __device__ KpLayout(int D, int Cp) {
+    __host__ __device__ KpLayout(int D, int Cp, int S, int G, int nacc, bool with_sums) {
         v_bytes = KM_TOK * D * 2;
         c_bytes = Cp * D * 2;
         off_v = 0;
-        off_chi = off_v + KP_STAGES * v_bytes;
+        off_chi = off_v + S * v_bytes;
         off_clo = off_chi + c_bytes;
-        off_sum = off_clo + c_bytes;                 // [64][D] double
-        off_cn = off_sum + 64 * D * 8;               // [2][64] float
-        off_ord = off_cn + 2 * 64 * 4;               // [stage][128] tile rows grouped by cluster
-        off_slab = off_ord + KP_STAGES * KM_TOK;     // [stage][128] their clusters
-        off_seg = off_slab + KP_STAGES * KM_TOK;     // [stage][KP_SEG] first grouped position of each cluster
-        off_cnt = off_seg + KP_STAGES * KP_SEG * 4;  // [2][2][64] label counts of a group's tile
-        off_misc = off_cnt + 2 * 2 * 64 * 4;         // [16] ints, see km_pass
+        off_sum = off_clo + c_bytes;                      // [64][D] double (the shape with update warps)
+        off_cn = off_sum + (with_sums ? 64 * D * 8 : 0);  // [G][64] float, then [G] max |c|^2 bits
+        off_ord = off_cn + ((G * 65 * 4 + 15) & ~15);     // [stage][128] tile rows grouped by cluster
+        off_slab = off_ord + S * KM_TOK;                  // [stage][128] their clusters
+        off_seg = off_slab + S * KM_TOK;                  // [stage][KP_SEG] first grouped position of each cluster
+        off_cnt = off_seg + S * KP_SEG * 4;               // [G][2][64] label counts of a group's tile
+        off_misc = off_cnt + G * 2 * 64 * 4;              // [16] ints, see km_pass
         off_bar = off_misc + 64;
-        bytes = off_bar + 8 * (3 * KP_STAGES + 7) + 1024;  // + alignment slack
+        bytes = off_bar + 8 * (3 * S + 2 * nacc + 3) + 1024;  // + alignment slack
     }
 };
 
@@ -490,26 +495,26 @@ __device__ __forceinline__ double bf16lo_scaled(uint32_t w) {  // bits 0..15 of 
     return bf16hi_scaled(w << 16);
 }
 
-template <int D>
-__global__ void __launch_bounds__(KP_THREADS, 1)
+template <int D, int G, bool UPD>
+__global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
     km_pass(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_chi,
             const __grid_constant__ CUtensorMap tm_clo, const float* __restrict__ cnorm, float* __restrict__ vnorm2,
             int32_t* __restrict__ labels, int32_t* __restrict__ hist, double* __restrict__ sums,
             KmTie* __restrict__ ties, int* __restrict__ tie_regions, KmState* __restrict__ state, int BH, int N,
             int C, int Cp, int it, int mode, DevCtl ctl) {
-    constexpr int S = KP_STAGES;
-    const bool accumulate = mode == 1;
+    using Shape = KpShape<G, UPD>;
+    constexpr int S = Shape::kStages, NACC = Shape::kAcc, ASG = 4 * G;
+    const bool accumulate = UPD && mode == 1;
     if (ctl_failed(ctl.status)) return;
     const int nblk = (N + KM_TOK - 1) / KM_TOK;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
-    const KpLayout L(D, Cp);
+    const KpLayout L(D, Cp, S, G, NACC, UPD);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // scratch: [0] TMEM base, [1] abort flag, [2..3] max |c|^2 bits of each
-    // group's head, [4] units, [5] first head, [6] first tile, [7] near ties
-    // listed, [8] near-tie region start
+    // scratch: [0] TMEM base, [1] abort flag, [4] units, [5] first head,
+    // [6] first tile, [7] near ties listed, [8] near-tie region start
     int* misc = reinterpret_cast<int*>(smem + L.off_misc);
     volatile int* abort_flag = misc + 1;
     int* tie_s = misc + 7;
@@ -519,16 +524,16 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
     auto b_vempty = [&](int st) { return bar0 + 8u * (S + st); };
     auto b_lfull = [&](int st) { return bar0 + 8u * (2 * S + st); };
     auto b_accfull = [&](int b) { return bar0 + 8u * (3 * S + b); };
-    auto b_accempty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
-    const uint32_t b_cfull = bar0 + 8u * (3 * S + 4), b_cempty = b_cfull + 8, b_mmadone = b_cfull + 16;
+    auto b_accempty = [&](int b) { return bar0 + 8u * (3 * S + NACC + b); };
+    const uint32_t b_cfull = bar0 + 8u * (3 * S + 2 * NACC), b_cempty = b_cfull + 8, b_mmadone = b_cfull + 16;
     if (tid == 0) {
         for (int st = 0; st < S; ++st) {
             mbar_init(b_vfull(st), 1);
             // the MMA warp's commit, the 4 warps of the assignment group, the update warps
-            mbar_init(b_vempty(st), 1 + 4 + (accumulate ? KP_UPD : 0));
+            mbar_init(b_vempty(st), 1 + 4 + (accumulate ? Shape::kUpd : 0));
             mbar_init(b_lfull(st), 4);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NACC; ++b) {
             mbar_init(b_accfull(b), 1);
             mbar_init(b_accempty(b), 4);
         }
@@ -539,11 +544,11 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
         *tie_s = 0;
         fence_mbar_init();
     }
-    for (int i = tid; i < 2 * 2 * 64; i += blockDim.x) cnt_s[i] = 0;
+    for (int i = tid; i < G * 2 * 64; i += blockDim.x) cnt_s[i] = 0;
     double* sums_s = reinterpret_cast<double*>(smem + L.off_sum);
     if (accumulate)
         for (int i = tid; i < 64 * D; i += blockDim.x) sums_s[i] = 0.0;
-    const uint32_t ncols = 2 * Cp <= 32 ? 32 : (2 * Cp <= 64 ? 64 : 128);
+    const uint32_t ncols = NACC * Cp <= 32 ? 32 : (NACC * Cp <= 64 ? 64 : (NACC * Cp <= 128 ? 128 : 256));
     if (warp == 1) {
         tmem_alloc(smem_u32(reinterpret_cast<uint32_t*>(misc)), ncols);
         tmem_relinquish();
@@ -631,9 +636,9 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
                     cur = w.bh;
                     if (!mbar_wait(b_cfull, hs & 1, ctl, abort_flag)) break;
                 }
-                const int st = i % S, b = i & 1;
+                const int st = i % S, b = i % NACC;
                 if (!mbar_wait(b_vfull(st), (i / S) & 1, ctl, abort_flag)) break;
-                if (i >= 2 && !mbar_wait(b_accempty(b), ((i >> 1) - 1) & 1, ctl, abort_flag)) break;
+                if (i >= NACC && !mbar_wait(b_accempty(b), ((i / NACC) - 1) & 1, ctl, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t sA = base + L.off_v + st * L.v_bytes, acc = tmem + b * Cp;
 #pragma unroll
@@ -654,15 +659,16 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
             mma_commit(b_mmadone);  // every MMA issued has finished before TMEM is released
             drain_wait(b_mmadone, 0, ctl);
         }
-    } else if (warp < 2 + KP_ASG) {
+    } else if (warp < 2 + ASG) {
         // ------------------------------------------------------------ assignment (thread per token)
-        // Group g takes tiles i = g, g + KP_GROUPS, ...  TMEM lane quadrant
-        // q = warp % 4 holds tile rows 32q..32q+31.
+        // Group g takes tiles i = g, g + G, ...  TMEM lane quadrant q = warp % 4
+        // holds tile rows 32q..32q+31.
         const int g = (warp - 2) >> 2;
         const int qd = warp & 3;
         const int r = qd * 32 + lane;
         const int bar_id = 1 + g;
         float* cn_s = reinterpret_cast<float*>(smem + L.off_cn) + g * 64;
+        uint32_t* cmax_s = reinterpret_cast<uint32_t*>(smem + L.off_cn) + G * 64 + g;
         uint8_t* ord_s = smem + L.off_ord;
         uint8_t* slab_s = smem + L.off_slab;
         int* seg_s = reinterpret_cast<int*>(smem + L.off_seg);
@@ -690,7 +696,7 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
             }
         };
         if (g < nunits) fetch(w);
-        for (int i = g; i < nunits; i += KP_GROUPS) {
+        for (int i = g; i < nunits; i += G) {
             const int bh = w.bh, tile = w.tile;
             if (bh != cur) {  // |c_k|^2 of the new head (pad clusters +inf, never chosen), max_k |c_k|^2
                 if (cur >= 0) flush_changed();
@@ -706,22 +712,22 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
                         if (k < C) mb = max(mb, __float_as_uint(x));  // x >= 0: bit order is value order
                     }
                     mb = __reduce_max_sync(0xffffffffu, mb);
-                    if (lane == 0) misc[2 + g] = (int)mb;
+                    if (lane == 0) *cmax_s = mb;
                 }
                 named_barrier_sync(bar_id, 128);
-                cmax_r = sqrtf(__uint_as_float((uint32_t)misc[2 + g]));
+                cmax_r = sqrtf(__uint_as_float(*cmax_s));
             }
             const int32_t old_label = nxt_old;
             float vn2 = nxt_vn2;
 #pragma unroll
-            for (int q = 0; q < KP_GROUPS; ++q) w.next(state, BH, nblk);  // this group's next tile
-            if (i + KP_GROUPS < nunits) fetch(w);
-            const int st = i % S, b = i & 1;
-            int* cnt = cnt_s + (g * 2 + ((i / KP_GROUPS) & 1)) * 64;  // this tile's label counts
+            for (int q = 0; q < G; ++q) w.next(state, BH, nblk);  // this group's next tile
+            if (i + G < nunits) fetch(w);
+            const int st = i % S, b = i % NACC;
+            int* cnt = cnt_s + (g * 2 + ((i / G) & 1)) * 64;  // this tile's label counts
             const int n = tile * KM_TOK + r;
             const bool valid = n < N;
             // the accumulator of tile i (its MMA also means V tile i has landed)
-            const bool okj = warp_wait(b_accfull(b), (i >> 1) & 1, ctl, abort_flag);
+            const bool okj = warp_wait(b_accfull(b), (i / NACC) & 1, ctl, abort_flag);
             int label = 0, rank = 0;
             if (okj) {
                 tc_fence_after();
@@ -754,7 +760,7 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(b_accempty(b));  // the accumulator is free for tile i + 2
+                if (lane == 0) mbar_arrive(b_accempty(b));  // the accumulator is free for tile i + NACC
                 // best and runner-up of d_k = |c_k|^2 - 2 v.c_k, four chains (k % 4)
                 float b4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
                 float s4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
@@ -879,10 +885,10 @@ __global__ void __launch_bounds__(KP_THREADS, 1)
             if (lane == 0) mbar_arrive(b_vempty(st));
         }
         if (cur >= 0) flush_changed();
-    } else if (accumulate && nunits > 0) {
+    } else if (UPD && accumulate && nunits > 0) {
         // ------------------------------------------------------------ update, mode 1 (D/32 channels a lane)
         constexpr int NCH = D / 32;
-        const int u = warp - 2 - KP_ASG;        // clusters 8u .. 8u + 7
+        const int u = warp - 2 - ASG;           // clusters 8u .. 8u + 7
         const int c0 = NCH * lane;              // channels c0 .. c0 + NCH - 1
         const int kc = c0 >> 6, q16 = (c0 & 63) >> 3, wo = (c0 & 7) * 2;  // chunk, 16-byte piece, byte
         const uint8_t* ord_s = smem + L.off_ord;
@@ -1652,7 +1658,9 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     if (!configured.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(km_pass<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(km_pass<D, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(km_pass<D, 3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(km_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, KM_SCAN_CHUNK * sizeof(int));
         if (e != cudaSuccess) return e;
@@ -1668,16 +1676,23 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     if (p.C <= 64) {
         // One fused pass a sweep (the member sums fit in shared memory); the
         // regroup is built once, from the last labels.
-        const KpLayout kl(D, Cp);
+        using Sum = KpShape<1, true>;   // passes that sum every token
+        using Move = KpShape<3, false>;  // passes that move changed tokens, and the last
+        const KpLayout ls(D, Cp, Sum::kStages, 1, Sum::kAcc, true), lm(D, Cp, Move::kStages, 3, Move::kAcc, false);
         const int grid = sms < KP_MAX_GRID ? sms : KP_MAX_GRID;
         int* regions = p.tie_count + 2;
         for (int it = 0; it < p.iters; ++it) {
             // the first two passes add every token (most labels still move);
             // later ones move the few tokens that change; the last needs no sums
             const int mode = it + 1 == p.iters ? 0 : (it < 2 ? 1 : 2);
-            km_pass<D><<<grid, KP_THREADS, kl.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels, p.hist, p.sums,
-                                                           p.ties, regions, p.state, p.BH, p.N, p.C, Cp, it, mode,
-                                                           p.ctl);
+            if (mode == 1)
+                km_pass<D, 1, true><<<grid, Sum::kThreads, ls.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels,
+                                                                         p.hist, p.sums, p.ties, regions, p.state,
+                                                                         p.BH, p.N, p.C, Cp, it, mode, p.ctl);
+            else
+                km_pass<D, 3, false><<<grid, Move::kThreads, lm.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels,
+                                                                           p.hist, p.sums, p.ties, regions, p.state,
+                                                                           p.BH, p.N, p.C, Cp, it, mode, p.ctl);
             km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, regions, grid, p.V, p.cent64, p.labels,
                                                   p.hist, p.sums, p.state, p.N, p.C, Cp, it, mode != 0,
                                                   p.ctl.status);
