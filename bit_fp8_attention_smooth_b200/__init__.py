@@ -71,6 +71,7 @@ def lib():
             "vc_check": (ctypes.c_int, [P, P]),
             "vc_attn_fwd_noalloc": (ctypes.c_int, [P, PR, PS, PP, P, P]),
             "vc_e4m3_encode": (ctypes.c_int, [P, P, i64, P]),
+            "vc_quantize_q": (ctypes.c_int, [P, P, P, i64, ctypes.c_int, P]),
             "vc_expcast_bytes": (ctypes.c_int, [P, P, P, P, i64, P]),
         }
         for name, (res, args) in sig.items():
@@ -373,6 +374,19 @@ def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
     out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _ok(lib().vc_e4m3_encode(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)), "vc_e4m3_encode")
     return out
+
+
+def quantize_q(q: torch.Tensor, stream=None):
+    """Per-token E4M3 Q as the attention call quantises it: q bf16 [..., d] ->
+    (codes uint8 [..., d], scales fp32 [...])."""
+    if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous() or q.dim() < 1:
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    d = q.shape[-1]
+    codes = torch.empty(q.shape, dtype=torch.uint8, device=q.device)
+    scales = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    _ok(lib().vc_quantize_q(q.data_ptr(), codes.data_ptr(), scales.data_ptr(), q.numel() // max(d, 1), d,
+                            _stream(stream)), "vc_quantize_q")
+    return codes, scales
 
 
 def expcast_bytes(A: torch.Tensor, s: torch.Tensor, cb: torch.Tensor, stream=None) -> torch.Tensor:

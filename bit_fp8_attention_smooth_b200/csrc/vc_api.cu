@@ -453,6 +453,19 @@ vc_status vc_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream) 
                                                                                                 : VC_ERR_CUDA;
 }
 
+vc_status vc_quantize_q(const void* Q, uint8_t* q_fp8, float* sq, int64_t tokens, int d, void* stream) {
+    if (tokens < 0) return VC_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return VC_ERR_UNSUPPORTED;
+    if (tokens == 0) return VC_OK;
+    if (!aligned16(Q) || !aligned16(q_fp8) || !sq || (reinterpret_cast<uintptr_t>(sq) & 3u)) return VC_ERR_INVALID_ARG;
+    vc_status st = check_device();
+    if (st != VC_OK) return st;
+    return vc::launch_quant_q(static_cast<const __nv_bfloat16*>(Q), q_fp8, sq, tokens, d,
+                              static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? VC_OK
+               : VC_ERR_CUDA;
+}
+
 vc_status vc_expcast_bytes(const float* A, const float* s, const float* cb, uint8_t* out, int64_t n, void* stream) {
     if (n < 0 || (n > 0 && (!A || !s || !cb || !out))) return VC_ERR_INVALID_ARG;
     vc_status st = check_device();

@@ -990,17 +990,31 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
     }
 }
 
-// fp64 decision of the near ties km_assign or km_pass listed: one warp a token, each
-// candidate's squared distance summed over D/32 channels a lane in fp64 and
-// added across the warp; candidates in ascending cluster order with a strict
-// comparison, so equal distances keep the lowest cluster (as the Lloyd step's
-// argmin).  When the decision differs from the tensor-core label, the label,
-// the tile's cluster counts and the head's change count are corrected.
-// The list is either one run counted in tie_count[it % 2] (km_assign) or, with
-// nreg > 0, km_pass's per-CTA regions: (start, count) pairs in tie_regions.
+// Decision of the near ties km_assign or km_pass listed, by the Lloyd step's
+// own distance (the fp64 sum over channels of (v - c)^2, argmin with equal
+// distances keeping the lowest cluster).  When the decision differs from the
+// tensor-core label, the label, the tile's cluster counts, the head's change
+// count and (when the sums are kept) the sums are corrected.  The list is
+// either one run counted in tie_count[it % 2] (km_assign) or, with nreg > 0,
+// km_pass's per-CTA regions: (start, count) pairs in tie_regions.
+//
+// Most ties are settled first in fp32 from the bf16 hi/lo centroids.
+// c32 = hi + lo lies within 2^-17.9 |c_i| of the fp64 centroid in every
+// channel (two bf16 roundings, and the fp32 sum), so D(c32) is within
+// 2^-16.9 sqrt(D) |c| + 2^-35.8 |c|^2 of D(c); the fp32 evaluation
+// (differences, then d/8 fused multiply-adds a lane and a three-level
+// butterfly: at most 20 roundings on any term) adds at most 2^-19.6 D.  With
+// each term doubled, E = 2^-16 sqrt(D32) |c| + 2^-35 |c|^2 + 2^-18 D32 bounds
+// |D32 - D|.  A candidate whose D32 + E is below every other candidate's
+// D32 - E is the exact argmin; otherwise all candidates are compared in fp64
+// from the fp64 centroids, in ascending cluster order with a strict
+// comparison.
 template <int D>
 __global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties, int* __restrict__ tie_count,
                                                  const int* __restrict__ tie_regions, int nreg,
+                                                 const __nv_bfloat16* __restrict__ c_hi,
+                                                 const __nv_bfloat16* __restrict__ c_lo,
+                                                 const float* __restrict__ cnorm,
                                                  const __nv_bfloat16* __restrict__ V,
                                                  const double* __restrict__ cent64, int32_t* __restrict__ labels,
                                                  int32_t* __restrict__ hist, double* __restrict__ sums,
@@ -1009,7 +1023,6 @@ __global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties,
     __shared__ int pre_s[KP_MAX_GRID + 1];  // entries before each region
     __shared__ int start_s[KP_MAX_GRID];
     if (ctl_failed(status)) return;
-    constexpr int CPL = D / 32;  // channels a lane
     int count;
     if (nreg > 0) {
         if (threadIdx.x < 32) {  // exclusive prefix of the region counts, 32 at a time
@@ -1035,13 +1048,21 @@ __global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties,
         count = tie_count[it & 1];
         if (blockIdx.x == 0 && threadIdx.x == 0) tie_count[(it + 1) & 1] = 0;  // the next pass's list starts empty
     }
-    const int lane = threadIdx.x & 31;
+    // Four ties a warp, eight lanes a tie (D/8 channels a lane): four ties'
+    // loads in flight at once.  Loops over candidate slots run the same count
+    // on every lane (the warp's largest candidate count), so every shuffle
+    // is reached by all 32 lanes.
+    constexpr int TL = 8, TPW = 32 / TL, CPT = D / TL;
+    const int lane = threadIdx.x & 31, sub = lane / TL, sl = lane % TL;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nblk = (N + KM_TOK - 1) / KM_TOK;
     const int words = (Cp + 31) >> 5;
-    for (int e0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; e0 < count; e0 += nwarps) {
+    for (int base = gw * TPW; base < count; base += nwarps * TPW) {
+        const int e0 = base + sub;
+        const bool act = e0 < count;
         int e = e0;
-        if (nreg > 0) {  // the region holding entry e0: the last r with pre_s[r] <= e0 (never an empty one)
+        if (act && nreg > 0) {  // the region holding entry e0: the last r with pre_s[r] <= e0 (never an empty one)
             int lo = 0, hi = nreg - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
@@ -1049,59 +1070,119 @@ __global__ void __launch_bounds__(256) km_refine(const KmTie* __restrict__ ties,
             }
             e = start_s[lo] + e0 - pre_s[lo];
         }
-        const int4 hd = *reinterpret_cast<const int4*>(ties + e);  // bh, n, old, prov
+        const int4 hd = act ? *reinterpret_cast<const int4*>(ties + e) : make_int4(0, 0, -1, -1);  // bh, n, old, prov
         const int bh = hd.x, n = hd.y;
-        float vx[CPL];
+        float vx[CPT];
         {
-            const __nv_bfloat16* vp = V + ((size_t)bh * N + n) * D + lane * CPL;
-            if constexpr (CPL == 4) {
-                const uint2 raw = __ldg(reinterpret_cast<const uint2*>(vp));
-                const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+            const uint4* vp = reinterpret_cast<const uint4*>(V + ((size_t)bh * N + n) * D + sl * CPT);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) vx[i] = bf2f(h[i]);
-            } else {
-                const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(vp));
-                const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+            for (int q = 0; q < CPT / 8; ++q) {
+                const uint4 x = act ? __ldg(vp + q) : make_uint4(0, 0, 0, 0);
+                const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) vx[i] = bf2f(h[i]);
+                for (int h = 0; h < 4; ++h) {
+                    vx[8 * q + 2 * h] = __uint_as_float(w4[h] << 16);
+                    vx[8 * q + 2 * h + 1] = __uint_as_float(w4[h] & 0xFFFF0000u);
+                }
             }
         }
-        double dbest = INFINITY;
-        int kbest = hd.w;
-        for (int w = 0; w < words; ++w) {
-            for (uint32_t m = ties[e].mask[w]; m; m &= m - 1) {
-                const int k = 32 * w + __ffs(m) - 1;
-                const double2* cp = reinterpret_cast<const double2*>(cent64 + ((size_t)bh * C + k) * D + lane * CPL);
-                double cx[CPL];
+        int nc = 0;
+        for (int w = 0; act && w < words; ++w) nc += __popc(ties[e].mask[w]);
+        const int ncmax = __reduce_max_sync(0xffffffffu, nc);
+        // fp32 bounds of every candidate's distance (uniform over the tie's lanes)
+        float umin = INFINITY, lmin1 = INFINITY, lmin2 = INFINITY;
+        int ku = -1, kl1 = -1;
+        int cw = 0;
+        uint32_t bits = act ? ties[e].mask[0] : 0u;
+        for (int j = 0; j < ncmax; ++j) {
+            while (bits == 0 && act && cw + 1 < words) bits = ties[e].mask[++cw];
+            const bool has = bits != 0;
+            const int k = has ? 32 * cw + __ffs(bits) - 1 : 0;
+            bits &= bits - 1;
+            float part = 0.0f;
+            if (has) {
+                const size_t row = ((size_t)bh * Cp + k) * D + sl * CPT;
 #pragma unroll
-                for (int i = 0; i < CPL / 2; ++i) {
-                    const double2 c2 = __ldg(cp + i);
-                    cx[2 * i] = c2.x;
-                    cx[2 * i + 1] = c2.y;
+                for (int q = 0; q < CPT / 8; ++q) {
+                    const uint4 h4 = __ldg(reinterpret_cast<const uint4*>(c_hi + row) + q);
+                    const uint4 l4 = __ldg(reinterpret_cast<const uint4*>(c_lo + row) + q);
+                    const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w}, lw[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float c0 = __fadd_rn(__uint_as_float(hw[h] << 16), __uint_as_float(lw[h] << 16));
+                        const float c1 = __fadd_rn(__uint_as_float(hw[h] & 0xFFFF0000u),
+                                                   __uint_as_float(lw[h] & 0xFFFF0000u));
+                        const float d0 = __fsub_rn(vx[8 * q + 2 * h], c0);
+                        const float d1 = __fsub_rn(vx[8 * q + 2 * h + 1], c1);
+                        part = __fmaf_rn(d0, d0, part);
+                        part = __fmaf_rn(d1, d1, part);
+                    }
                 }
+            }
+#pragma unroll
+            for (int o = TL / 2; o > 0; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+            if (has) {
+                const float c2 = cnorm[(size_t)bh * Cp + k];
+                const float err = 0x1p-16f * sqrtf(part * c2) + 0x1p-35f * c2 + 0x1p-18f * part;
+                const float up = part + err, lo = part - err;
+                if (up < umin) {
+                    umin = up;
+                    ku = k;
+                }
+                if (lo < lmin1) {
+                    lmin2 = lmin1;
+                    lmin1 = lo;
+                    kl1 = k;
+                } else if (lo < lmin2) {
+                    lmin2 = lo;
+                }
+            }
+        }
+        // the fp32 winner is certain when its upper bound is below every other lower bound
+        const bool sure = ku >= 0 && umin < (kl1 == ku ? lmin2 : lmin1);
+        int kbest = sure ? ku : hd.w;
+        const bool need = act && !sure;
+        if (__any_sync(0xffffffffu, need)) {
+            // fp64 decision: candidates in ascending order, strict comparison
+            // (equal distances keep the lowest cluster, as the Lloyd argmin)
+            double dbest = INFINITY;
+            cw = 0;
+            bits = need ? ties[e].mask[0] : 0u;
+            for (int j = 0; j < ncmax; ++j) {
+                while (bits == 0 && need && cw + 1 < words) bits = ties[e].mask[++cw];
+                const bool has = bits != 0;
+                const int k = has ? 32 * cw + __ffs(bits) - 1 : 0;
+                bits &= bits - 1;
                 double part = 0.0;
+                if (has) {
+                    const double2* cp =
+                        reinterpret_cast<const double2*>(cent64 + ((size_t)bh * C + k) * D + sl * CPT);
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) {
-                    const double diff = __dsub_rn((double)vx[i], cx[i]);
-                    part = __dadd_rn(part, __dmul_rn(diff, diff));
+                    for (int i = 0; i < CPT / 2; ++i) {
+                        const double2 c2 = __ldg(cp + i);
+                        const double d0 = __dsub_rn((double)vx[2 * i], c2.x);
+                        const double d1 = __dsub_rn((double)vx[2 * i + 1], c2.y);
+                        part = __dadd_rn(part, __dmul_rn(d0, d0));
+                        part = __dadd_rn(part, __dmul_rn(d1, d1));
+                    }
                 }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
-                if (part < dbest) {
+                for (int o = TL / 2; o > 0; o >>= 1) part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+                if (has && part < dbest) {
                     dbest = part;
                     kbest = k;
                 }
             }
         }
-        if (kbest != hd.w) {  // uniform over the warp: every lane holds the same sums
+        if (act && kbest != hd.w) {  // uniform over the tie's lanes
             if (accumulate) {  // the token's channels move from the tensor-core cluster's sums to the new one's
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) {
-                    atomicAdd(&sums[((size_t)bh * C + hd.w) * D + lane * CPL + i], -(double)vx[i]);
-                    atomicAdd(&sums[((size_t)bh * C + kbest) * D + lane * CPL + i], (double)vx[i]);
+                for (int i = 0; i < CPT; ++i) {
+                    atomicAdd(&sums[((size_t)bh * C + hd.w) * D + sl * CPT + i], -(double)vx[i]);
+                    atomicAdd(&sums[((size_t)bh * C + kbest) * D + sl * CPT + i], (double)vx[i]);
                 }
             }
-            if (lane == 0) {
+            if (sl == 0) {
                 labels[(size_t)bh * N + n] = kbest;
                 const int tile = n / KM_TOK;
                 atomicSub(&hist[((size_t)bh * C + hd.w) * nblk + tile], 1);
@@ -1398,9 +1479,18 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat1
     const __nv_bfloat16* ksh = reinterpret_cast<const __nv_bfloat16*>(ks);
     const __nv_bfloat16* vsh = reinterpret_cast<const __nv_bfloat16*>(vs);
     const int c = tid % D, rg = tid / D;
-    double vsum = 0.0;
-    for (int r = rg; r < valid; r += RG) vsum += (double)bf2f(vsh[r * D + c]);
-    vsum_s[rg][c] = vsum;
+    // The channel's sum over the block in fp64, four partial sums of the
+    // bf16 values placed as v * 2^-896 (exact, see bf16lo_scaled); scaled
+    // back once below.  Exact additions make the order irrelevant.
+    const uint16_t* vbits = reinterpret_cast<const uint16_t*>(vs);
+    double vp[4] = {0.0, 0.0, 0.0, 0.0};
+    int r = rg;
+    for (; r + 3 * RG < valid; r += 4 * RG) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) vp[e] += bf16lo_scaled(vbits[(r + e * RG) * D + c]);
+    }
+    for (; r < valid; r += RG) vp[0] += bf16lo_scaled(vbits[r * D + c]);
+    vsum_s[rg][c] = (vp[0] + vp[1]) + (vp[2] + vp[3]);
     // K codes, four channels a thread (one 32-bit store); padding rows are 0
     uint32_t* kout = reinterpret_cast<uint32_t*>(k_fp8 + ((size_t)bh * T * BK + (size_t)b * BK) * D);
 #pragma unroll 4
@@ -1419,11 +1509,17 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat1
     double tot = 0.0;
 #pragma unroll
     for (int q = 0; q < RG; ++q) tot += vsum_s[q][c];
+    tot *= kBf16Unscale;  // exact
     const float mu = smooth ? (float)(tot / (double)valid) : 0.0f;
     if (rg == 0) v_mean[((size_t)bh * T + b) * D + c] = mu;
-    float vmax = 0.0f;
-    for (int r = rg; r < valid; r += RG) vmax = fmaxf(vmax, fabsf(__fsub_rn(bf2f(vsh[r * D + c]), mu)));
-    vmax_s[rg][c] = vmax;
+    float vm[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    r = rg;
+    for (; r + 3 * RG < valid; r += 4 * RG) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) vm[e] = fmaxf(vm[e], fabsf(__fsub_rn(bf2f(vsh[(r + e * RG) * D + c]), mu)));
+    }
+    for (; r < valid; r += RG) vm[0] = fmaxf(vm[0], fabsf(__fsub_rn(bf2f(vsh[r * D + c]), mu)));
+    vmax_s[rg][c] = fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3]));
     __syncthreads();
     if (rg == 0) {
         float m = vmax_s[0][c];
@@ -1587,41 +1683,53 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_v_quant_nvfp4(const __nv_bf
 }
 
 // Per-token Q: amax over d, inv = 448/amax, code = E4M3(q * inv), sq = amax/448.
+// Per-token E4M3 Q: amax over the d channels, inv = 448/amax, code = E4M3(q *
+// inv), scale = amax/448.  A token's row is read by D/8 lanes, 16 bytes each
+// (amax over those lanes by xor shuffles), and every lane has four rows' loads
+// in flight, so a warp covers 4 * 256/D tokens.
+constexpr int QQ_TOK_PER_CTA = 8 * 4;  // warps x loads in flight, times 256/D tokens a load
+
 template <int D>
 __global__ void __launch_bounds__(256) quant_q(const __nv_bfloat16* __restrict__ Q, uint8_t* __restrict__ q_fp8,
                                                float* __restrict__ sq, int64_t tokens) {
-    constexpr int PER = D / 32;  // values per lane
-    const int64_t tok = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (tok >= tokens) return;
-    float x[PER];
-    const __nv_bfloat16* src = Q + tok * D + lane * PER;
-    if constexpr (PER == 4) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(src);
-        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+    constexpr int LPT = D / 8;     // lanes per token
+    constexpr int TPW = 32 / LPT;  // tokens a warp covers per load
+    constexpr int U = 4;           // loads in flight per lane
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / LPT, part = lane % LPT;
+    const int64_t tok0 = ((int64_t)blockIdx.x * 8 + warp) * (TPW * U) + sub;
+    uint4 raw[U];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = bf2f(h[e]);
-    } else {
-        const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
-        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-        for (int e = 0; e < PER; ++e) x[e] = bf2f(h[e]);
+    for (int u = 0; u < U; ++u) {
+        const int64_t tok = tok0 + u * TPW;
+        raw[u] = tok < tokens ? __ldg(reinterpret_cast<const uint4*>(Q + tok * D) + part) : make_uint4(0, 0, 0, 0);
     }
-    float m = 0.0f;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) m = fmaxf(m, fabsf(x[e]));
+    for (int u = 0; u < U; ++u) {
+        const int64_t tok = tok0 + u * TPW;
+        const uint32_t wd[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+        float x[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float inv = m > 0.0f ? __fdiv_rn(448.0f, m) : 0.0f;
-    if constexpr (PER == 4) {
-        const uint32_t w = (uint32_t)e4m3x2(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv)) |
-                           ((uint32_t)e4m3x2(__fmul_rn(x[2], inv), __fmul_rn(x[3], inv)) << 16);
-        *reinterpret_cast<uint32_t*>(q_fp8 + tok * D + lane * 4) = w;
-    } else {
-        *reinterpret_cast<uint16_t*>(q_fp8 + tok * D + lane * 2) =
-            e4m3x2(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv));
+        for (int h = 0; h < 4; ++h) {
+            x[2 * h] = __uint_as_float(wd[h] << 16);
+            x[2 * h + 1] = __uint_as_float(wd[h] & 0xFFFF0000u);
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(x[e]));
+#pragma unroll
+        for (int o = LPT / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float inv = m > 0.0f ? __fdiv_rn(448.0f, m) : 0.0f;
+        uint32_t w[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            w[h] = (uint32_t)e4m3x2(__fmul_rn(x[4 * h], inv), __fmul_rn(x[4 * h + 1], inv)) |
+                   ((uint32_t)e4m3x2(__fmul_rn(x[4 * h + 2], inv), __fmul_rn(x[4 * h + 3], inv)) << 16);
+        if (tok < tokens) {
+            *reinterpret_cast<uint2*>(q_fp8 + tok * D + part * 8) = make_uint2(w[0], w[1]);
+            if (part == 0) sq[tok] = __fdiv_rn(m, 448.0f);
+        }
     }
-    if (lane == 0) sq[tok] = __fdiv_rn(m, 448.0f);
 }
 
 __global__ void e4m3_encode_kernel(const float* __restrict__ x, uint8_t* __restrict__ out, int64_t n) {
@@ -1693,7 +1801,8 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
                 km_pass<D, 3, false><<<grid, Move::kThreads, lm.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels,
                                                                            p.hist, p.sums, p.ties, regions, p.state,
                                                                            p.BH, p.N, p.C, Cp, it, mode, p.ctl);
-            km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, regions, grid, p.V, p.cent64, p.labels,
+            km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, regions, grid, p.c_hi, p.c_lo, p.cnorm,
+                                                  p.V, p.cent64, p.labels,
                                                   p.hist, p.sums, p.state, p.N, p.C, Cp, it, mode != 0,
                                                   p.ctl.status);
             if (mode != 0)  // the sums stay for a following pass that moves changed tokens only
@@ -1711,7 +1820,8 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
         km_assign<D><<<dim3(nchunk, p.BH), 128, smem, s>>>(tv, th, tl, p.cnorm, p.cent64, p.V, p.vnorm2, p.labels,
                                                             p.hist, p.ties, p.tie_count, p.state, p.N, p.C, Cp,
                                                             it, tpc, p.ctl);
-        km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, nullptr, 0, p.V, p.cent64, p.labels, p.hist,
+        km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, nullptr, 0, p.c_hi, p.c_lo, p.cnorm, p.V,
+                                              p.cent64, p.labels, p.hist,
                                               p.sums, p.state, p.N, p.C, Cp, it, 0, p.ctl.status);
         km_scan<<<p.BH, 1024, KM_SCAN_CHUNK * sizeof(int), s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N,
                                                                  p.C, nblk, it, 1, p.ctl.status);
@@ -1781,7 +1891,8 @@ cudaError_t launch_prep(const PrepLaunch& p, cudaStream_t s) {
 
 cudaError_t launch_quant_q(const __nv_bfloat16* Q, uint8_t* q_fp8, float* sq, int64_t tokens, int D,
                            cudaStream_t s) {
-    const unsigned grid = (unsigned)((tokens + 7) / 8);
+    const int64_t per_cta = QQ_TOK_PER_CTA * 256 / D;  // 32 tokens a CTA at d 128, 64 at d 64
+    const unsigned grid = (unsigned)((tokens + per_cta - 1) / per_cta);
     if (D == 128)
         quant_q<128><<<grid, 256, 0, s>>>(Q, q_fp8, sq, tokens);
     else

@@ -251,6 +251,18 @@ vc_status vc_check(void* workspace, void* stream);
  * +-448), the encoder every quantiser above uses.  x fp32 [n] -> out uint8 [n]. */
 vc_status vc_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream);
 
+/* Per-token E4M3 quantisation of Q, the first step of vc_attn_fwd (both
+ * operands of QK^T in FP8: chooseai.io news 7051, ExpCast-FP8 section).  For
+ * each token: amax over its d channels, q_fp8 = E4M3(q * (448 / amax)),
+ * sq = amax / 448 (0 and all-zero codes for an all-zero row).
+ *   Q      device, bf16 [tokens, d] row-major, 16-byte aligned
+ *   q_fp8  device, uint8 [tokens, d] out, 16-byte aligned
+ *   sq     device, fp32 [tokens] out, 4-byte aligned
+ *   d      64 or 128
+ * Asynchronous on `stream`.  VC_ERR_INVALID_ARG for null or misaligned
+ * pointers or tokens < 0, VC_ERR_UNSUPPORTED for another d. */
+vc_status vc_quantize_q(const void* Q, uint8_t* q_fp8, float* sq, int64_t tokens, int d, void* stream);
+
 /* Element-wise ExpCast byte map used inside vc_attn_fwd:
  * out[i] = max(0, round_half_even(A[i] * s[i] + cb[i])), one fp32 FMA with the
  * rounding inside it.  cb must hold integers with |cb| < 2^22.

@@ -58,3 +58,34 @@ def test_expcast_bit_exact(vc):
     ref = oracle.expcast_bytes(A, s, cb)
     bad = np.nonzero(got != ref)[0]
     assert bad.size == 0, (A[bad[:8]], s[bad[:8]], cb[bad[:8]], got[bad[:8]], ref[bad[:8]])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("tokens", [1, 31, 1000, 70001])
+def test_quantize_q_bit_exact(vc, d, tokens):
+    """The attention call's per-token Q quantiser against the oracle's: codes
+    and scales bit-exact, on rows of mixed scale (lognormal), all-zero rows,
+    rows of one nonzero channel, tiny (1e-30) and huge (1e30) rows, and rows
+    of subnormal values beside one normal value, at token counts that leave a
+    ragged last CTA.  (Rows whose amax is so small that 448/amax overflows are
+    left out: both sides then encode 0 * inf, a NaN.)"""
+    rng = np.random.default_rng(7 + d + tokens)
+    q = (rng.standard_normal((tokens, d)) * np.exp(rng.normal(0.0, 2.0, (tokens, 1)))).astype(np.float32)
+    q[::17] = 0.0
+    q[5::23] = 0.0
+    q[5::23, 3 % d] = -2.5
+    q[7::29] *= 1e-30
+    q[11::31] *= 1e30
+    q[13::37] = 1e-39 * np.sign(q[13::37])
+    q[13::37, 0] = 1.0
+    bits = (torch.from_numpy(q).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16))
+    codes, scales = vc.quantize_q(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda())
+    ref_codes, ref_scales = oracle.quant_q(bits)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_scales.view(np.uint32))
+
+
+def test_quantize_q_rejects_bad_arguments(vc):
+    q = torch.zeros(4, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(RuntimeError, match="vc_quantize_q"):
+        vc.quantize_q(q)
