@@ -391,9 +391,9 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
 //               v . c_hi + v . c_lo in TMEM), ties to the lowest k, near ties
 //               listed for km_refine, the tile's cluster histogram, and the
 //               tile's tokens grouped by cluster (a counting sort);
-//   update      the member sums from the same V tile in shared memory: update
-//               warp u owns clusters 8u .. 8u + 7, whose tokens are one
-//               contiguous block of the grouped tile; it walks the block four
+//   update      the member sums from the same V tile in shared memory: each
+//               update warp owns a contiguous range of clusters, whose tokens
+//               are one contiguous block of the grouped tile; it walks the block four
 //               tokens at a time, adds each run of a cluster in registers and
 //               the run's sum to the CTA's fp64 sums in shared memory; those go
 //               to the head's global sums
@@ -403,7 +403,10 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
 //               oracle's sequential ones.  Loops stay short: with four warp
 //               roles in one CTA, long unrolled code stalls on instruction
 //               fetch.
-// `mode` 1 is that full accumulation (the sums start from zero).  Mode 2 keeps
+// `mode` 1 is that full accumulation (the sums start from zero).  Mode 3 keeps
+// the sums and has the update warps move only the tokens whose label changed:
+// the tile's changed tokens grouped by new cluster are added, grouped by old
+// cluster subtracted (for pass 1, where most labels still hold).  Mode 2 keeps
 // the sums of the previous pass and moves only the tokens whose label changed
 // (the assignment warps subtract the row from the old cluster's global sums
 // and add it to the new one's, fp64 atomics): exact like a fresh sum, and
@@ -412,17 +415,20 @@ __global__ void __launch_bounds__(128, 3) km_assign(const __grid_constant__ CUte
 // Warps: 0 TMA producer (V tiles through a ring of stages; a head's centroids
 // when the CTA enters it), 1 MMA issuer (tile i into TMEM accumulator
 // i % kAcc), then G assignment groups of four warps (group g takes the CTA's
-// tiles i = g mod G; a thread per token), then, in the shape that sums every
-// token, 8 update warps (D/32 channels a lane).  Passes that move changed
-// tokens only run three assignment groups and no update warps.
+// tiles i = g mod G; a thread per token), then U update warps (D/32 channels a
+// lane; warp u owns clusters (64/U)u onwards).  Shapes: passes 0 and 1 (sum
+// every token; move a seventh of them) 1 group and 8 update warps (2 groups
+// and 4 measured slower for pass 1); later passes (move a few per mille by
+// atomics) 3 groups and none.
 constexpr int KP_SEG = 68;  // per stage: 65 cluster offsets, padded
 constexpr int KP_MAX_GRID = kKmTieRegions;  // near-tie regions the workspace holds
 
-template <int G, bool UPD>
+template <int G, int U>
 struct KpShape {
     static constexpr int kGroups = G;
-    static constexpr int kUpd = UPD ? 8 : 0;  // update warps
-    static constexpr int kStages = UPD ? 3 : 4;
+    static constexpr int kUpd = U;                  // update warps
+    static constexpr int kCpw = U > 0 ? 64 / U : 0;  // clusters a update warp owns
+    static constexpr int kStages = U > 0 ? 3 : 4;
     static constexpr int kAcc = G < 2 ? 2 : G;  // TMEM accumulators
     static constexpr int kThreads = 32 * (2 + 4 * G + kUpd);
 };
@@ -432,8 +438,8 @@ struct KpShape {
 //   tile order and its labels per stage | cluster offsets per stage | label
 //   counts per group x2 | scratch | barriers
 struct KpLayout {
-    uint32_t v_bytes, c_bytes, off_v, off_chi, off_clo, off_sum, off_cn, off_ord, off_slab, off_seg, off_cnt, off_misc,
-        off_bar, bytes;
+    uint32_t v_bytes, c_bytes, off_v, off_chi, off_clo, off_sum, off_cn, off_ord, off_slab, off_seg, off_ord2,
+        off_slab2, off_seg2, off_cnt, off_misc, off_bar, bytes;
     __host__ __device__ KpLayout(int D, int Cp, int S, int G, int nacc, bool with_sums) {
         v_bytes = KM_TOK * D * 2;
         c_bytes = Cp * D * 2;
@@ -445,8 +451,11 @@ struct KpLayout {
         off_ord = off_cn + ((G * 65 * 4 + 15) & ~15);     // [stage][128] tile rows grouped by cluster
         off_slab = off_ord + S * KM_TOK;                  // [stage][128] their clusters
         off_seg = off_slab + S * KM_TOK;                  // [stage][KP_SEG] first grouped position of each cluster
-        off_cnt = off_seg + S * KP_SEG * 4;               // [G][2][64] label counts of a group's tile
-        off_misc = off_cnt + G * 2 * 64 * 4;              // [16] ints, see km_pass
+        off_ord2 = off_seg + S * KP_SEG * 4;              // the same for the subtract list of mode 3
+        off_slab2 = off_ord2 + S * KM_TOK;
+        off_seg2 = off_slab2 + S * KM_TOK;
+        off_cnt = off_seg2 + S * KP_SEG * 4;              // [G][2][3][64] label counts of a group's tile
+        off_misc = off_cnt + G * 2 * 3 * 64 * 4;          // [16] ints, see km_pass
         off_bar = off_misc + 64;
         bytes = off_bar + 8 * (3 * S + 2 * nacc + 3) + 1024;  // + alignment slack
     }
@@ -495,16 +504,18 @@ __device__ __forceinline__ double bf16lo_scaled(uint32_t w) {  // bits 0..15 of 
     return bf16hi_scaled(w << 16);
 }
 
-template <int D, int G, bool UPD>
-__global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
+template <int D, int G, int U>
+__global__ void __launch_bounds__(KpShape<G, U>::kThreads, 1)
     km_pass(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_chi,
             const __grid_constant__ CUtensorMap tm_clo, const float* __restrict__ cnorm, float* __restrict__ vnorm2,
             int32_t* __restrict__ labels, int32_t* __restrict__ hist, double* __restrict__ sums,
             KmTie* __restrict__ ties, int* __restrict__ tie_regions, KmState* __restrict__ state, int BH, int N,
             int C, int Cp, int it, int mode, DevCtl ctl) {
-    using Shape = KpShape<G, UPD>;
+    using Shape = KpShape<G, U>;
+    constexpr bool UPD = U > 0;
+    constexpr int CPW = Shape::kCpw;
     constexpr int S = Shape::kStages, NACC = Shape::kAcc, ASG = 4 * G;
-    const bool accumulate = UPD && mode == 1;
+    const bool accumulate = UPD && (mode == 1 || mode == 3);
     if (ctl_failed(ctl.status)) return;
     const int nblk = (N + KM_TOK - 1) / KM_TOK;
     extern __shared__ uint8_t smem_raw[];
@@ -544,7 +555,7 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
         *tie_s = 0;
         fence_mbar_init();
     }
-    for (int i = tid; i < G * 2 * 64; i += blockDim.x) cnt_s[i] = 0;
+    for (int i = tid; i < G * 2 * 3 * 64; i += blockDim.x) cnt_s[i] = 0;
     double* sums_s = reinterpret_cast<double*>(smem + L.off_sum);
     if (accumulate)
         for (int i = tid; i < 64 * D; i += blockDim.x) sums_s[i] = 0.0;
@@ -672,6 +683,9 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
         uint8_t* ord_s = smem + L.off_ord;
         uint8_t* slab_s = smem + L.off_slab;
         int* seg_s = reinterpret_cast<int*>(smem + L.off_seg);
+        uint8_t* ord2_s = smem + L.off_ord2;
+        uint8_t* slab2_s = smem + L.off_slab2;
+        int* seg2_s = reinterpret_cast<int*>(smem + L.off_seg2);
         const int tie_base = misc[8];
         KpWalk w = start;
         for (int q = 0; q < g; ++q) w.next(state, BH, nblk);
@@ -723,12 +737,16 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
             for (int q = 0; q < G; ++q) w.next(state, BH, nblk);  // this group's next tile
             if (i + G < nunits) fetch(w);
             const int st = i % S, b = i % NACC;
-            int* cnt = cnt_s + (g * 2 + ((i / G) & 1)) * 64;  // this tile's label counts
+            // this tile's label counts: all valid tokens, the add list, the subtract list
+            int* cnt = cnt_s + (g * 2 + ((i / G) & 1)) * 3 * 64;
+            int* cnt_add = cnt + 64;
+            int* cnt_sub = cnt + 128;
             const int n = tile * KM_TOK + r;
             const bool valid = n < N;
             // the accumulator of tile i (its MMA also means V tile i has landed)
             const bool okj = warp_wait(b_accfull(b), (i / NACC) & 1, ctl, abort_flag);
-            int label = 0, rank = 0;
+            int label = 0, rank = 0, rank_sub = 0;
+            bool in_add = false, in_sub = false;
             if (okj) {
                 tc_fence_after();
                 const uint32_t lane_tmem = tmem + b * Cp + ((uint32_t)(qd * 32) << 16);
@@ -819,7 +837,12 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
                     label = bestk;
                     if (it == 0 || old_label != label) ++changed;
                     labels[(size_t)bh * N + n] = label;
-                    rank = atomicAdd(&cnt[label], 1);  // the token's place among its cluster's in this tile
+                    // the token's place among its cluster's in this tile's lists
+                    in_add = mode == 1 || (mode == 3 && old_label != label);
+                    in_sub = mode == 3 && old_label != label;
+                    if (in_add) rank = atomicAdd(&cnt_add[label], 1);
+                    if (in_sub) rank_sub = atomicAdd(&cnt_sub[old_label], 1);
+                    if (mode != 1) atomicAdd(&cnt[label], 1);  // mode 1: the add list is the histogram
                 }
                 if (mode == 2) {  // move the tokens that changed cluster, a row at a time over the warp
                     constexpr int NCH = D / 32;
@@ -852,31 +875,47 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
             // one decision for the four warps: leave together or go on together
             if (!named_barrier_and(bar_id, 128, okj)) break;
             int* seg = seg_s + st * KP_SEG;
+            int* seg2 = seg2_s + st * KP_SEG;
             if (qd == 0) {  // the tile's histogram, to global; cluster offsets for the grouping
                 const int k0 = 2 * lane;
-                const int h0 = cnt[k0], h1 = cnt[k0 + 1];
-                cnt[k0] = 0;  // ready for this group's tile after next
-                cnt[k0 + 1] = 0;
-                if (k0 < C) hist[((size_t)bh * C + k0) * nblk + tile] = h0;
-                if (k0 + 1 < C) hist[((size_t)bh * C + k0 + 1) * nblk + tile] = h1;
-                if (accumulate) {
-                    int x = h0 + h1;
+                // counts of clusters k0, k0 + 1 in one list, zeroed for this group's tile after next;
+                // with `seg`, that list's exclusive scan over the clusters
+                auto take = [&](int* cn, int* sg) {
+                    const int h0 = cn[k0], h1 = cn[k0 + 1];
+                    cn[k0] = 0;
+                    cn[k0 + 1] = 0;
+                    if (sg) {
+                        int x = h0 + h1;
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int y = __shfl_up_sync(0xffffffffu, x, o);
-                        if (lane >= o) x += y;
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int y = __shfl_up_sync(0xffffffffu, x, o);
+                            if (lane >= o) x += y;
+                        }
+                        sg[k0] = x - h0 - h1;
+                        sg[k0 + 1] = x - h1;
+                        if (lane == 31) sg[64] = x;
                     }
-                    seg[k0] = x - h0 - h1;
-                    seg[k0 + 1] = x - h1;
-                    if (lane == 31) seg[64] = x;
+                    return make_int2(h0, h1);
+                };
+                const int2 h = mode == 1 ? take(cnt_add, seg) : take(cnt, nullptr);
+                if (mode == 3) {
+                    take(cnt_add, seg);
+                    take(cnt_sub, seg2);
                 }
+                if (k0 < C) hist[((size_t)bh * C + k0) * nblk + tile] = h.x;
+                if (k0 + 1 < C) hist[((size_t)bh * C + k0 + 1) * nblk + tile] = h.y;
             }
             if (accumulate) {
                 named_barrier_sync(bar_id, 128);
-                if (valid) {
+                if (in_add) {
                     const int pos = st * KM_TOK + seg[label] + rank;
                     ord_s[pos] = (uint8_t)r;
                     slab_s[pos] = (uint8_t)label;
+                }
+                if (in_sub) {
+                    const int pos = st * KM_TOK + seg2[old_label] + rank_sub;
+                    ord2_s[pos] = (uint8_t)r;
+                    slab2_s[pos] = (uint8_t)old_label;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(b_lfull(st));  // the tile's grouping, for the update warps
@@ -886,17 +925,14 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
         }
         if (cur >= 0) flush_changed();
     } else if (UPD && accumulate && nunits > 0) {
-        // ------------------------------------------------------------ update, mode 1 (D/32 channels a lane)
+        // ------------------------------------------------------------ update, modes 1 and 3 (D/32 channels a lane)
         constexpr int NCH = D / 32;
-        const int u = warp - 2 - ASG;           // clusters 8u .. 8u + 7
+        const int u = warp - 2 - ASG;           // clusters CPW u .. CPW u + CPW - 1
         const int c0 = NCH * lane;              // channels c0 .. c0 + NCH - 1
         const int kc = c0 >> 6, q16 = (c0 & 63) >> 3, wo = (c0 & 7) * 2;  // chunk, 16-byte piece, byte
-        const uint8_t* ord_s = smem + L.off_ord;
-        const uint8_t* slab_s = smem + L.off_slab;
-        const int* seg_s = reinterpret_cast<const int*>(smem + L.off_seg);
         auto flush = [&](int bh) {  // this warp's sums of head bh to the global sums, then zero
 #pragma unroll 1
-            for (int k = 8 * u; k < 8 * u + 8 && k < C; ++k) {
+            for (int k = CPW * u; k < CPW * u + CPW && k < C; ++k) {
 #pragma unroll
                 for (int e = 0; e < NCH; ++e) {
                     double* sp = sums_s + k * D + c0 + e;
@@ -916,60 +952,67 @@ __global__ void __launch_bounds__(KpShape<G, UPD>::kThreads, 1)
             const int st = i % S;
             // the update trails the assignment by a tile: wait without polling hard
             if (!(ok = warp_wait_idle(b_lfull(st), (i / S) & 1, ctl, abort_flag, 100))) break;
-            const uint8_t* ord = ord_s + st * KM_TOK;
-            const uint8_t* slab = slab_s + st * KM_TOK;
             const uint8_t* vt = smem + L.off_v + st * L.v_bytes + kc * (KM_TOK * 128) + wo;
-            // clusters 8u .. 8u + 7 hold grouped positions [P0, P1)
-            const int P0 = seg_s[st * KP_SEG + 8 * u], P1 = seg_s[st * KP_SEG + 8 * u + 8];
-            double run[NCH];
+            // One grouped list of the tile: the warp's clusters hold its
+            // positions [P0, P1); each run is added to (or subtracted from)
+            // the CTA's sums.
+            auto walk = [&](uint32_t off_ord, uint32_t off_slab, uint32_t off_seg, bool subtract) {
+                const uint8_t* ord = smem + off_ord + st * KM_TOK;
+                const uint8_t* slab = smem + off_slab + st * KM_TOK;
+                const int* segp = reinterpret_cast<const int*>(smem + off_seg) + st * KP_SEG + CPW * u;
+                const int P0 = segp[0], P1 = segp[CPW];
+                double run[NCH];
 #pragma unroll
-            for (int e = 0; e < NCH; ++e) run[e] = 0.0;
-            int rk = P0 < P1 ? slab[P0] : 0;  // cluster of the run being added
-            auto flush_run = [&]() {
-                double* sp = sums_s + rk * D + c0;
+                for (int e = 0; e < NCH; ++e) run[e] = 0.0;
+                int rk = P0 < P1 ? slab[P0] : 0;  // cluster of the run being added
+                auto flush_run = [&]() {
+                    double* sp = sums_s + rk * D + c0;
 #pragma unroll
-                for (int e = 0; e < NCH; ++e) {
-                    sp[e] += run[e];
-                    run[e] = 0.0;
-                }
-            };
+                    for (int e = 0; e < NCH; ++e) {
+                        sp[e] = subtract ? sp[e] - run[e] : sp[e] + run[e];
+                        run[e] = 0.0;
+                    }
+                };
 #pragma unroll 1
-            for (int p = P0; p < P1; p += 4) {
-                // four positions' rows and clusters first, so their loads overlap
-                int j[4], kk[4];
+                for (int p = P0; p < P1; p += 4) {
+                    // four positions' rows and clusters first, so their loads overlap
+                    int j[4], kk[4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int pp = min(p + t, P1 - 1);
-                    j[t] = ord[pp];
-                    kk[t] = p + t < P1 ? (int)slab[pp] : -1;
-                }
-                uint32_t x[4][NCH / 2];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const uint8_t* src = vt + j[t] * 128 + ((q16 ^ (j[t] & 7)) << 4);  // row j, 128-byte swizzle
-                    if constexpr (NCH == 4) {
-                        const uint2 y = *reinterpret_cast<const uint2*>(src);
-                        x[t][0] = y.x;
-                        x[t][1] = y.y;
-                    } else {
-                        x[t][0] = *reinterpret_cast<const uint32_t*>(src);
+                    for (int t = 0; t < 4; ++t) {
+                        const int pp = min(p + t, P1 - 1);
+                        j[t] = ord[pp];
+                        kk[t] = p + t < P1 ? (int)slab[pp] : -1;
                     }
-                }
+                    uint32_t x[4][NCH / 2];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    if (kk[t] < 0) break;
-                    if (kk[t] != rk) {  // a new cluster's run starts (uniform over the warp)
-                        flush_run();
-                        rk = kk[t];
+                    for (int t = 0; t < 4; ++t) {
+                        const uint8_t* src = vt + j[t] * 128 + ((q16 ^ (j[t] & 7)) << 4);  // row j, 128-byte swizzle
+                        if constexpr (NCH == 4) {
+                            const uint2 y = *reinterpret_cast<const uint2*>(src);
+                            x[t][0] = y.x;
+                            x[t][1] = y.y;
+                        } else {
+                            x[t][0] = *reinterpret_cast<const uint32_t*>(src);
+                        }
                     }
 #pragma unroll
-                    for (int h = 0; h < NCH / 2; ++h) {
-                        run[2 * h] += bf16lo_scaled(x[t][h]);
-                        run[2 * h + 1] += bf16hi_scaled(x[t][h]);
+                    for (int t = 0; t < 4; ++t) {
+                        if (kk[t] < 0) break;
+                        if (kk[t] != rk) {  // a new cluster's run starts (uniform over the warp)
+                            flush_run();
+                            rk = kk[t];
+                        }
+#pragma unroll
+                        for (int h = 0; h < NCH / 2; ++h) {
+                            run[2 * h] += bf16lo_scaled(x[t][h]);
+                            run[2 * h + 1] += bf16hi_scaled(x[t][h]);
+                        }
                     }
                 }
-            }
-            if (P0 < P1) flush_run();
+                if (P0 < P1) flush_run();
+            };
+            walk(L.off_ord, L.off_slab, L.off_seg, false);
+            if (mode == 3) walk(L.off_ord2, L.off_slab2, L.off_seg2, true);
             __syncwarp();
             if (lane == 0) mbar_arrive(b_vempty(st));
         }
@@ -1766,9 +1809,9 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     if (!configured.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(km_assign<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(km_pass<D, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(km_pass<D, 1, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(km_pass<D, 3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(km_pass<D, 3, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(km_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, KM_SCAN_CHUNK * sizeof(int));
         if (e != cudaSuccess) return e;
@@ -1784,30 +1827,31 @@ static cudaError_t kmeans_t(const PrepLaunch& p, cudaStream_t s) {
     if (p.C <= 64) {
         // One fused pass a sweep (the member sums fit in shared memory); the
         // regroup is built once, from the last labels.
-        using Sum = KpShape<1, true>;   // passes that sum every token
-        using Move = KpShape<3, false>;  // passes that move changed tokens, and the last
+        using Sum = KpShape<1, 8>;   // passes 0 and 1: the update warps sum every token, then move the changed ones
+        using Move = KpShape<3, 0>;  // later passes: atomics move the few changed tokens; the last pass
         const KpLayout ls(D, Cp, Sum::kStages, 1, Sum::kAcc, true), lm(D, Cp, Move::kStages, 3, Move::kAcc, false);
         const int grid = sms < KP_MAX_GRID ? sms : KP_MAX_GRID;
         int* regions = p.tie_count + 2;
         for (int it = 0; it < p.iters; ++it) {
-            // the first two passes add every token (most labels still move);
-            // later ones move the few tokens that change; the last needs no sums
-            const int mode = it + 1 == p.iters ? 0 : (it < 2 ? 1 : 2);
-            if (mode == 1)
-                km_pass<D, 1, true><<<grid, Sum::kThreads, ls.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels,
-                                                                         p.hist, p.sums, p.ties, regions, p.state,
-                                                                         p.BH, p.N, p.C, Cp, it, mode, p.ctl);
+            // pass 0 adds every token; pass 1 moves the tokens that change
+            // (about a seventh of them) through the update warps, later passes
+            // (a few per mille) with atomics; the last needs no sums
+            const int mode = it + 1 == p.iters ? 0 : (it == 0 ? 1 : (it == 1 ? 3 : 2));
+            if (mode == 1 || mode == 3)
+                km_pass<D, 1, 8><<<grid, Sum::kThreads, ls.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels,
+                                                                      p.hist, p.sums, p.ties, regions, p.state, p.BH,
+                                                                      p.N, p.C, Cp, it, mode, p.ctl);
             else
-                km_pass<D, 3, false><<<grid, Move::kThreads, lm.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels,
-                                                                           p.hist, p.sums, p.ties, regions, p.state,
-                                                                           p.BH, p.N, p.C, Cp, it, mode, p.ctl);
+                km_pass<D, 3, 0><<<grid, Move::kThreads, lm.bytes, s>>>(tv, th, tl, p.cnorm, p.vnorm2, p.labels,
+                                                                       p.hist, p.sums, p.ties, regions, p.state, p.BH,
+                                                                       p.N, p.C, Cp, it, mode, p.ctl);
             km_refine<D><<<sms * 8, 256, 0, s>>>(p.ties, p.tie_count, regions, grid, p.c_hi, p.c_lo, p.cnorm,
                                                   p.V, p.cent64, p.labels,
                                                   p.hist, p.sums, p.state, p.N, p.C, Cp, it, mode != 0,
                                                   p.ctl.status);
-            if (mode != 0)  // the sums stay for a following pass that moves changed tokens only
+            if (mode != 0)  // the sums stay: every later pass moves changed tokens only
                 km_finalize<<<dim3(p.C, p.BH), D, 0, s>>>(p.c_hi, p.c_lo, p.cnorm, p.cent64, p.sums, p.ccount,
-                                                          p.hist, p.state, p.C, Cp, D, nblk, it, 1, it + 1 >= 2,
+                                                          p.hist, p.state, p.C, Cp, D, nblk, it, 1, 1,
                                                           p.ctl.status);
         }
         km_scan<<<p.BH, 1024, KM_SCAN_CHUNK * sizeof(int), s>>>(p.hist, p.offs, p.cstart, p.ccount, p.state, p.N,
