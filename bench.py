@@ -65,11 +65,13 @@ def kernel_code_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def attn_traffic_bytes(heads: int, kernel: str = "vc_attn_kernel"):
+def attn_traffic_bytes(heads: int, kernel: str = "vc_attn_kernel", N=None, d=None, block=None):
     """DRAM bytes (read + write) of one attention-kernel launch over `heads`
     heads, from the ncu capture recorded in profiles/attn_traffic.json; None
-    when there is no record for the kernel or its code has changed since the
-    capture (the counters no longer apply)."""
+    when there is no record for the kernel, its code has changed since the
+    capture (the counters no longer apply), or the record names the shape it
+    was captured on (N, d, block) and the launch's shape differs (the bytes a
+    head grow with N)."""
     try:
         with open(os.path.join(ROOT, "profiles", "attn_traffic.json")) as f:
             rec = json.load(f).get(kernel)
@@ -78,6 +80,9 @@ def attn_traffic_bytes(heads: int, kernel: str = "vc_attn_kernel"):
         return None
     if not rec or rec.get("sources_sha256_16") != code:
         return None
+    for key, val in (("N", N), ("d", d), ("block", block)):
+        if key in rec and val is not None and int(rec[key]) != int(val):
+            return None
     return int(rec["dram_bytes_per_head"]) * heads
 
 
@@ -288,12 +293,17 @@ def prep_roofline(w, prep_ms: float, peaks, timed_s: float) -> dict:
 
 def launches_per_step(p) -> int:
     """Kernels of the library one step launches (the launch list in profiles/
-    shows the same sequence): km_init; per k-means pass km_assign, km_refine,
-    km_scan, km_scatter; between passes km_update, km_finalize; then
-    prep_kv_block, prep_v_quant, quant_q and the attention kernel.  V-Smooth
-    off (smooth 0): identity_order, prep_kv_block, prep_v_quant (plus a
-    memset).  A kept regroup (smooth 2): prep_kv_block and prep_v_quant."""
-    if p.smooth == 1:
+    shows the same sequence).  V-Smooth with C <= 64: km_init; per k-means
+    pass km_pass and km_refine; between passes km_finalize; after the last,
+    km_scan and km_scatter.  With C > 64: km_init; per pass km_assign,
+    km_refine, km_scan, km_scatter; between passes km_update, km_finalize.
+    Then prep_kv_block and prep_v_quant.  V-Smooth off (smooth 0):
+    identity_order, prep_kv_block, prep_v_quant (plus a memset).  A kept
+    regroup (smooth 2): prep_kv_block and prep_v_quant.  Every step then
+    launches quant_q and the attention kernel."""
+    if p.smooth == 1 and p.C <= 64:
+        prep = 1 + 2 * p.iters + (p.iters - 1) + 2 + 2
+    elif p.smooth == 1:
         prep = 1 + 4 * p.iters + 2 * (p.iters - 1) + 2
     else:
         prep = 3 if p.smooth == 0 else 2
@@ -481,8 +491,8 @@ def run_ours(args, w):
                 "peak_source": peak_src, "timed_region_s": timed_s,
                 "frac_of_nominal": attn_tflops / nominal, "nominal_peak": nominal,
                 "traffic": None if tile_mask is not None else attn_traffic_bytes(
-                    w.B * w.H, "vc_attn4_kernel" if four_bit else "vc_attn_kernel"),
-                "traffic_unit": "DRAM bytes per launch (ncu capture on fewer heads, scaled by heads)",
+                    w.B * w.H, "vc_attn4_kernel" if four_bit else "vc_attn_kernel", w.N, w.d, w.block),
+                "traffic_unit": "DRAM bytes per launch (ncu capture on fewer heads of the same shape, scaled by heads)",
             },
             "accuracy": acc,
             "e2e": {"value": dense_job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,

@@ -18,10 +18,17 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.mark.parametrize("iters", [1, 2, 10])
 def test_launches_per_step_by_mode(iters):
-    base = vc.Params(C=16, iters=iters, block=128)
-    # k-means: init, 4 per pass, 2 between passes, then K/V block quantisation
-    assert bench.launches_per_step(base) == 1 + 4 * iters + 2 * (iters - 1) + 2 + 2
     import dataclasses
+
+    base = vc.Params(C=16, iters=iters, block=128)
+    # C <= 64, the fused pass: init, km_pass and km_refine a pass, km_finalize
+    # between passes, scan and scatter once, then K/V block quantisation
+    assert bench.launches_per_step(base) == 1 + 2 * iters + (iters - 1) + 2 + 2 + 2
+    assert bench.launches_per_step(dataclasses.replace(base, C=64)) == bench.launches_per_step(base)
+    # C > 64: init, 4 a pass (assign, refine, scan, scatter), update and
+    # finalize between passes, then K/V block quantisation
+    big = dataclasses.replace(base, C=256)
+    assert bench.launches_per_step(big) == 1 + 4 * iters + 2 * (iters - 1) + 2 + 2
 
     assert bench.launches_per_step(dataclasses.replace(base, smooth=0)) == 3 + 2
     assert bench.launches_per_step(dataclasses.replace(base, smooth=2)) == 2 + 2
@@ -71,6 +78,18 @@ def test_traffic_without_a_profile_is_null(tmp_path, monkeypatch):
     _write_profile(tmp_path, bench.kernel_code_hash(), 99, kernel="vc_attn4_kernel")
     assert bench.attn_traffic_bytes(40) is None
     assert bench.attn_traffic_bytes(40, "vc_attn4_kernel") == 99 * 40
+
+
+def test_traffic_applies_only_to_the_captured_shape(tmp_path, monkeypatch):
+    _fake_root(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles" / "attn_traffic.json").write_text(json.dumps({"vc_attn_kernel": {
+        "sources_sha256_16": bench.kernel_code_hash(), "dram_bytes_per_head": 77, "N": 32768, "d": 128,
+        "block": 128}}))
+    assert bench.attn_traffic_bytes(40, "vc_attn_kernel", 32768, 128, 128) == 77 * 40
+    assert bench.attn_traffic_bytes(40, "vc_attn_kernel", 75600, 128, 128) is None
+    assert bench.attn_traffic_bytes(2, "vc_attn_kernel", 32768, 64, 128) is None
+    assert bench.attn_traffic_bytes(40, "vc_attn_kernel", 32768, 128, 64) is None
 
 
 def test_committed_traffic_records_are_well_formed():
