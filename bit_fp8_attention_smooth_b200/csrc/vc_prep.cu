@@ -8,15 +8,20 @@
 //
 // Kernels, per call, for all (b, h) at once:
 //   km_init                   strided centroid init c_k = v[floor(k N / C)]
-//   per pass: km_assign       labels = argmin_k |c_k|^2 - 2 v.c_k on tensor cores (ties ->
-//                             lowest k), per-(cluster, 128-token block) histogram, change
-//                             count; near ties listed for km_refine
-//             km_refine       fp64 decision of the near ties; fixes labels and counts
-//             km_scan         exclusive scan -> stable positions; a head whose labels
+//   C <= 64, per pass:
+//     km_pass                 one persistent launch: labels = argmin_k |c_k|^2 - 2 v.c_k on
+//                             tensor cores (ties -> lowest k), per-(cluster, 128-token tile)
+//                             histogram, change count, near ties listed per CTA; the fp64
+//                             member sums from the same V tile (pass 0: every token; later:
+//                             the tokens whose label changed, moved between sums)
+//     km_refine               the near ties decided exactly (fp32 bounds, else fp64); fixes
+//                             labels, counts and sums
+//     km_finalize             c_k = sum / count (empty clusters keep c_k); a head whose labels
 //                             did not change is final (its later passes would repeat)
-//             km_scatter      perm[position] = token (stable within a cluster)
-//             km_update       fp64 member sums over fixed slices of the stable order
-//             km_finalize     c_k = sum / count (empty clusters keep c_k)
+//   then once: km_scan, km_scatter (the stable regroup from the last labels)
+//   C > 64, per pass: km_assign (the assignment alone), km_refine, km_scan (the head's
+//     final check), km_scatter, km_update (fp64 sums over slices of the stable order),
+//     km_finalize
 //   identity_order            V-Smooth off (smooth 0): perm = identity, labels 0, no k-means
 //   (smooth 2 runs no k-means kernel and keeps the perm already in the prep buffers)
 //   prep_kv_block             per block: K amax scale + E4M3 K, V block mean (fp64 sum),
