@@ -30,7 +30,8 @@ def libpath():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("vc_smooth_prepare", "vc_attn_fwd", "vc_attention", "vc_workspace_bytes", "vc_prep_buffer_bytes",
-              "vc_check", "vc_status_string", "vc_abi_version", "vc_e4m3_encode", "vc_expcast_bytes"):
+              "vc_check", "vc_status_string", "vc_abi_version", "vc_e4m3_encode", "vc_expcast_bytes",
+              "vc_quantize_q"):
         assert n in names
 
 
@@ -103,6 +104,13 @@ def test_argument_checks_run_before_any_device_call(libpath):
     no_scales = vc._Prep(*([fake.value] * 7 + [None]))
     assert L.vc_attn_fwd(fake, ctypes.byref(no_scales), ctypes.byref(shape), ctypes.byref(p4.c()), fake, fake,
                          ctypes.c_size_t(1 << 40), None) == vc.VC_ERR_INVALID_ARG
+    # the per-token Q quantiser: d, the token count and alignment, before the device
+    assert L.vc_quantize_q(fake, fake, fake, 10, 96, None) == vc.VC_ERR_UNSUPPORTED
+    assert L.vc_quantize_q(fake, fake, fake, -1, 128, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_quantize_q(odd, fake, fake, 10, 128, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_quantize_q(fake, odd, fake, 10, 128, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_quantize_q(fake, fake, ctypes.c_void_p((1 << 20) + 2), 10, 128, None) == vc.VC_ERR_INVALID_ARG
+    assert L.vc_quantize_q(None, None, None, 0, 128, None) == vc.VC_OK  # nothing to do
 
 
 def test_product_path_fails_loudly_without_the_library(monkeypatch, tmp_path):
