@@ -1457,8 +1457,9 @@ __global__ void km_finalize(__nv_bfloat16* __restrict__ c_hi, __nv_bfloat16* __r
 
 // ------------------------------------------------------------------ block quantisation
 // One CTA per (block of BK regrouped tokens, head), 256 threads.  The block's
-// gathered K and V rows are read once, 16 bytes a thread, into shared memory;
-// every pass below works from there.  K: amax over the block, inv = 448/amax,
+// gathered K rows, then its V rows, are copied once, 16 bytes a piece with
+// every piece of a thread in flight, into one shared buffer; every pass below
+// works from there.  K: amax over the block, inv = 448/amax,
 // code = E4M3(k * inv), k_scale = amax/448.  V: block mean (fp64 sum / valid,
 // rounded to fp32; zero when smooth == 0), residual channel amax folded into
 // vamax with an integer max on the fp32 bits (all >= 0).
@@ -1468,9 +1469,11 @@ constexpr int PREP_THREADS = 256;
 // the caller (the reuse mode) can then never index outside the head.
 __device__ __forceinline__ int clamp_tok(int32_t t, int N) { return (uint32_t)t < (uint32_t)N ? t : 0; }
 
+// One buffer of a block's rows: first its K rows, then its V rows, so that
+// about six CTAs share an SM and some are always loading.
 template <int D, int BK>
 constexpr int kv_block_smem() {
-    return 2 * BK * D * 2;
+    return BK * D * 2;
 }
 
 template <int D, int BK>
@@ -1483,7 +1486,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat1
     constexpr int NT = PREP_THREADS;
     constexpr int RG = NT / D;  // row groups of the per-channel passes
     constexpr int CH = D / 8;   // 16-byte pieces per row
-    extern __shared__ uint4 kv_s[];  // K rows [BK][CH], then V rows [BK][CH]
+    extern __shared__ uint4 kv_s[];  // the block's K rows [BK][CH], later its V rows
     __shared__ int tok_s[BK];
     __shared__ uint32_t red_s[NT / 32];
     __shared__ double vsum_s[RG][D];
@@ -1494,20 +1497,22 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat1
     for (int r = tid; r < BK; r += NT) tok_s[r] = r < valid ? clamp_tok(perm[(size_t)bh * N + b * BK + r], N) : 0;
     __syncthreads();
     uint4* ks = kv_s;
-    uint4* vs = kv_s + BK * CH;
+    uint4* vs = kv_s;
     const uint4* kg = reinterpret_cast<const uint4*>(K + (size_t)bh * N * D);
     const uint4* vg = reinterpret_cast<const uint4*>(V + (size_t)bh * N * D);
-    uint32_t kmax_bits = 0;  // |k| >= 0: the fp32 bit order is the value order
 #pragma unroll
     for (int u = 0; u < BK * CH / NT; ++u) {
         const int i = tid + u * NT;
-        const int r = i / CH, q = i % CH;
-        if (r < valid) {
-            const size_t src = (size_t)tok_s[r] * CH + q;
-            const uint4 kx = __ldg(kg + src);
-            const uint4 vx = __ldg(vg + src);
-            ks[i] = kx;
-            vs[i] = vx;
+        const int r = i / CH;
+        if (r < valid) cp_async16(ks + i, kg + (size_t)tok_s[r] * CH + i % CH);
+    }
+    cp_async_wait_all();
+    uint32_t kmax_bits = 0;  // |k| >= 0: the fp32 bit order is the value order
+#pragma unroll
+    for (int u = 0; u < BK * CH / NT; ++u) {  // the thread's own pieces
+        const int i = tid + u * NT;
+        if (i / CH < valid) {
+            const uint4 kx = ks[i];
             const uint32_t w[4] = {kx.x, kx.y, kx.z, kx.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e)  // bf16 -> fp32 bits of |k|: the high half, sign cleared
@@ -1527,18 +1532,6 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat1
     const __nv_bfloat16* ksh = reinterpret_cast<const __nv_bfloat16*>(ks);
     const __nv_bfloat16* vsh = reinterpret_cast<const __nv_bfloat16*>(vs);
     const int c = tid % D, rg = tid / D;
-    // The channel's sum over the block in fp64, four partial sums of the
-    // bf16 values placed as v * 2^-896 (exact, see bf16lo_scaled); scaled
-    // back once below.  Exact additions make the order irrelevant.
-    const uint16_t* vbits = reinterpret_cast<const uint16_t*>(vs);
-    double vp[4] = {0.0, 0.0, 0.0, 0.0};
-    int r = rg;
-    for (; r + 3 * RG < valid; r += 4 * RG) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) vp[e] += bf16lo_scaled(vbits[(r + e * RG) * D + c]);
-    }
-    for (; r < valid; r += RG) vp[0] += bf16lo_scaled(vbits[r * D + c]);
-    vsum_s[rg][c] = (vp[0] + vp[1]) + (vp[2] + vp[3]);
     // K codes, four channels a thread (one 32-bit store); padding rows are 0
     uint32_t* kout = reinterpret_cast<uint32_t*>(k_fp8 + ((size_t)bh * T * BK + (size_t)b * BK) * D);
 #pragma unroll 4
@@ -1553,6 +1546,27 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kv_block(const __nv_bfloat1
         }
         kout[i] = w;
     }
+    __syncthreads();  // every K row read: the buffer takes the V rows
+#pragma unroll
+    for (int u = 0; u < BK * CH / NT; ++u) {
+        const int i = tid + u * NT;
+        const int r = i / CH;
+        if (r < valid) cp_async16(vs + i, vg + (size_t)tok_s[r] * CH + i % CH);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // The channel's sum over the block in fp64, four partial sums of the
+    // bf16 values placed as v * 2^-896 (exact, see bf16lo_scaled); scaled
+    // back once below.  Exact additions make the order irrelevant.
+    const uint16_t* vbits = reinterpret_cast<const uint16_t*>(vs);
+    double vp[4] = {0.0, 0.0, 0.0, 0.0};
+    int r = rg;
+    for (; r + 3 * RG < valid; r += 4 * RG) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) vp[e] += bf16lo_scaled(vbits[(r + e * RG) * D + c]);
+    }
+    for (; r < valid; r += RG) vp[0] += bf16lo_scaled(vbits[r * D + c]);
+    vsum_s[rg][c] = (vp[0] + vp[1]) + (vp[2] + vp[3]);
     __syncthreads();
     double tot = 0.0;
 #pragma unroll
@@ -1586,7 +1600,7 @@ __global__ void identity_order(int32_t* __restrict__ perm, int32_t* __restrict__
 }
 
 // E4M3 residual with per-channel scales, written transposed: vt[bh][c][token].
-// The block's gathered V rows are read once, 16 bytes a thread, into shared
+// The block's gathered V rows are copied once, 16 bytes a piece, into shared
 // memory; codes are built per channel and leave as 16-byte pieces of vt rows.
 template <int D, int BK>
 constexpr int v_quant_smem() {
@@ -1618,8 +1632,9 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_v_quant(const __nv_bfloat16
     for (int u = 0; u < BK * CH / NT; ++u) {
         const int i = tid + u * NT;
         const int r = i / CH;
-        if (r < valid) v_s[i] = __ldg(vg + (size_t)tok_s[r] * CH + i % CH);
+        if (r < valid) cp_async16(v_s + i, vg + (size_t)tok_s[r] * CH + i % CH);
     }
+    cp_async_wait_all();
     const int c = tid % D, rg = tid / D;
     const float amax = __uint_as_float(vamax[(size_t)bh * D + c]);
     const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
@@ -1683,8 +1698,9 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_v_quant_nvfp4(const __nv_bf
     for (int u = 0; u < BK * CH / NT; ++u) {
         const int i = tid + u * NT;
         const int r = i / CH;
-        if (r < valid) v_s[i] = __ldg(vg + (size_t)tok_s[r] * CH + i % CH);
+        if (r < valid) cp_async16(v_s + i, vg + (size_t)tok_s[r] * CH + i % CH);
     }
+    cp_async_wait_all();
     const int c = tid % D, rg = tid / D;
     const float amax = __uint_as_float(vamax[(size_t)bh * D + c]);
     const float inv = amax > 0.0f ? __fdiv_rn(2688.0f, amax) : 0.0f;
