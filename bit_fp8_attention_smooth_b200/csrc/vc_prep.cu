@@ -36,6 +36,18 @@
 namespace vc {
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// 16 bytes from global to shared memory without passing through registers
+// (both addresses 16-byte aligned), so a thread keeps all its pieces of a
+// gather in flight at once; cp_async_wait_all makes the thread's own copies
+// complete and visible to it (other threads need a barrier after).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 // ------------------------------------------------------------------ k-means
